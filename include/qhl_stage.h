@@ -1,0 +1,232 @@
+/*
+ * qhl_stage.h - C ABI of the quantized hybrid layer-stage library (B200, sm_100a).
+ *
+ * A "stage" is a contiguous range of decoder layers of a hybrid Gated-DeltaNet +
+ * attention model that a peer runs on the hidden state it is handed:
+ *   - Unstable Legion: the peer-to-peer ChatGPT, "Splitting the workload": the
+ *     model is cut into contiguous layer stages; each stage runs its own range
+ *     of layers and keeps its own attention cache.  "The runtime": run an
+ *     arbitrary range of layers with activations passed in and out.
+ *   - Peer-to-peer LLM inference in browser tabs, Qwen 3.8 27B (SwarmLLM
+ *     README): peers hold layers 0-21 / 22-42 / 43-63 of a 64-layer model with a
+ *     5,120-float hidden state, GGUF Q4_0 weights ("4-bit blocks with f16
+ *     scales"), prefill in 16-token batches, multi-token-prediction drafts
+ *     verified "in a single batched pass with exact rollback of the recurrent
+ *     state", and a speculative path equal to plain decoding.
+ *   - ChatTorrent README, "What it can run": Gated DeltaNet layers mixed with
+ *     full-attention layers that have partial RoPE, QK-norm and an output gate;
+ *     RMSNorm and SwiGLU blocks; weights f32, f16 or q8.
+ *
+ * Each layer: h += mixer(RMSNorm1(h)); h += W_down(silu(W_gate x) * (W_up x)),
+ * x = RMSNorm2(h).  Layer i is full attention iff i % attn_every == attn_every-1,
+ * else gated DeltaNet.
+ *
+ * Conventions for every call:
+ *   - All functions return a stage_status (0 = ok, negative = error); none
+ *     throws, none aborts.  On error the stage's observable state (committed
+ *     length, recurrent states, KV caches, pending pass) is unchanged and
+ *     stage_last_error() describes the failure.
+ *   - Device work is asynchronous and ordered on the CUDA stream given to
+ *     stage_load.  Device-side faults of the stage's own kernels (a bounded
+ *     wait that ran out) are reported by stage_sync().
+ *   - A stage is not thread-safe; use one stage from one host thread at a time.
+ */
+#ifndef QHL_STAGE_H
+#define QHL_STAGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct stage stage_t;
+
+typedef enum {
+  STAGE_OK = 0,
+  STAGE_E_ARG = -1,          /* null pointer, size or range out of bounds, unknown tensor name */
+  STAGE_E_STATE = -2,        /* call not allowed now: pending pass, pos != committed length, nothing pending */
+  STAGE_E_OOM = -3,          /* device memory allocation failed */
+  STAGE_E_CUDA = -4,         /* a CUDA runtime call failed (message in stage_last_error) */
+  STAGE_E_FORMAT = -5,       /* a required tensor is missing or has the wrong byte size */
+  STAGE_E_UNSUPPORTED = -6,  /* shape the kernels do not implement */
+  STAGE_E_DEVICE = -7        /* a stage kernel reported a device-side error (see stage_sync) */
+} stage_status;
+
+/* GGUF type ids of the supported block formats. */
+typedef enum { STAGE_Q4_0 = 2, STAGE_Q8_0 = 8 } stage_qtype;
+
+/* Model shape.  Supported: hidden, ffn multiples of 256; dn_dim == 128;
+ * dn_v_heads a multiple of dn_k_heads; att_dim == 256; rope_dims == 64;
+ * att_q_heads a multiple of att_kv_heads with att_q_heads/att_kv_heads <= 7;
+ * max_ctx >= 16.  The 27B hybrid: 5120, 17408, 16, 48, 128, 24, 4, 256, 64,
+ * 1e7, 1e-6, 4. */
+typedef struct {
+  int hidden;          /* H: width of the hidden state */
+  int ffn;             /* F: SwiGLU intermediate width */
+  int dn_k_heads;      /* DeltaNet key (and query) heads */
+  int dn_v_heads;      /* DeltaNet value heads (state heads) */
+  int dn_dim;          /* DeltaNet head dim (key and value) */
+  int att_q_heads;     /* attention query heads */
+  int att_kv_heads;    /* attention KV heads (GQA) */
+  int att_dim;         /* attention head dim */
+  int rope_dims;       /* leading head dims that RoPE rotates */
+  double rope_theta;   /* RoPE base */
+  float eps;           /* RMSNorm / QK-norm epsilon */
+  int attn_every;      /* layer i is attention iff i % attn_every == attn_every - 1 */
+  int max_ctx;         /* KV-cache rows per attention layer */
+  int qtype;           /* STAGE_Q4_0 or STAGE_Q8_0 */
+} stage_config;
+
+/* One host tensor handed to stage_load.  The library reads `data` only during
+ * the call (it is copied to the device and repacked); the caller keeps
+ * ownership.  Names and contents, for each layer L of the range:
+ *   "blk.L.norm1", "blk.L.norm2"            f32 [H]   RMSNorm weights
+ *   DeltaNet layers:
+ *     "blk.L.dn_in"   GGUF blocks [2*Hk*dk + Hv*dv + 2*Hv, H], rows q | k | v | b | a
+ *     "blk.L.dn_out"  GGUF blocks [H, Hv*dv]
+ *   attention layers:
+ *     "blk.L.attn_in"     GGUF blocks [2*Hq*dh + 2*Hkv*dh, H], rows q | gate | k | v
+ *     "blk.L.attn_q_norm", "blk.L.attn_k_norm"   f32 [dh]
+ *     "blk.L.attn_out"    GGUF blocks [H, Hq*dh]
+ *   "blk.L.ffn_gate", "blk.L.ffn_up"  GGUF blocks [F, H];  "blk.L.ffn_down"  GGUF blocks [H, F]
+ * A GGUF matrix [rows, cols] is rows * cols/32 blocks in row-major block order;
+ * Q4_0 block = binary16 d + 16 bytes (element j low nibble of byte j, element
+ * j+16 high nibble, weight (nibble-8)*d); Q8_0 block = binary16 d + 32 int8
+ * (weight q*d). */
+typedef struct {
+  const char* name;
+  const void* data;
+  size_t bytes;
+} stage_tensor;
+
+/* Create a stage for layers [layer_begin, layer_end) on the current CUDA
+ * device.  Uploads and repacks the weights, allocates recurrent states (zero),
+ * KV caches (zero), a rollback ring of 17 snapshots per DeltaNet layer and all
+ * scratch.  cuda_stream (a cudaStream_t, may be NULL for the legacy default
+ * stream) orders every later call of this stage.  Blocks until the upload is
+ * done.  On success *out owns all device memory until stage_free. */
+stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, int n_tensors,
+                        int layer_begin, int layer_end, void* cuda_stream, stage_t** out);
+
+/* Run n_tok tokens (1..16) at positions pos .. pos+n_tok-1 through every layer
+ * of the stage (one CUDA-graph launch).  hidden_dev: caller-owned device f32
+ * [n_tok, H], row-major, read and overwritten in place with the stage output.
+ * pos must equal the committed length.  Leaves the pass pending: the next
+ * forward is refused until stage_commit / stage_rollback.  Token t's output is
+ * bit-identical to running the same tokens one at a time (forward(1) +
+ * commit(1) each). */
+stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos);
+
+/* Keep the first n_accepted tokens (0..n_tok) of the pending pass: each
+ * DeltaNet state becomes the snapshot after token n_accepted (no copy: the
+ * ring index moves) and the committed length becomes pos + n_accepted.  KV
+ * rows beyond it stay in memory but are never read and are overwritten by the
+ * next pass.  The result is bit-identical to having run only those tokens. */
+stage_status stage_commit(stage_t* st, int n_accepted);
+
+/* Discard the pending pass: identical to stage_commit(st, 0). */
+stage_status stage_rollback(stage_t* st);
+
+/* Start a new sequence: zero every recurrent state, committed length 0.
+ * Refused while a pass is pending. */
+stage_status stage_reset(stage_t* st);
+
+/* Wait for the stage's stream; returns STAGE_E_DEVICE if a stage kernel
+ * reported a device-side error since the last stage_sync (and clears it). */
+stage_status stage_sync(stage_t* st);
+
+/* Committed length (positions in the KV caches that are part of the sequence). */
+int stage_committed_len(const stage_t* st);
+
+/* Number of tokens of the pending pass, 0 if none. */
+int stage_pending(const stage_t* st);
+
+/* Copy the current state of DeltaNet layer `layer` (absolute index) to/from
+ * host memory: f32 [Hv, dv, dk] row-major (S[h][i][j], i the value dim), bytes
+ * must be Hv*dv*dk*4.  Synchronous.  Refused while a pass is pending. */
+stage_status stage_get_dn_state(stage_t* st, int layer, float* host_dst, size_t bytes);
+stage_status stage_set_dn_state(stage_t* st, int layer, const float* host_src, size_t bytes);
+
+/* Copy the KV cache of attention layer `layer` to/from host memory: binary16
+ * bit patterns [Hkv, max_ctx, dh] for K and for V, bytes_each =
+ * Hkv*max_ctx*dh*2.  Synchronous.  Refused while a pass is pending. */
+stage_status stage_get_kv(stage_t* st, int layer, uint16_t* k_host, uint16_t* v_host, size_t bytes_each);
+stage_status stage_set_kv(stage_t* st, int layer, const uint16_t* k_host, const uint16_t* v_host,
+                          size_t bytes_each);
+
+/* Set the committed length (e.g. after filling the KV caches with stage_set_kv).
+ * 0 <= kv_len <= max_ctx - 1.  Refused while a pass is pending. */
+stage_status stage_set_kv_len(stage_t* st, int kv_len);
+
+/* Dequantise row `row` of weight tensor `tensor` (a name as in stage_tensor)
+ * from the stage's packed device copy, with the same device code the GEMV
+ * uses, into host_dst (f32 [cols]).  Synchronous.  Used to check that the
+ * repacked weights dequantise bit-exactly. */
+stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst);
+
+/* Bytes of weight storage the stage streams per pass (packed quants + scales). */
+size_t stage_weight_bytes(const stage_t* st);
+
+/* Human-readable description of the last error of this stage ("" if none). */
+const char* stage_last_error(const stage_t* st);
+
+/* Free all device memory of the stage (waits for its stream).  NULL is a no-op. */
+void stage_free(stage_t* st);
+
+/* ---------------------------------------------------------------------------
+ * Kernel-level entry points (one hot-path kernel each, no stage object).
+ * Pointers named *_dev are device memory owned by the caller; the call is
+ * asynchronous on `stream`.  Return 0 on success or a negative stage_status;
+ * qhl_last_error() gives the message (per host thread).
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of the packed (repacked) form of a GGUF matrix [rows, cols]:
+ * ceil(rows/64) * cols/256 items of 9216 (Q4_0) or 17408 (Q8_0) bytes.
+ * For a gate/up pair (paired != 0) rows is the number of features of each
+ * matrix and the result holds both: ceil(rows/32) items per 256 columns.
+ * Returns 0 for an unsupported shape (cols % 256 != 0, rows <= 0). */
+size_t qhl_packed_bytes(int qtype, int rows, int cols, int paired);
+
+/* Repack GGUF blocks (device, [rows, cols/32] blocks) into the packed layout
+ * the GEMV streams.  gguf_b_dev: second matrix of a gate/up pair (its rows are
+ * interleaved tile by tile with gguf_dev's for the SwiGLU epilogue), or NULL.
+ * packed_dev must hold qhl_packed_bytes(qtype, rows, cols, gguf_b_dev != NULL)
+ * bytes and be 16-byte aligned. */
+int qhl_repack(int qtype, int rows, int cols, const void* gguf_dev, const void* gguf_b_dev,
+               void* packed_dev, void* stream);
+
+/* Dequantise rows [row0, row0+nrows) of a packed matrix into out_dev (f32
+ * [nrows, cols]) with the GEMV's own conversion code; bit-exact by design.
+ * paired != 0: rows 0..rows-1 address the first matrix of a pair, rows
+ * rows..2*rows-1 the second. */
+int qhl_dequant(int qtype, int rows, int cols, const void* packed_dev, int paired, int row0, int nrows,
+                float* out_dev, void* stream);
+
+/* y = x W^T for n_tok tokens (1..16): x_dev f32 [n_tok, cols], y_dev f32
+ * [n_tok, rows], W packed (not paired).  Reduction order is fixed and
+ * independent of n_tok (a batched call equals n_tok single calls bit for bit).
+ * Uses library-owned scratch (stream-K partials and tile counters, allocated
+ * on first use per device and grown on demand); concurrent calls on different
+ * streams of the same device must not overlap. */
+int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float* x_dev, int n_tok,
+              float* y_dev, void* stream);
+
+/* n_tok sequential gated-DeltaNet steps (dn_dim 128) for all Hv value heads.
+ * y_dev: f32 [n_tok, 2*Hk*128 + Hv*128 + 2*Hv] raw in-projection rows
+ * q | k | v | b | a per token (q, k are L2-normalised here; beta = sigmoid(b),
+ * alpha = exp(-softplus(a))).  s_in_dev: f32 [Hv, 128, 128] state before the
+ * first token (not modified).  snaps_dev: f32 [n_tok, Hv, 128, 128] receives
+ * the state after each token.  o_dev: f32 [n_tok, Hv*128] receives o_t = S_t q_t. */
+int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float* s_in_dev,
+                      float* snaps_dev, float* o_dev, void* stream);
+
+/* Message of the last failed qhl_* call on this host thread ("" if none). */
+const char* qhl_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QHL_STAGE_H */

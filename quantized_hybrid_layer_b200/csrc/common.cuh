@@ -1,0 +1,147 @@
+// Device helpers shared by the stage kernels (sm_100a only).
+//
+// Inline PTX for: packed f32x2 FMA, mbarrier phases, non-tensor bulk copies
+// global -> shared (no cluster multicast), L2 eviction hints and programmatic
+// dependent launch.  Every wait here is bounded: on timeout it records an error
+// bit in a device word the host reads, and returns.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define QHL_DEV __device__ __forceinline__
+
+namespace qhl {
+
+// Bits of the device error word.
+enum : unsigned {
+  ERR_WAIT_TIMEOUT = 1u,   // an mbarrier wait ran out of iterations
+  ERR_BAD_SHAPE = 2u,      // a kernel saw parameters it cannot handle
+};
+
+// Iteration cap of every mbarrier wait (each try_wait blocks for a short
+// hardware-defined time, so this bounds a stuck wait to well under a minute).
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+QHL_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// d = a * b + c on two f32 lanes, each rounded to nearest (fma.rn.f32x2).
+QHL_DEV float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long A, B, C, D;
+  A = (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+  B = (static_cast<unsigned long long>(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
+  C = (static_cast<unsigned long long>(__float_as_uint(c.y)) << 32) | __float_as_uint(c.x);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(D) : "l"(A), "l"(B), "l"(C));
+  return make_float2(__uint_as_float(static_cast<uint32_t>(D)),
+                     __uint_as_float(static_cast<uint32_t>(D >> 32)));
+}
+
+// ---- mbarrier -------------------------------------------------------------
+QHL_DEV void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+QHL_DEV void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+QHL_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+QHL_DEV void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+QHL_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete; false (and an error
+// bit) if it did not within kWaitLimit tries.
+QHL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
+  return false;
+}
+
+// ---- bulk copies (non-tensor TMA) -----------------------------------------
+QHL_DEV uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// Copy `bytes` (multiple of 16, both addresses 16-byte aligned) from global to
+// this CTA's shared memory; completion is signalled on `bar` as tx bytes.
+QHL_DEV void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+QHL_DEV void bulk_g2s_plain(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same memory.
+QHL_DEV void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- programmatic dependent launch ---------------------------------------
+// Block until every grid this one depends on has completed and its memory is
+// visible (no-op when launched without a programmatic dependency).
+QHL_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the dependent grid to be scheduled.
+QHL_DEV void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---- named barrier among a subset of warps ---------------------------------
+QHL_DEV void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---- warp reductions: xor butterflies give every lane the same bits --------
+QHL_DEV float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+QHL_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Sum of squares of 64 values in row order; the one definition used for the
+// per-tile RMSNorm partials everywhere, so a stage's result never depends on
+// which kernel produced its input.
+QHL_DEV float sumsq64(const float* v) {
+  float s = 0.f;
+#pragma unroll 8
+  for (int r = 0; r < 64; ++r) s = __fmaf_rn(v[r], v[r], s);
+  return s;
+}
+
+// 1 / sqrt(mean + eps) from per-tile partial sums, summed in tile order.
+QHL_DEV float rstd_from_partials(const float* ss, int ntiles, float inv_dim, float eps) {
+  float s = 0.f;
+  for (int i = 0; i < ntiles; ++i) s = __fadd_rn(s, ss[i]);
+  return __frcp_rn(__fsqrt_rn(__fadd_rn(__fmul_rn(s, inv_dim), eps)));
+}
+
+QHL_DEV float sigmoidf_(float x) { return __frcp_rn(__fadd_rn(1.f, expf(-x))); }
+
+}  // namespace qhl

@@ -1,0 +1,100 @@
+// Gated-DeltaNet state step over n_tok tokens (Gated DeltaNet: ChatTorrent
+// README, "What it can run"; SwarmLLM README model table "hybrid
+// Gated-DeltaNet + attention"; the gated delta rule of the Gated DeltaNet paper
+// its prior-work line names).
+//
+// Per value head h (key head g = h / (Hv/Hk)), with q, k L2-normalised,
+// beta = sigmoid(b) and alpha = exp(-softplus(a)) = 1 / (1 + e^a):
+//     S <- alpha * S (I - beta k k^T) + beta v k^T,      o = S q  (updated S)
+// Row i of S (value dim) changes independently of the others:
+//     S_i <- alpha S_i + beta (v_i - alpha (S_i . k)) k,   o_i = S_i . q
+//
+// Each warp keeps 4 rows of one head's 128x128 f32 state in registers (lane l
+// holds columns 4l..4l+3) for all NT tokens, so the state is read from HBM once
+// and written once per token as the snapshot S_t used for exact rollback
+// (SwarmLLM README: batched verify "with exact rollback of the recurrent
+// state").  The state rows are loaded before griddepcontrol.wait, overlapping
+// the in-projection that produces q, k, v, b, a.  Reductions are xor
+// butterflies over fixed lane partials, so every token's arithmetic is the
+// same whatever NT is.
+#pragma once
+
+#include "common.cuh"
+
+namespace qhl {
+
+constexpr int kDnDim = 128;
+
+struct DnArgs {
+  const float* y;          // [NT][y_stride] in-projection output: q | k | v | b | a
+  int y_stride;
+  int Hk, Hv;
+  // state source / snapshot destinations:
+  //   cur != nullptr (stage): S_0 = ring[*cur], S_t -> ring[(*cur + t) % ring_size]
+  //   cur == nullptr: S_0 = s_in, S_t -> ring[t - 1]
+  float* ring;
+  long long state_elems;   // Hv * 128 * 128
+  int ring_size;
+  const int* cur;
+  const float* s_in;
+  float* o;                // [NT][o_stride], o_stride >= Hv * 128
+  int o_stride;
+};
+
+QHL_DEV float dot4(float4 a, float4 b) {
+  float s = __fmul_rn(a.x, b.x);
+  s = __fmaf_rn(a.y, b.y, s);
+  s = __fmaf_rn(a.z, b.z, s);
+  return __fmaf_rn(a.w, b.w, s);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(128) dn_step_kernel(const DnArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x >> 3;                       // 8 CTAs of 16 rows per head
+  const int row0 = (blockIdx.x & 7) * 16 + warp * 4;
+  const int g = h / (a.Hv / a.Hk);
+  if (threadIdx.x == 0) pdl_launch();
+
+  const int cur = a.cur ? *a.cur : 0;
+  const float* s_in = a.cur ? a.ring + (size_t)cur * a.state_elems : a.s_in;
+  float4 S[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    S[r] = __ldg(reinterpret_cast<const float4*>(s_in + ((size_t)h * kDnDim + row0 + r) * kDnDim) + lane);
+
+  pdl_wait();
+
+  const int off_k = a.Hk * kDnDim;
+  const int off_v = 2 * a.Hk * kDnDim;
+  const int off_b = off_v + a.Hv * kDnDim;
+  const int off_a = off_b + a.Hv;
+  for (int t = 0; t < NT; ++t) {
+    const float* yt = a.y + (size_t)t * a.y_stride;
+    float4 q = *(reinterpret_cast<const float4*>(yt + g * kDnDim) + lane);
+    float4 k = *(reinterpret_cast<const float4*>(yt + off_k + g * kDnDim) + lane);
+    const float rq = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(q, q)), 1e-6f)));
+    const float rk = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(k, k)), 1e-6f)));
+    q = make_float4(__fmul_rn(q.x, rq), __fmul_rn(q.y, rq), __fmul_rn(q.z, rq), __fmul_rn(q.w, rq));
+    k = make_float4(__fmul_rn(k.x, rk), __fmul_rn(k.y, rk), __fmul_rn(k.z, rk), __fmul_rn(k.w, rk));
+    const float beta = __frcp_rn(__fadd_rn(1.f, expf(-yt[off_b + h])));
+    const float alpha = __frcp_rn(__fadd_rn(1.f, expf(yt[off_a + h])));
+    float* dst = a.cur ? a.ring + (size_t)((cur + 1 + t) % a.ring_size) * a.state_elems
+                       : a.ring + (size_t)t * a.state_elems;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float v = yt[off_v + h * kDnDim + row0 + r];
+      const float kS = warp_sum(dot4(S[r], k));
+      const float coef = __fmul_rn(beta, __fsub_rn(v, __fmul_rn(alpha, kS)));
+      S[r].x = __fmaf_rn(coef, k.x, __fmul_rn(alpha, S[r].x));
+      S[r].y = __fmaf_rn(coef, k.y, __fmul_rn(alpha, S[r].y));
+      S[r].z = __fmaf_rn(coef, k.z, __fmul_rn(alpha, S[r].z));
+      S[r].w = __fmaf_rn(coef, k.w, __fmul_rn(alpha, S[r].w));
+      const float o = warp_sum(dot4(S[r], q));
+      if (lane == 0) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
+      reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = S[r];
+    }
+  }
+}
+
+}  // namespace qhl

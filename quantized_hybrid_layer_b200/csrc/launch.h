@@ -1,0 +1,62 @@
+// Host-side launch wrappers for the stage kernels (one translation unit per
+// kernel family; the runtime only sees these declarations).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <utility>
+
+#include "attention.cuh"
+#include "deltanet.cuh"
+#include "qgemv.cuh"
+
+namespace qhl {
+
+// cudaLaunchKernelEx with an optional programmatic-dependent-launch attribute:
+// the kernel may start while the previous kernel on the stream is still
+// running; it must call griddepcontrol.wait before reading that kernel's output.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// GEMV: qt in {2, 8}, nt in 1..16, epi in {EPI_STORE, EPI_SWIGLU, EPI_RESID}.
+cudaError_t gemv_prepare(int qt);   // sets the dynamic shared-memory limit of every instantiation
+cudaError_t launch_gemv(int qt, int nt, int epi, const GemvArgs& a, int grid, cudaStream_t s, bool pdl);
+int gemv_smem(int qt, int nt);
+
+cudaError_t mixers_prepare(int rep);   // rep = query heads per KV head
+cudaError_t launch_dn_step(int nt, const DnArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_attn_partial(int nt, const AttnArgs& a, int nchunk, int hkv, cudaStream_t s, bool pdl);
+cudaError_t launch_attn_combine(int nt, const AttnArgs& a, cudaStream_t s, bool pdl);
+cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, float* z, float* ss,
+                               int ss_stride, cudaStream_t s);
+
+cudaError_t launch_repack(int qt, const uint8_t* a, const uint8_t* b, int rows, int cols, uint8_t* out,
+                          cudaStream_t s);
+cudaError_t launch_dequant(int qt, const uint8_t* packed, int rows, int cols, int paired, int row0, int nrows,
+                           float* out, cudaStream_t s);
+cudaError_t launch_rope_table(float2* tab, int max_ctx, int rope_dims, double theta, cudaStream_t s);
+cudaError_t launch_commit(int* ctrl, int n_accepted, int n_dn, int ring, cudaStream_t s);
+cudaError_t launch_set_int(int* p, int v, cudaStream_t s);
+
+// packed-layout geometry
+inline int packed_tiles(int rows, bool paired) { return paired ? (rows + 31) / 32 : (rows + 63) / 64; }
+inline size_t packed_bytes(int qt, int rows, int cols, bool paired) {
+  if (rows <= 0 || cols <= 0 || cols % kChunkCols || (qt != kQ4_0 && qt != kQ8_0)) return 0;
+  return (size_t)packed_tiles(rows, paired) * (cols / kChunkCols) * item_bytes(qt);
+}
+
+}  // namespace qhl

@@ -1,0 +1,665 @@
+// Stage runtime and the C ABI (include/qhl_stage.h).
+//
+// A stage owns, on one GPU: the packed weights of its layer range, a rollback
+// ring of DeltaNet state snapshots per DeltaNet layer, an f16 KV cache per
+// attention layer, activation buffers for up to 16 tokens, and one CUDA graph
+// per token count.  stage_forward launches that graph: "one command submit per
+// token" (SwarmLLM README, paragraph after the peer diagram).  Inside the graph
+// every kernel after the first is launched with programmatic dependent launch,
+// so a projection's weights start streaming while the previous kernel drains.
+//
+// The position of the pass and each DeltaNet layer's current ring slot live in
+// a small device control block (ctrl[0] = committed length, ctrl[1 + i] = ring
+// slot of DeltaNet layer i), so the graphs never change; commit advances them
+// with one tiny kernel and rollback touches nothing on the device.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/qhl_stage.h"
+#include "launch.h"
+
+using namespace qhl;
+
+namespace qhl {
+void set_last_error(const std::string& s);   // kernel_abi.cu: message for qhl_last_error()
+}
+
+namespace {
+
+constexpr int kMaxTok = 16;
+constexpr int kRing = kMaxTok + 1;
+
+struct Layer {
+  int index = 0;
+  bool attn = false;
+  uint8_t* w_in = nullptr;
+  int in_rows = 0, in_tiles = 0;
+  uint8_t* w_out = nullptr;
+  int out_cols = 0;
+  uint8_t* w_gu = nullptr;
+  uint8_t* w_down = nullptr;
+  float* norm1 = nullptr;
+  float* norm2 = nullptr;
+  float* qn = nullptr;
+  float* kn = nullptr;
+  float* ring = nullptr;   // DeltaNet: [kRing][Hv][128][128]
+  int dn_slot = -1;
+  uint16_t* K = nullptr;   // attention: [Hkv][max_ctx][256] f16 bits
+  uint16_t* V = nullptr;
+};
+
+std::string cuda_msg(const char* what, cudaError_t e) {
+  return std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+}
+
+}  // namespace
+
+struct stage {
+  stage_config cfg{};
+  int begin = 0, end = 0;
+  cudaStream_t stream = nullptr;   // caller's stream: orders every call
+  cudaStream_t cap = nullptr;      // private stream used only to capture graphs
+  int device = 0, sms = 0;
+  std::vector<Layer> layers;
+  std::vector<void*> allocs;
+  float *h = nullptr, *z = nullptr, *ss = nullptr, *y = nullptr, *o = nullptr, *u = nullptr;
+  float *pm = nullptr, *pl = nullptr, *po = nullptr;
+  int nchunk = 0;
+  float2* rope = nullptr;
+  float* partials = nullptr;
+  int* counters = nullptr;
+  unsigned* err = nullptr;
+  int* ctrl = nullptr;
+  int n_dn = 0;
+  int ss_stride = 0, y_stride = 0, o_stride = 0;
+  long long state_elems = 0;
+  int committed = 0, pending_n = 0, pending_pos = 0;
+  std::vector<int> cur;
+  cudaGraphExec_t exec[kMaxTok + 1] = {};
+  size_t weight_bytes = 0;
+  std::string last_error;
+};
+
+namespace {
+
+stage_status fail(stage* st, stage_status code, const std::string& msg) {
+  if (st) st->last_error = msg;
+  return code;
+}
+
+#define CK(call)                                                            \
+  do {                                                                      \
+    cudaError_t e_ = (call);                                                \
+    if (e_ != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg(#call, e_)); \
+  } while (0)
+
+stage_status dalloc(stage* st, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return STAGE_OK;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    *p = nullptr;
+    return fail(st, STAGE_E_OOM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed: " + cudaGetErrorString(e));
+  }
+  st->allocs.push_back(*p);
+  return STAGE_OK;
+}
+
+template <typename T>
+stage_status dalloc_t(stage* st, T** p, size_t bytes) {
+  void* v = nullptr;
+  stage_status s = dalloc(st, &v, bytes);
+  *p = static_cast<T*>(v);
+  return s;
+}
+
+void destroy(stage* st) {
+  if (!st) return;
+  if (st->stream || st->cap) cudaDeviceSynchronize();
+  for (auto& g : st->exec)
+    if (g) cudaGraphExecDestroy(g);
+  for (void* p : st->allocs) cudaFree(p);
+  if (st->cap) cudaStreamDestroy(st->cap);
+  delete st;
+}
+
+size_t qbytes(int qt, long long rows, long long cols) { return (size_t)(rows * (cols / 32) * gguf_block_bytes(qt)); }
+
+bool parse_name(const char* name, int* layer, std::string* tag) {
+  if (!name || std::strncmp(name, "blk.", 4) != 0) return false;
+  const char* p = name + 4;
+  char* e = nullptr;
+  long v = std::strtol(p, &e, 10);
+  if (e == p || *e != '.') return false;
+  *layer = (int)v;
+  *tag = std::string(e + 1);
+  return true;
+}
+
+// Upload one GGUF matrix into the staging buffer.
+stage_status upload(stage* st, void* staging, const stage_tensor* t) {
+  CK(cudaMemcpy(staging, t->data, t->bytes, cudaMemcpyHostToDevice));
+  return STAGE_OK;
+}
+
+GemvArgs gemv_base(const stage* st) {
+  GemvArgs a = {};
+  a.partials = st->partials;
+  a.counters = st->counters;
+  a.err = st->err;
+  a.eps = st->cfg.eps;
+  a.inv_dim = 1.0f / (float)st->cfg.hidden;
+  return a;
+}
+
+cudaError_t run_gemv(const stage* st, int n, int epi, GemvArgs& a, cudaStream_t s) {
+  const long long items = (long long)a.tiles * a.chunks;
+  a.workers = (int)std::min<long long>(st->sms, items);
+  return launch_gemv(st->cfg.qtype, n, epi, a, a.workers, s, true);
+}
+
+// Record one pass of n tokens onto stream s (being captured).
+cudaError_t record_pass(stage* st, int n, cudaStream_t s) {
+  const stage_config& c = st->cfg;
+  const int H = c.hidden, F = c.ffn;
+  cudaError_t e = launch_stage_input(n, st->h, H, st->layers[0].norm1, st->z, st->ss, st->ss_stride, s);
+  if (e != cudaSuccess) return e;
+  for (size_t i = 0; i < st->layers.size(); ++i) {
+    const Layer& L = st->layers[i];
+    const float* next_norm1 = i + 1 < st->layers.size() ? st->layers[i + 1].norm1 : nullptr;
+    // mixer in-projection with the RMSNorm1 scale folded into the epilogue
+    GemvArgs a = gemv_base(st);
+    a.W = L.w_in;
+    a.tiles = L.in_tiles;
+    a.chunks = H / kChunkCols;
+    a.x = st->z;
+    a.x_stride = H;
+    a.y = st->y;
+    a.y_stride = st->y_stride;
+    a.out_valid = L.in_rows;
+    a.ss_in = st->ss;
+    a.ss_tiles = H / 64;
+    a.ss_stride = st->ss_stride;
+    if ((e = run_gemv(st, n, EPI_STORE, a, s)) != cudaSuccess) return e;
+    if (!L.attn) {
+      DnArgs d = {};
+      d.y = st->y;
+      d.y_stride = st->y_stride;
+      d.Hk = c.dn_k_heads;
+      d.Hv = c.dn_v_heads;
+      d.ring = L.ring;
+      d.state_elems = st->state_elems;
+      d.ring_size = kRing;
+      d.cur = st->ctrl + 1 + L.dn_slot;
+      d.o = st->o;
+      d.o_stride = st->o_stride;
+      if ((e = launch_dn_step(n, d, c.dn_v_heads * (kDnDim / 16), s, true)) != cudaSuccess) return e;
+    } else {
+      AttnArgs at = {};
+      at.y = st->y;
+      at.y_stride = st->y_stride;
+      at.Hq = c.att_q_heads;
+      at.Hkv = c.att_kv_heads;
+      at.K = L.K;
+      at.V = L.V;
+      at.max_ctx = c.max_ctx;
+      at.kv_len = st->ctrl;
+      at.gq = L.qn;
+      at.gk = L.kn;
+      at.rope = st->rope;
+      at.eps = c.eps;
+      at.pm = st->pm;
+      at.pl = st->pl;
+      at.po = st->po;
+      at.nchunk = st->nchunk;
+      at.out = st->o;
+      at.out_stride = st->o_stride;
+      if ((e = launch_attn_partial(n, at, st->nchunk, c.att_kv_heads, s, true)) != cudaSuccess) return e;
+      if ((e = launch_attn_combine(n, at, s, true)) != cudaSuccess) return e;
+    }
+    // out-projection + residual; z = h * norm2 and its tile sums of squares
+    a = gemv_base(st);
+    a.W = L.w_out;
+    a.tiles = H / 64;
+    a.chunks = L.out_cols / kChunkCols;
+    a.x = st->o;
+    a.x_stride = st->o_stride;
+    a.y = st->h;
+    a.y_stride = H;
+    a.out_valid = H;
+    a.gamma_next = L.norm2;
+    a.z_out = st->z;
+    a.z_stride = H;
+    a.ss_out = st->ss;
+    a.ss_out_stride = st->ss_stride;
+    if ((e = run_gemv(st, n, EPI_RESID, a, s)) != cudaSuccess) return e;
+    // gate/up with the RMSNorm2 scale and the SwiGLU epilogue
+    a = gemv_base(st);
+    a.W = L.w_gu;
+    a.tiles = (F + 31) / 32;
+    a.chunks = H / kChunkCols;
+    a.x = st->z;
+    a.x_stride = H;
+    a.y = st->u;
+    a.y_stride = F;
+    a.out_valid = F;
+    a.ss_in = st->ss;
+    a.ss_tiles = H / 64;
+    a.ss_stride = st->ss_stride;
+    if ((e = run_gemv(st, n, EPI_SWIGLU, a, s)) != cudaSuccess) return e;
+    // down + residual; z for the next layer's RMSNorm1
+    a = gemv_base(st);
+    a.W = L.w_down;
+    a.tiles = H / 64;
+    a.chunks = F / kChunkCols;
+    a.x = st->u;
+    a.x_stride = F;
+    a.y = st->h;
+    a.y_stride = H;
+    a.out_valid = H;
+    if (next_norm1) {
+      a.gamma_next = next_norm1;
+      a.z_out = st->z;
+      a.z_stride = H;
+      a.ss_out = st->ss;
+      a.ss_out_stride = st->ss_stride;
+    }
+    if ((e = run_gemv(st, n, EPI_RESID, a, s)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+stage_status build_graph(stage* st, int n) {
+  CK(cudaStreamBeginCapture(st->cap, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = record_pass(st, n, st->cap);
+  cudaGraph_t g = nullptr;
+  cudaError_t e2 = cudaStreamEndCapture(st->cap, &g);
+  if (e != cudaSuccess || e2 != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    (void)cudaGetLastError();
+    return fail(st, STAGE_E_CUDA, cuda_msg("recording the pass", e != cudaSuccess ? e : e2));
+  }
+  cudaGraphExec_t ex = nullptr;
+  e = cudaGraphInstantiate(&ex, g, 0);
+  cudaGraphDestroy(g);
+  if (e != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg("cudaGraphInstantiate", e));
+  st->exec[n] = ex;
+  return STAGE_OK;
+}
+
+const Layer* find_layer(const stage* st, int layer) {
+  if (layer < st->begin || layer >= st->end) return nullptr;
+  return &st->layers[layer - st->begin];
+}
+
+}  // namespace
+
+extern "C" {
+
+stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, int n_tensors, int layer_begin,
+                        int layer_end, void* cuda_stream, stage_t** out) {
+  if (!out) return STAGE_E_ARG;
+  *out = nullptr;
+  if (!cfg || (!tensors && n_tensors > 0) || n_tensors < 0) return STAGE_E_ARG;
+  const stage_config c = *cfg;
+  if (layer_begin < 0 || layer_end <= layer_begin) return STAGE_E_ARG;
+  if (c.qtype != STAGE_Q4_0 && c.qtype != STAGE_Q8_0) return STAGE_E_UNSUPPORTED;
+  if (c.hidden <= 0 || c.hidden % kChunkCols || c.ffn <= 0 || c.ffn % kChunkCols) return STAGE_E_UNSUPPORTED;
+  if (c.dn_dim != kDnDim || c.dn_k_heads <= 0 || c.dn_v_heads <= 0 || c.dn_v_heads % c.dn_k_heads)
+    return STAGE_E_UNSUPPORTED;
+  if (c.att_dim != kAttDim || c.rope_dims != kRopeDims || c.att_kv_heads <= 0 || c.att_q_heads <= 0 ||
+      c.att_q_heads % c.att_kv_heads || c.att_q_heads / c.att_kv_heads > 7)
+    return STAGE_E_UNSUPPORTED;
+  if (c.attn_every <= 0 || c.max_ctx < kMaxTok || !(c.eps > 0.f) || !(c.rope_theta > 0.0)) return STAGE_E_ARG;
+
+  stage* st = new (std::nothrow) stage();
+  if (!st) return STAGE_E_OOM;
+  st->cfg = c;
+  st->begin = layer_begin;
+  st->end = layer_end;
+  st->stream = static_cast<cudaStream_t>(cuda_stream);
+  auto bail = [&](stage_status s) {
+    // the stage is gone: its message stays readable through qhl_last_error()
+    set_last_error(st->last_error.empty() ? "stage_load failed" : st->last_error);
+    destroy(st);
+    return s;
+  };
+
+  // --- tensor table ------------------------------------------------------
+  std::unordered_map<std::string, const stage_tensor*> by_name;
+  for (int i = 0; i < n_tensors; ++i) {
+    if (!tensors[i].name || !tensors[i].data) return bail(STAGE_E_ARG);
+    by_name[tensors[i].name] = &tensors[i];
+  }
+  const int H = c.hidden, F = c.ffn, qt = c.qtype;
+  const int dn_in = 2 * c.dn_k_heads * kDnDim + c.dn_v_heads * kDnDim + 2 * c.dn_v_heads;
+  const int dn_o = c.dn_v_heads * kDnDim;
+  const int at_in = 2 * c.att_q_heads * kAttDim + 2 * c.att_kv_heads * kAttDim;
+  const int at_o = c.att_q_heads * kAttDim;
+  auto need = [&](int layer, const char* tag, size_t bytes, const stage_tensor** t) -> bool {
+    auto it = by_name.find("blk." + std::to_string(layer) + "." + tag);
+    if (it == by_name.end()) {
+      st->last_error = std::string("missing tensor blk.") + std::to_string(layer) + "." + tag;
+      return false;
+    }
+    if (it->second->bytes != bytes) {
+      st->last_error = std::string("tensor blk.") + std::to_string(layer) + "." + tag + " has " +
+                       std::to_string(it->second->bytes) + " bytes, expected " + std::to_string(bytes);
+      return false;
+    }
+    *t = it->second;
+    return true;
+  };
+  bool any_attn = false;
+  size_t max_q = 0;
+  for (int l = layer_begin; l < layer_end; ++l) {
+    const bool attn = l % c.attn_every == c.attn_every - 1;
+    any_attn |= attn;
+    const stage_tensor* t;
+    if (!need(l, "norm1", (size_t)H * 4, &t) || !need(l, "norm2", (size_t)H * 4, &t)) return bail(STAGE_E_FORMAT);
+    if (attn) {
+      if (!need(l, "attn_in", qbytes(qt, at_in, H), &t) || !need(l, "attn_out", qbytes(qt, H, at_o), &t) ||
+          !need(l, "attn_q_norm", (size_t)kAttDim * 4, &t) || !need(l, "attn_k_norm", (size_t)kAttDim * 4, &t))
+        return bail(STAGE_E_FORMAT);
+      max_q = std::max({max_q, qbytes(qt, at_in, H), qbytes(qt, H, at_o)});
+    } else {
+      if (!need(l, "dn_in", qbytes(qt, dn_in, H), &t) || !need(l, "dn_out", qbytes(qt, H, dn_o), &t))
+        return bail(STAGE_E_FORMAT);
+      max_q = std::max({max_q, qbytes(qt, dn_in, H), qbytes(qt, H, dn_o)});
+    }
+    if (!need(l, "ffn_gate", qbytes(qt, F, H), &t) || !need(l, "ffn_up", qbytes(qt, F, H), &t) ||
+        !need(l, "ffn_down", qbytes(qt, H, F), &t))
+      return bail(STAGE_E_FORMAT);
+    max_q = std::max({max_q, qbytes(qt, F, H), qbytes(qt, H, F)});
+  }
+
+  // --- device setup ------------------------------------------------------
+  cudaError_t e;
+  if ((e = cudaGetDevice(&st->device)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaGetDevice", e)));
+  if ((e = cudaDeviceGetAttribute(&st->sms, cudaDevAttrMultiProcessorCount, st->device)) != cudaSuccess)
+    return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaDeviceGetAttribute", e)));
+  if ((e = cudaStreamCreateWithFlags(&st->cap, cudaStreamNonBlocking)) != cudaSuccess)
+    return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaStreamCreate", e)));
+  if ((e = gemv_prepare(qt)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("gemv_prepare", e)));
+  if ((e = mixers_prepare(c.att_q_heads / c.att_kv_heads)) != cudaSuccess)
+    return bail(fail(st, STAGE_E_CUDA, cuda_msg("mixers_prepare", e)));
+  if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("sync", e)));
+
+  uint8_t *stage_a = nullptr, *stage_b = nullptr;
+  stage_status s;
+  if ((s = dalloc_t(st, &stage_a, max_q)) != STAGE_OK) return bail(s);
+  if ((s = dalloc_t(st, &stage_b, max_q)) != STAGE_OK) return bail(s);
+
+  st->state_elems = (long long)c.dn_v_heads * kDnDim * kDnDim;
+  const size_t kv_elems = (size_t)c.att_kv_heads * c.max_ctx * kAttDim;
+  for (int l = layer_begin; l < layer_end; ++l) {
+    Layer L;
+    L.index = l;
+    L.attn = l % c.attn_every == c.attn_every - 1;
+    auto T = [&](const char* tag) { return by_name["blk." + std::to_string(l) + "." + tag]; };
+    auto qmat = [&](const stage_tensor* t, int rows, int cols, uint8_t** dst) -> stage_status {
+      stage_status r;
+      const size_t pb = packed_bytes(qt, rows, cols, false);
+      if ((r = dalloc_t(st, dst, pb)) != STAGE_OK) return r;
+      if ((r = upload(st, stage_a, t)) != STAGE_OK) return r;
+      cudaError_t ee = launch_repack(qt, stage_a, nullptr, rows, cols, *dst, nullptr);
+      if (ee != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg("repack", ee));
+      if ((ee = cudaDeviceSynchronize()) != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg("repack sync", ee));
+      st->weight_bytes += pb;
+      return STAGE_OK;
+    };
+    auto vec = [&](const stage_tensor* t, float** dst) -> stage_status {
+      stage_status r;
+      if ((r = dalloc_t(st, dst, t->bytes)) != STAGE_OK) return r;
+      CK(cudaMemcpy(*dst, t->data, t->bytes, cudaMemcpyHostToDevice));
+      return STAGE_OK;
+    };
+    if ((s = vec(T("norm1"), &L.norm1)) != STAGE_OK || (s = vec(T("norm2"), &L.norm2)) != STAGE_OK) return bail(s);
+    if (L.attn) {
+      L.in_rows = at_in;
+      L.out_cols = at_o;
+      if ((s = qmat(T("attn_in"), at_in, H, &L.w_in)) != STAGE_OK) return bail(s);
+      if ((s = qmat(T("attn_out"), H, at_o, &L.w_out)) != STAGE_OK) return bail(s);
+      if ((s = vec(T("attn_q_norm"), &L.qn)) != STAGE_OK || (s = vec(T("attn_k_norm"), &L.kn)) != STAGE_OK)
+        return bail(s);
+      if ((s = dalloc_t(st, &L.K, kv_elems * 2)) != STAGE_OK || (s = dalloc_t(st, &L.V, kv_elems * 2)) != STAGE_OK)
+        return bail(s);
+      if ((e = cudaMemset(L.K, 0, kv_elems * 2)) != cudaSuccess || (e = cudaMemset(L.V, 0, kv_elems * 2)) != cudaSuccess)
+        return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
+    } else {
+      L.in_rows = dn_in;
+      L.out_cols = dn_o;
+      if ((s = qmat(T("dn_in"), dn_in, H, &L.w_in)) != STAGE_OK) return bail(s);
+      if ((s = qmat(T("dn_out"), H, dn_o, &L.w_out)) != STAGE_OK) return bail(s);
+      const size_t rb = (size_t)kRing * st->state_elems * 4;
+      if ((s = dalloc_t(st, &L.ring, rb)) != STAGE_OK) return bail(s);
+      if ((e = cudaMemset(L.ring, 0, rb)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
+      L.dn_slot = st->n_dn++;
+    }
+    L.in_tiles = packed_tiles(L.in_rows, false);
+    {
+      // gate and up, interleaved tile by tile for the SwiGLU epilogue
+      const size_t pb = packed_bytes(qt, F, H, true);
+      if ((s = dalloc_t(st, &L.w_gu, pb)) != STAGE_OK) return bail(s);
+      if ((s = upload(st, stage_a, T("ffn_gate"))) != STAGE_OK) return bail(s);
+      if ((s = upload(st, stage_b, T("ffn_up"))) != STAGE_OK) return bail(s);
+      if ((e = launch_repack(qt, stage_a, stage_b, F, H, L.w_gu, nullptr)) != cudaSuccess ||
+          (e = cudaDeviceSynchronize()) != cudaSuccess)
+        return bail(fail(st, STAGE_E_CUDA, cuda_msg("repack gate/up", e)));
+      st->weight_bytes += pb;
+    }
+    if ((s = qmat(T("ffn_down"), H, F, &L.w_down)) != STAGE_OK) return bail(s);
+    st->layers.push_back(L);
+  }
+  // staging no longer needed
+  cudaFree(stage_a);
+  cudaFree(stage_b);
+  st->allocs.erase(std::remove_if(st->allocs.begin(), st->allocs.end(),
+                                  [&](void* p) { return p == stage_a || p == stage_b; }),
+                   st->allocs.end());
+
+  // --- activations and scratch --------------------------------------------
+  const int y_rows = std::max(dn_in, at_in);
+  st->y_stride = (y_rows + 63) / 64 * 64;
+  st->o_stride = std::max(dn_o, at_o);
+  st->ss_stride = H / 64;
+  if ((s = dalloc_t(st, &st->h, (size_t)kMaxTok * H * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->z, (size_t)kMaxTok * H * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->ss, (size_t)kMaxTok * st->ss_stride * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->y, (size_t)kMaxTok * st->y_stride * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->o, (size_t)kMaxTok * st->o_stride * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->u, (size_t)kMaxTok * F * 4)) != STAGE_OK)
+    return bail(s);
+  if (any_attn) {
+    st->nchunk = (c.max_ctx + kAttChunk - 1) / kAttChunk;
+    const size_t np = (size_t)kMaxTok * c.att_q_heads * st->nchunk;
+    if ((s = dalloc_t(st, &st->pm, np * 4)) != STAGE_OK || (s = dalloc_t(st, &st->pl, np * 4)) != STAGE_OK ||
+        (s = dalloc_t(st, &st->po, np * kAttDim * 4)) != STAGE_OK ||
+        (s = dalloc_t(st, &st->rope, (size_t)c.max_ctx * (kRopeDims / 2) * sizeof(float2))) != STAGE_OK)
+      return bail(s);
+    if ((e = launch_rope_table(st->rope, c.max_ctx, c.rope_dims, c.rope_theta, nullptr)) != cudaSuccess)
+      return bail(fail(st, STAGE_E_CUDA, cuda_msg("rope table", e)));
+  }
+  const int max_tiles = std::max({packed_tiles(y_rows, false), packed_tiles(F, true), H / 64});
+  if ((s = dalloc_t(st, &st->partials, (size_t)2 * st->sms * kMaxTok * 64 * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->counters, (size_t)max_tiles * 4)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->err, 16)) != STAGE_OK ||
+      (s = dalloc_t(st, &st->ctrl, (size_t)(1 + st->n_dn) * 4)) != STAGE_OK)
+    return bail(s);
+  if ((e = cudaMemset(st->counters, 0, (size_t)max_tiles * 4)) != cudaSuccess ||
+      (e = cudaMemset(st->err, 0, 16)) != cudaSuccess ||
+      (e = cudaMemset(st->ctrl, 0, (size_t)(1 + st->n_dn) * 4)) != cudaSuccess ||
+      (e = cudaMemset(st->h, 0, (size_t)kMaxTok * H * 4)) != cudaSuccess)
+    return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
+  st->cur.assign(st->n_dn, 0);
+  if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("load sync", e)));
+  *out = st;
+  return STAGE_OK;
+}
+
+stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos) {
+  if (!st) return STAGE_E_ARG;
+  if (!hidden_dev) return fail(st, STAGE_E_ARG, "hidden_dev is NULL");
+  if (n_tok < 1 || n_tok > kMaxTok) return fail(st, STAGE_E_ARG, "n_tok must be in 1..16");
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending: commit or roll back first");
+  if (pos != st->committed) return fail(st, STAGE_E_STATE, "pos must equal the committed length");
+  if (pos + n_tok > st->cfg.max_ctx) return fail(st, STAGE_E_ARG, "pass would overflow max_ctx");
+  if (!st->exec[n_tok]) {
+    stage_status s = build_graph(st, n_tok);
+    if (s != STAGE_OK) return s;
+  }
+  const size_t bytes = (size_t)n_tok * st->cfg.hidden * 4;
+  CK(cudaMemcpyAsync(st->h, hidden_dev, bytes, cudaMemcpyDeviceToDevice, st->stream));
+  CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
+  CK(cudaMemcpyAsync(hidden_dev, st->h, bytes, cudaMemcpyDeviceToDevice, st->stream));
+  st->pending_n = n_tok;
+  st->pending_pos = pos;
+  return STAGE_OK;
+}
+
+stage_status stage_commit(stage_t* st, int n_accepted) {
+  if (!st) return STAGE_E_ARG;
+  if (!st->pending_n) return fail(st, STAGE_E_STATE, "no pending pass");
+  if (n_accepted < 0 || n_accepted > st->pending_n) return fail(st, STAGE_E_ARG, "n_accepted out of range");
+  if (n_accepted > 0) CK(launch_commit(st->ctrl, n_accepted, st->n_dn, kRing, st->stream));
+  st->committed = st->pending_pos + n_accepted;
+  for (int& v : st->cur) v = (v + n_accepted) % kRing;
+  st->pending_n = 0;
+  return STAGE_OK;
+}
+
+stage_status stage_rollback(stage_t* st) { return stage_commit(st, 0); }
+
+stage_status stage_reset(stage_t* st) {
+  if (!st) return STAGE_E_ARG;
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  CK(cudaMemsetAsync(st->ctrl, 0, (size_t)(1 + st->n_dn) * 4, st->stream));
+  for (const Layer& L : st->layers)
+    if (!L.attn) CK(cudaMemsetAsync(L.ring, 0, (size_t)st->state_elems * 4, st->stream));
+  st->committed = 0;
+  std::fill(st->cur.begin(), st->cur.end(), 0);
+  return STAGE_OK;
+}
+
+stage_status stage_sync(stage_t* st) {
+  if (!st) return STAGE_E_ARG;
+  CK(cudaStreamSynchronize(st->stream));
+  unsigned err = 0;
+  CK(cudaMemcpy(&err, st->err, sizeof(err), cudaMemcpyDeviceToHost));
+  if (err) {
+    CK(cudaMemset(st->err, 0, sizeof(err)));
+    return fail(st, STAGE_E_DEVICE, "device error word " + std::to_string(err) + " (bounded wait timed out)");
+  }
+  return STAGE_OK;
+}
+
+int stage_committed_len(const stage_t* st) { return st ? st->committed : -1; }
+int stage_pending(const stage_t* st) { return st ? st->pending_n : -1; }
+
+static stage_status dn_state_io(stage_t* st, int layer, void* host, size_t bytes, bool to_host) {
+  if (!st) return STAGE_E_ARG;
+  const Layer* L = find_layer(st, layer);
+  if (!L || L->attn) return fail(st, STAGE_E_ARG, "not a DeltaNet layer of this stage");
+  if (!host || bytes != (size_t)st->state_elems * 4) return fail(st, STAGE_E_ARG, "bad buffer or size");
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  CK(cudaStreamSynchronize(st->stream));
+  float* dev = L->ring + (size_t)st->cur[L->dn_slot] * st->state_elems;
+  if (to_host)
+    CK(cudaMemcpy(host, dev, bytes, cudaMemcpyDeviceToHost));
+  else
+    CK(cudaMemcpy(dev, host, bytes, cudaMemcpyHostToDevice));
+  return STAGE_OK;
+}
+
+stage_status stage_get_dn_state(stage_t* st, int layer, float* host_dst, size_t bytes) {
+  return dn_state_io(st, layer, host_dst, bytes, true);
+}
+stage_status stage_set_dn_state(stage_t* st, int layer, const float* host_src, size_t bytes) {
+  return dn_state_io(st, layer, const_cast<float*>(host_src), bytes, false);
+}
+
+static stage_status kv_io(stage_t* st, int layer, uint16_t* k, uint16_t* v, size_t bytes, bool to_host) {
+  if (!st) return STAGE_E_ARG;
+  const Layer* L = find_layer(st, layer);
+  if (!L || !L->attn) return fail(st, STAGE_E_ARG, "not an attention layer of this stage");
+  const size_t need = (size_t)st->cfg.att_kv_heads * st->cfg.max_ctx * kAttDim * 2;
+  if (!k || !v || bytes != need) return fail(st, STAGE_E_ARG, "bad buffer or size");
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  CK(cudaStreamSynchronize(st->stream));
+  if (to_host) {
+    CK(cudaMemcpy(k, L->K, bytes, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(v, L->V, bytes, cudaMemcpyDeviceToHost));
+  } else {
+    CK(cudaMemcpy(L->K, k, bytes, cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(L->V, v, bytes, cudaMemcpyHostToDevice));
+  }
+  return STAGE_OK;
+}
+
+stage_status stage_get_kv(stage_t* st, int layer, uint16_t* k_host, uint16_t* v_host, size_t bytes_each) {
+  return kv_io(st, layer, k_host, v_host, bytes_each, true);
+}
+stage_status stage_set_kv(stage_t* st, int layer, const uint16_t* k_host, const uint16_t* v_host, size_t bytes_each) {
+  return kv_io(st, layer, const_cast<uint16_t*>(k_host), const_cast<uint16_t*>(v_host), bytes_each, false);
+}
+
+stage_status stage_set_kv_len(stage_t* st, int kv_len) {
+  if (!st) return STAGE_E_ARG;
+  if (kv_len < 0 || kv_len >= st->cfg.max_ctx) return fail(st, STAGE_E_ARG, "kv_len out of range");
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  CK(launch_set_int(st->ctrl, kv_len, st->stream));
+  CK(cudaStreamSynchronize(st->stream));
+  st->committed = kv_len;
+  return STAGE_OK;
+}
+
+stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst) {
+  if (!st) return STAGE_E_ARG;
+  int layer;
+  std::string tag;
+  if (!host_dst || !parse_name(tensor, &layer, &tag)) return fail(st, STAGE_E_ARG, "bad tensor name or buffer");
+  const Layer* L = find_layer(st, layer);
+  if (!L) return fail(st, STAGE_E_ARG, "layer not in this stage");
+  const int H = st->cfg.hidden, F = st->cfg.ffn;
+  const uint8_t* P = nullptr;
+  int rows = 0, cols = 0, paired = 0, r = row;
+  if ((tag == "dn_in" && !L->attn) || (tag == "attn_in" && L->attn)) {
+    P = L->w_in; rows = L->in_rows; cols = H;
+  } else if ((tag == "dn_out" && !L->attn) || (tag == "attn_out" && L->attn)) {
+    P = L->w_out; rows = H; cols = L->out_cols;
+  } else if (tag == "ffn_gate" || tag == "ffn_up") {
+    P = L->w_gu; rows = F; cols = H; paired = 1;
+    if (tag == "ffn_up") r = row + F;
+  } else if (tag == "ffn_down") {
+    P = L->w_down; rows = H; cols = F;
+  } else {
+    return fail(st, STAGE_E_ARG, "not a quantised tensor of this layer");
+  }
+  if (row < 0 || row >= rows) return fail(st, STAGE_E_ARG, "row out of range");
+  float* tmp = nullptr;
+  cudaError_t e = cudaMalloc(&tmp, (size_t)cols * 4);
+  if (e != cudaSuccess) return fail(st, STAGE_E_OOM, cuda_msg("cudaMalloc", e));
+  e = launch_dequant(st->cfg.qtype, P, rows, cols, paired, r, 1, tmp, st->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st->stream);
+  if (e == cudaSuccess) e = cudaMemcpy(host_dst, tmp, (size_t)cols * 4, cudaMemcpyDeviceToHost);
+  cudaFree(tmp);
+  if (e != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg("dequant", e));
+  return STAGE_OK;
+}
+
+size_t stage_weight_bytes(const stage_t* st) { return st ? st->weight_bytes : 0; }
+
+const char* stage_last_error(const stage_t* st) { return st ? st->last_error.c_str() : "null stage"; }
+
+void stage_free(stage_t* st) { destroy(st); }
+
+}  // extern "C"
