@@ -28,16 +28,8 @@ QHL_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// d = a * b + c on two f32 lanes, each rounded to nearest (fma.rn.f32x2).
-QHL_DEV float2 ffma2(float2 a, float2 b, float2 c) {
-  unsigned long long A, B, C, D;
-  A = (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
-  B = (static_cast<unsigned long long>(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
-  C = (static_cast<unsigned long long>(__float_as_uint(c.y)) << 32) | __float_as_uint(c.x);
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(D) : "l"(A), "l"(B), "l"(C));
-  return make_float2(__uint_as_float(static_cast<uint32_t>(D)),
-                     __uint_as_float(static_cast<uint32_t>(D >> 32)));
-}
+// d = a * b + c on two f32 lanes, each rounded to nearest (packed FFMA2).
+QHL_DEV float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 // ---- mbarrier -------------------------------------------------------------
 QHL_DEV void mbar_init(uint32_t bar, uint32_t count) {
@@ -142,6 +134,12 @@ QHL_DEV float rstd_from_partials(const float* ss, int ntiles, float inv_dim, flo
   return __frcp_rn(__fsqrt_rn(__fadd_rn(__fmul_rn(s, inv_dim), eps)));
 }
 
-QHL_DEV float sigmoidf_(float x) { return __frcp_rn(__fadd_rn(1.f, expf(-x))); }
+// 1 / (1 + e^-x) without overflow: e^-|x| <= 1 always, so the result only
+// underflows where the true value is below the f32 range.
+QHL_DEV float sigmoidf_(float x) {
+  const float e = expf(-fabsf(x));
+  const float d = __fadd_rn(1.f, e);
+  return x >= 0.f ? __frcp_rn(d) : __fdiv_rn(e, d);
+}
 
 }  // namespace qhl

@@ -77,8 +77,8 @@ __global__ void __launch_bounds__(128) dn_step_kernel(const DnArgs a) {
     const float rk = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(k, k)), 1e-6f)));
     q = make_float4(__fmul_rn(q.x, rq), __fmul_rn(q.y, rq), __fmul_rn(q.z, rq), __fmul_rn(q.w, rq));
     k = make_float4(__fmul_rn(k.x, rk), __fmul_rn(k.y, rk), __fmul_rn(k.z, rk), __fmul_rn(k.w, rk));
-    const float beta = __frcp_rn(__fadd_rn(1.f, expf(-yt[off_b + h])));
-    const float alpha = __frcp_rn(__fadd_rn(1.f, expf(yt[off_a + h])));
+    const float beta = sigmoidf_(yt[off_b + h]);     // sigmoid(b)
+    const float alpha = sigmoidf_(-yt[off_a + h]);   // exp(-softplus(a)) = sigmoid(-a)
     float* dst = a.cur ? a.ring + (size_t)((cur + 1 + t) % a.ring_size) * a.state_elems
                        : a.ring + (size_t)t * a.state_elems;
 #pragma unroll

@@ -50,7 +50,7 @@ int get_scratch(int tiles, int qt, GemvScratch** out) {
   if (!s.ready) {
     if ((e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
       return cuda_err("cudaDeviceGetAttribute", e);
-    if ((e = cudaMalloc(&s.partials, (size_t)2 * s.sms * 16 * 64 * 4)) != cudaSuccess) return cuda_err("cudaMalloc", e);
+    if ((e = cudaMalloc(&s.partials, (size_t)2 * kCtasPerSm * s.sms * 16 * 64 * 4)) != cudaSuccess) return cuda_err("cudaMalloc", e);
     if ((e = cudaMalloc(&s.err, 16)) != cudaSuccess) return cuda_err("cudaMalloc", e);
     if ((e = cudaMemset(s.err, 0, 16)) != cudaSuccess) return cuda_err("cudaMemset", e);
     s.ready = true;
@@ -132,7 +132,7 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
   a.counters = s->counters;
   a.err = s->err;
   const long long items = (long long)a.tiles * a.chunks;
-  a.workers = (int)(items < s->sms ? items : s->sms);
+  a.workers = (int)(items < (long long)kCtasPerSm * s->sms ? items : (long long)kCtasPerSm * s->sms);
   cudaError_t e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, static_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? 0 : cuda_err("qgemv launch", e);
 }

@@ -57,20 +57,33 @@ struct GemvArgs {
   unsigned* err;           // device error word
 };
 
-template <int QT> struct GemvCfg;
-template <> struct GemvCfg<kQ4_0> { static constexpr int kStages = 10; };
-template <> struct GemvCfg<kQ8_0> { static constexpr int kStages = 5; };
-
 constexpr int kConsumerWarps = 8;
 constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
+// Stream-K workers per SM: the grid is kCtasPerSm * SMs for every token count
+// (the split, and hence the summation order, must not depend on NT).
+constexpr int kCtasPerSm = 2;
+
+// A stage holds one item's packed weights followed by the item's x columns for
+// every token ([NT][256] f32).  Up to 2 tokens the ring is small enough for two
+// CTAs of this kernel plus one of the next (under programmatic dependent
+// launch) to share an SM; up to 4 tokens two CTAs fit; beyond that one CTA per
+// SM runs at a time.
+template <int QT, int NT>
+struct GemvCfg {
+  static constexpr int kStageBytes = QLayout<QT>::kItemBytes + NT * kChunkCols * 4;
+  static constexpr int kBudget = NT <= 2 ? 72 * 1024 : (NT <= 4 ? 104 * 1024 : 196 * 1024);
+  static constexpr int kRaw = (kBudget - kConsumerWarps * NT * 64 * 4 - 512) / kStageBytes;
+  static constexpr int kStages = kRaw < 3 ? 3 : (kRaw > 12 ? 12 : kRaw);
+  static constexpr int kMinBlocks = NT <= 2 ? 3 : (NT <= 4 ? 2 : 1);
+};
 
 template <int QT, int NT>
 constexpr int gemv_smem_bytes() {
-  return GemvCfg<QT>::kStages * QLayout<QT>::kItemBytes      // stage ring
-         + kConsumerWarps * NT * 64 * 4                       // per-warp tile partials
-         + 16 * 4                                             // rstd
-         + 2 * GemvCfg<QT>::kStages * 8                       // full/empty mbarriers
-         + 16;                                                // flags
+  return GemvCfg<QT, NT>::kStages * GemvCfg<QT, NT>::kStageBytes   // stage ring
+         + kConsumerWarps * NT * 64 * 4                           // per-warp tile partials
+         + 16 * 4                                                 // rstd
+         + 2 * GemvCfg<QT, NT>::kStages * 8                       // full/empty mbarriers
+         + 16;                                                    // flags
 }
 
 // First item of CTA `w` in a balanced contiguous split of `n` items over `p` CTAs.
@@ -110,8 +123,8 @@ QHL_DEV void load_item(const uint8_t* st, int warp, int lane, ItemRegs<QT>& r) {
 // operation sequence is fixed: packed FMAs over the block's element pairs in
 // word order, the two lanes added, then one FMA with the block scale.
 template <int QT, int NT>
-QHL_DEV void compute_item(const ItemRegs<QT>& r, const float* xcol, int x_stride,
-                          float (&r0)[NT], float (&r1)[NT]) {
+QHL_DEV void compute_item(const ItemRegs<QT>& r, const float* xcol, float (&r0)[NT], float (&r1)[NT]) {
+  constexpr int x_stride = kChunkCols;   // x chunk in shared memory: [NT][256]
   float2 a0[NT], a1[NT];
 #pragma unroll
   for (int t = 0; t < NT; ++t) { a0[t] = make_float2(0.f, 0.f); a1[t] = make_float2(0.f, 0.f); }
@@ -123,9 +136,9 @@ QHL_DEV void compute_item(const ItemRegs<QT>& r, const float* xcol, int x_stride
       q4_word(r.b[i], q);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        const float4* xv = reinterpret_cast<const float4*>(xcol + (size_t)t * x_stride);
-        const float4 xa = __ldg(xv + i);
-        const float4 xb = __ldg(xv + 4 + i);
+        const float4* xv = reinterpret_cast<const float4*>(xcol + t * x_stride);
+        const float4 xa = xv[i];
+        const float4 xb = xv[4 + i];
         const float2 x0 = make_float2(xa.x, xa.y), x1 = make_float2(xa.z, xa.w);
         const float2 x2 = make_float2(xb.x, xb.y), x3 = make_float2(xb.z, xb.w);
         a0[t] = ffma2(p[0], x0, a0[t]);
@@ -146,7 +159,7 @@ QHL_DEV void compute_item(const ItemRegs<QT>& r, const float* xcol, int x_stride
       q8_word(r.b[i], q);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
-        const float4 xa = __ldg(reinterpret_cast<const float4*>(xcol + (size_t)t * x_stride) + i);
+        const float4 xa = reinterpret_cast<const float4*>(xcol + t * x_stride)[i];
         const float2 x0 = make_float2(xa.x, xa.y), x1 = make_float2(xa.z, xa.w);
         a0[t] = ffma2(p[0], x0, a0[t]);
         a0[t] = ffma2(p[1], x1, a0[t]);
@@ -202,12 +215,14 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float
 }
 
 template <int QT, int NT, int EPI>
-__global__ void __launch_bounds__(kGemvThreads, (NT <= 4 ? 2 : 1)) qgemv_kernel(const GemvArgs a) {
-  constexpr int S = GemvCfg<QT>::kStages;
+__global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
+  constexpr int S = GemvCfg<QT, NT>::kStages;
   constexpr int IB = QLayout<QT>::kItemBytes;
+  constexpr int SB = GemvCfg<QT, NT>::kStageBytes;
+  constexpr int XB = kChunkCols * 4;      // bytes of one token's x chunk
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* stages = smem;
-  float* red = reinterpret_cast<float*>(smem + S * IB);                 // [8][NT][64]
+  float* red = reinterpret_cast<float*>(smem + S * SB);                 // [8][NT][64]
   float* rstd = red + kConsumerWarps * NT * 64;                          // [16]
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstd + 16);              // full[S], empty[S]
   int* flag = reinterpret_cast<int*>(bars + 2 * S);
@@ -231,14 +246,37 @@ __global__ void __launch_bounds__(kGemvThreads, (NT <= 4 ? 2 : 1)) qgemv_kernel(
 
   if (warp == kConsumerWarps) {
     // ---------------- producer: stream this CTA's items into the ring ----------
+    // Weights never depend on earlier kernels: the first S items' weights are
+    // requested before griddepcontrol.wait.  Their x chunks (written by the
+    // previous kernel) follow once the dependency is resolved.
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      for (long long it = i0; it < i1; ++it) {
-        const int k = (int)(it - i0), s = k % S, round = k / S;
-        if (round > 0) mbar_wait(smem_u32(&bars[S + s]), (round - 1) & 1, a.err);
+      const int n_local = (int)(i1 - i0);
+      const int pre = n_local < S ? n_local : S;
+      const int c0 = (int)(i0 % a.chunks);
+      auto issue_x = [&](int k, int s) {
+        // chunk of local item k: (c0 + k) mod chunks, without 64-bit division
+        int c = c0 + k;
+        while (c >= a.chunks) c -= a.chunks;
         const uint32_t full = smem_u32(&bars[s]);
-        mbar_arrive_expect_tx(full, IB);
-        bulk_g2s(smem_u32(stages + s * IB), a.W + it * IB, IB, full, pol);
+        for (int t = 0; t < NT; ++t)
+          bulk_g2s_plain(smem_u32(stages + s * SB + IB + t * XB), a.x + (size_t)t * a.x_stride + (size_t)c * kChunkCols,
+                         XB, full);
+      };
+      for (int k = 0; k < pre; ++k) {
+        const uint32_t full = smem_u32(&bars[k]);
+        mbar_arrive_expect_tx(full, SB);
+        bulk_g2s(smem_u32(stages + k * SB), a.W + (i0 + k) * IB, IB, full, pol);
+      }
+      pdl_wait();
+      for (int k = 0; k < pre; ++k) issue_x(k, k);
+      for (int k = pre; k < n_local; ++k) {
+        const int s = k % S, round = k / S;
+        mbar_wait(smem_u32(&bars[S + s]), (round - 1) & 1, a.err);
+        const uint32_t full = smem_u32(&bars[s]);
+        mbar_arrive_expect_tx(full, SB);
+        bulk_g2s(smem_u32(stages + s * SB), a.W + (i0 + k) * IB, IB, full, pol);
+        issue_x(k, s);
       }
     }
     return;
@@ -309,20 +347,28 @@ __global__ void __launch_bounds__(kGemvThreads, (NT <= 4 ? 2 : 1)) qgemv_kernel(
   };
 
   named_sync(1, 256);   // rstd visible
-  for (long long it = i0; it < i1; ++it) {
-    const int t_it = (int)(it / a.chunks), c = (int)(it % a.chunks);
-    if (t_it != tile) {
+  const int n_local = (int)(i1 - i0);
+  int chunk = (int)(i0 - (long long)tile * a.chunks);
+  int s = 0;
+  uint32_t phase = 0;
+  for (int k = 0; k < n_local; ++k) {
+    if (chunk == a.chunks) {
       flush(tile);
-      tile = t_it;
+      ++tile;
+      chunk = 0;
     }
-    const int k = (int)(it - i0), s = k % S, round = k / S;
-    if (!mbar_wait(smem_u32(&bars[s]), round & 1, a.err)) timed_out = true;
+    if (!mbar_wait(smem_u32(&bars[s]), phase, a.err)) timed_out = true;
     ItemRegs<QT> regs;
-    load_item<QT>(stages + s * IB, warp, lane, regs);
+    const uint8_t* st = stages + s * SB;
+    load_item<QT>(st, warp, lane, regs);
+    compute_item<QT, NT>(regs, reinterpret_cast<const float*>(st + IB) + warp * 32, r0, r1);
     __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&bars[S + s]));   // stage free: its words are in registers
-    const float* xcol = a.x + (size_t)c * kChunkCols + warp * 32;
-    compute_item<QT, NT>(regs, xcol, a.x_stride, r0, r1);
+    if (lane == 0) mbar_arrive(smem_u32(&bars[S + s]));   // stage free for the producer
+    ++chunk;
+    if (++s == S) {
+      s = 0;
+      phase ^= 1u;
+    }
   }
   if (i1 > i0) flush(tile);
   if (timed_out && lane == 0) {

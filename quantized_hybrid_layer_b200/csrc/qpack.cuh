@@ -54,6 +54,15 @@ inline __host__ __device__ int gguf_block_bytes(int qt) { return qt == kQ4_0 ? 1
 // applied.
 constexpr uint32_t kMagic = 0x4B000000u;   // bit pattern of 2^23
 
+// (a & MASK) | magic in one LOP3 (the mask is an immediate, the magic a
+// register), reinterpreted as a float.
+template <uint32_t MASK>
+QHL_DEV float magic_field(uint32_t a, uint32_t magic) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(magic));
+  return __uint_as_float(d);
+}
+
 // Q4_0: the 32-bit word i (bytes 4i .. 4i+3) of a block holds elements
 // 4i, 4i+16, 4i+1, 4i+17, 4i+2, 4i+18, 4i+3, 4i+19 in its eight nibbles.
 // Returns them as (q-8) pairs: p[0] = (e4i, e4i+1), p[1] = (e4i+2, e4i+3),
@@ -63,11 +72,12 @@ QHL_DEV void q4_word(uint32_t w, float2 p[4]) {
   const float2 c_lo = make_float2(-8388616.0f, -32776.0f);     // -(2^23+8), -(2^15+8)
   const float2 s_hi = make_float2(0.0625f, 0.000244140625f);   // 2^-4, 2^-12
   const float2 c_hi = make_float2(-524296.0f, -2056.0f);       // -(2^19+8), -(2^11+8)
+  const uint32_t m = kMagic;
   const uint32_t w2 = w >> 16;
-  p[0] = ffma2(make_float2(__uint_as_float(kMagic | (w & 0x000Fu)), __uint_as_float(kMagic | (w & 0x0F00u))), s_lo, c_lo);
-  p[1] = ffma2(make_float2(__uint_as_float(kMagic | (w2 & 0x000Fu)), __uint_as_float(kMagic | (w2 & 0x0F00u))), s_lo, c_lo);
-  p[2] = ffma2(make_float2(__uint_as_float(kMagic | (w & 0x00F0u)), __uint_as_float(kMagic | (w & 0xF000u))), s_hi, c_hi);
-  p[3] = ffma2(make_float2(__uint_as_float(kMagic | (w2 & 0x00F0u)), __uint_as_float(kMagic | (w2 & 0xF000u))), s_hi, c_hi);
+  p[0] = ffma2(make_float2(magic_field<0x000Fu>(w, m), magic_field<0x0F00u>(w, m)), s_lo, c_lo);
+  p[1] = ffma2(make_float2(magic_field<0x000Fu>(w2, m), magic_field<0x0F00u>(w2, m)), s_lo, c_lo);
+  p[2] = ffma2(make_float2(magic_field<0x00F0u>(w, m), magic_field<0xF000u>(w, m)), s_hi, c_hi);
+  p[3] = ffma2(make_float2(magic_field<0x00F0u>(w2, m), magic_field<0xF000u>(w2, m)), s_hi, c_hi);
 }
 
 // Q8_0 (offset-binary bytes): word i holds elements 4i .. 4i+3.
@@ -75,9 +85,10 @@ QHL_DEV void q4_word(uint32_t w, float2 p[4]) {
 QHL_DEV void q8_word(uint32_t w, float2 p[2]) {
   const float2 s = make_float2(1.0f, 0.00390625f);
   const float2 c = make_float2(-8388736.0f, -32896.0f);        // -(2^23+128), -(2^15+128)
+  const uint32_t m = kMagic;
   const uint32_t w2 = w >> 16;
-  p[0] = ffma2(make_float2(__uint_as_float(kMagic | (w & 0xFFu)), __uint_as_float(kMagic | (w & 0xFF00u))), s, c);
-  p[1] = ffma2(make_float2(__uint_as_float(kMagic | (w2 & 0xFFu)), __uint_as_float(kMagic | (w2 & 0xFF00u))), s, c);
+  p[0] = ffma2(make_float2(magic_field<0x00FFu>(w, m), magic_field<0xFF00u>(w, m)), s, c);
+  p[1] = ffma2(make_float2(magic_field<0x00FFu>(w2, m), magic_field<0xFF00u>(w2, m)), s, c);
 }
 
 }  // namespace qhl

@@ -163,7 +163,7 @@ GemvArgs gemv_base(const stage* st) {
 
 cudaError_t run_gemv(const stage* st, int n, int epi, GemvArgs& a, cudaStream_t s) {
   const long long items = (long long)a.tiles * a.chunks;
-  a.workers = (int)std::min<long long>(st->sms, items);
+  a.workers = (int)std::min<long long>((long long)kCtasPerSm * st->sms, items);
   return launch_gemv(st->cfg.qtype, n, epi, a, a.workers, s, true);
 }
 
@@ -490,7 +490,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
       return bail(fail(st, STAGE_E_CUDA, cuda_msg("rope table", e)));
   }
   const int max_tiles = std::max({packed_tiles(y_rows, false), packed_tiles(F, true), H / 64});
-  if ((s = dalloc_t(st, &st->partials, (size_t)2 * st->sms * kMaxTok * 64 * 4)) != STAGE_OK ||
+  if ((s = dalloc_t(st, &st->partials, (size_t)2 * kCtasPerSm * st->sms * kMaxTok * 64 * 4)) != STAGE_OK ||
       (s = dalloc_t(st, &st->counters, (size_t)max_tiles * 4)) != STAGE_OK ||
       (s = dalloc_t(st, &st->err, 16)) != STAGE_OK ||
       (s = dalloc_t(st, &st->ctrl, (size_t)(1 + st->n_dn) * 4)) != STAGE_OK)

@@ -16,8 +16,11 @@ Workload recipe (one stream per tensor, so any subset can be regenerated alone):
 * Q4_0 matrix [rows, cols]: first ``rows*cols/32`` scale draws
   ``d = f16(|N(0,1)| * 0.02)`` (row-major over (row, block)), then
   ``rows*cols/32*16`` uniform random bytes (two uniform nibbles each).
-* Q8_0 matrix: the same scale draws, then ``rows*cols`` int8 draws uniform on
-  [-127, 127].
+* Q8_0 matrix: scale draws ``d = f16(|N(0,1)| * 0.02 * 8/127)``, then
+  ``rows*cols`` int8 draws uniform on [-127, 127].  (Reading: the Q8_0 variant
+  is the same model quantised to 8 bits, so a block's scale is the Q4_0 scale
+  times 8/127, as a max-abs quantiser gives for 4-bit [-8, 7] vs 8-bit
+  [-127, 127] codes; weights then have the Q4_0 magnitudes.)
 * RMSNorm / QK-norm weights: ``1 + N(0, 0.02)`` in f32.
 * Hidden states: ``N(0, 1)`` f32.  DeltaNet states: ``N(0, 0.01)`` f32.
   KV-cache prefill: ``N(0, 1)`` rounded to f16.
@@ -105,8 +108,8 @@ def rng_for(seed: int, *key: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed, spawn_key=tuple(int(k) for k in key))))
 
 
-def _scales(rng: np.random.Generator, nblocks: int) -> np.ndarray:
-    return (np.abs(rng.standard_normal(nblocks)) * 0.02).astype(np.float16)
+def _scales(rng: np.random.Generator, nblocks: int, scale: float = 0.02) -> np.ndarray:
+    return (np.abs(rng.standard_normal(nblocks)) * scale).astype(np.float16)
 
 
 def q4_0_matrix(rng: np.random.Generator, rows: int, cols: int) -> np.ndarray:
@@ -125,7 +128,7 @@ def q8_0_matrix(rng: np.random.Generator, rows: int, cols: int) -> np.ndarray:
     """GGUF Q8_0 blocks, uint8 [rows, cols/32, 34]: binary16 d then 32 int8 in [-127, 127]."""
     assert cols % QK == 0
     nb = cols // QK
-    d = _scales(rng, rows * nb)
+    d = _scales(rng, rows * nb, 0.02 * 8.0 / 127.0)
     qs = rng.integers(-127, 128, size=(rows, nb, 32), dtype=np.int8)
     out = np.empty((rows, nb, 34), dtype=np.uint8)
     out[:, :, 0:2] = d.view(np.uint8).reshape(rows, nb, 2)

@@ -71,10 +71,11 @@ def test_four_layer_stage_decode_matches_oracle(stage3):
         for l in attn_layers(0, 4):
             K, V = st.get_kv(l)
             for X, R in ((K, orc.K[l]), (V, orc.V[l])):
-                row = X[:, pos].astype(np.float64)
-                ref_row = R[:, pos].astype(np.float64)
-                assert max(rel_err_rows(row, ref_row)) <= TOL
-                assert np.array_equal(X[:, :pos], R[:, :pos])          # older rows untouched
+                # rows this run wrote: f16 of an f32 (GPU) vs f64 (oracle) value, so
+                # they agree within the tolerance, not code for code
+                for p in range(CTX, pos + 1):
+                    assert max(rel_err_rows(X[:, p].astype(np.float64), R[:, p].astype(np.float64))) <= TOL
+                assert np.array_equal(X[:, :CTX], R[:, :CTX])          # prefilled rows untouched
     assert st.committed_len == CTX + 2
 
 
