@@ -60,7 +60,7 @@ typedef enum { STAGE_Q4_0 = 2, STAGE_Q8_0 = 8 } stage_qtype;
 /* Model shape.  Supported: hidden, ffn multiples of 256; dn_dim == 128;
  * dn_v_heads a multiple of dn_k_heads; att_dim == 256; rope_dims == 64;
  * att_q_heads a multiple of att_kv_heads with att_q_heads/att_kv_heads <= 7;
- * max_ctx >= 16.  The 27B hybrid: 5120, 17408, 16, 48, 128, 24, 4, 256, 64,
+ * 16 <= max_ctx <= 262144.  The 27B hybrid: 5120, 17408, 16, 48, 128, 24, 4, 256, 64,
  * 1e7, 1e-6, 4. */
 typedef struct {
   int hidden;          /* H: width of the hidden state */

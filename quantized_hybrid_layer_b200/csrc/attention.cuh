@@ -17,7 +17,7 @@
 // uses the rounded values, exactly what a later pass reads back.
 #pragma once
 
-#include "common.cuh"
+#include "qact.cuh"
 
 namespace qhl {
 
@@ -41,8 +41,10 @@ struct AttnArgs {
   float* pl;               // [NT][Hq][nchunk]: chunk sum of exp
   float* po;               // [NT][Hq][nchunk][256]: chunk sum of exp * v
   int nchunk;
-  float* out;              // [NT][out_stride] gated output
+  float* out;              // optional f32 gated output [NT][out_stride]
   int out_stride;
+  uint8_t* qout;           // gated output in block fixed point (the out-projection's input)
+  int qout_stride;
 };
 
 template <int NT>
@@ -50,7 +52,8 @@ constexpr int attn_smem_bytes(int rep) {
   return 2 * kAttChunk * kAttDim * 2            // K, V chunk (f16)
          + NT * rep * kAttDim * 4               // normalised, rotated queries
          + NT * rep * kAttChunk * 4             // scores / probabilities
-         + 8 * kAttDim * 4;                     // per-warp scratch vector
+         + 8 * kAttDim * 4                      // per-warp scratch vector
+         + 16;                                  // mbarrier
 }
 
 // RMSNorm over one 256-wide head vector held as 8 values per lane (dims 8l..8l+7)
@@ -91,6 +94,7 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
   float* qs = reinterpret_cast<float*>(Vs + kAttChunk * kAttDim);   // [NT*rep][256]
   float* sc = qs + NT * rep * kAttDim;                                 // [NT*rep][64]
   float* scratch = sc + NT * rep * kAttChunk;                          // [8][256]
+  uint64_t* kvbar = reinterpret_cast<uint64_t*>(scratch + 8 * kAttDim);
 
   const int c = blockIdx.x, g = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -102,15 +106,20 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
   const int nkeys = min(kAttChunk, ctx_end - k0);           // rows this chunk covers for any token
   const int n_old = max(0, min(kAttChunk, pos - k0));        // rows already in the cache
 
-  // cached rows do not depend on this pass: load them before the dependency wait
-  {
-    const uint4* Kg = reinterpret_cast<const uint4*>(a.K + ((size_t)g * a.max_ctx + k0) * kAttDim);
-    const uint4* Vg = reinterpret_cast<const uint4*>(a.V + ((size_t)g * a.max_ctx + k0) * kAttDim);
-    for (int i = tid; i < n_old * (kAttDim / 8); i += 256) {
-      reinterpret_cast<uint4*>(Ks)[i] = Kg[i];
-      reinterpret_cast<uint4*>(Vs)[i] = Vg[i];
+  // cached rows do not depend on this pass: two bulk copies (rows are
+  // contiguous per KV head) requested before the dependency wait
+  const uint32_t bar = smem_u32(kvbar);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    if (n_old > 0) {
+      const uint32_t bytes = (uint32_t)n_old * kAttDim * 2;
+      mbar_arrive_expect_tx(bar, 2 * bytes);
+      bulk_g2s_plain(smem_u32(Ks), a.K + ((size_t)g * a.max_ctx + k0) * kAttDim, bytes, bar);
+      bulk_g2s_plain(smem_u32(Vs), a.V + ((size_t)g * a.max_ctx + k0) * kAttDim, bytes, bar);
     }
   }
+  __syncthreads();   // barrier initialised before anyone waits on it
   pdl_wait();
 
   float* vec = scratch + warp * kAttDim;
@@ -153,6 +162,7 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
     reinterpret_cast<float4*>(qs + job * kAttDim)[2 * lane + 1] = reinterpret_cast<const float4*>(vec)[2 * lane + 1];
     __syncwarp();
   }
+  if (n_old > 0) mbar_wait(bar, 0, nullptr);
   __syncthreads();
 
   // scores q.k / 16: warp w takes rows 8w .. 8w+7, lanes split the 256 dims
@@ -228,25 +238,48 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
 }
 
 // Combine the chunk partials of one (token, query head) in chunk order and
-// apply the sigmoid output gate.  Thread = dim.
+// apply the sigmoid output gate.  Thread = dim.  The per-chunk statistics are
+// staged in shared memory and the weighted sums' loads are issued in batches
+// ahead of the (in-order) accumulation, so the kernel is not a chain of
+// dependent L2 round trips.
 template <int NT>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnArgs a) {
+  extern __shared__ float cs[];                  // [nchunk] max, [nchunk] weight, [nchunk] sum
   const int t = blockIdx.x / a.Hq, head = blockIdx.x % a.Hq, dim = threadIdx.x;
   if (threadIdx.x == 0) pdl_launch();
   const int pos = *a.kv_len;
   pdl_wait();
   const int nc = (pos + t + 1 + kAttChunk - 1) / kAttChunk;
   const size_t base = ((size_t)t * a.Hq + head) * a.nchunk;
+  float* cm = cs;
+  float* cw = cs + a.nchunk;
+  float* cl = cs + 2 * a.nchunk;
+  for (int c = threadIdx.x; c < nc; c += 256) {
+    cm[c] = a.pm[base + c];
+    cl[c] = a.pl[base + c];
+  }
+  __syncthreads();
   float M = -INFINITY;
-  for (int c = 0; c < nc; ++c) M = fmaxf(M, a.pm[base + c]);
+  for (int c = 0; c < nc; ++c) M = fmaxf(M, cm[c]);
+  for (int c = threadIdx.x; c < nc; c += 256) cw[c] = expf(__fsub_rn(cm[c], M));
+  __syncthreads();
   float L = 0.f, O = 0.f;
-  for (int c = 0; c < nc; ++c) {
-    const float w = expf(__fsub_rn(a.pm[base + c], M));
-    L = __fmaf_rn(a.pl[base + c], w, L);
-    O = __fmaf_rn(a.po[(base + c) * kAttDim + dim], w, O);
+  for (int c = 0; c < nc; ++c) L = __fmaf_rn(cl[c], cw[c], L);
+  constexpr int B = 16;
+  const float* po = a.po + base * kAttDim + dim;
+  for (int c0 = 0; c0 < nc; c0 += B) {
+    float v[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) v[j] = c0 + j < nc ? __ldg(po + (size_t)(c0 + j) * kAttDim) : 0.f;
+#pragma unroll
+    for (int j = 0; j < B; ++j)
+      if (c0 + j < nc) O = __fmaf_rn(v[j], cw[c0 + j], O);
   }
   const float gate = a.y[(size_t)t * a.y_stride + a.Hq * kAttDim + head * kAttDim + dim];
-  a.out[(size_t)t * a.out_stride + head * kAttDim + dim] = __fmul_rn(__fdiv_rn(O, L), sigmoidf_(gate));
+  const float r = __fmul_rn(__fdiv_rn(O, L), sigmoidf_(gate));
+  if (a.out) a.out[(size_t)t * a.out_stride + head * kAttDim + dim] = r;
+  if (a.qout)   // warp w holds dims 32w..32w+31: one block
+    qact_store_block(r, a.qout + (size_t)t * a.qout_stride, head * (kAttDim / 32) + (dim >> 5), dim & 31);
 }
 
 }  // namespace qhl

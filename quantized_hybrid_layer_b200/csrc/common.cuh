@@ -130,7 +130,15 @@ QHL_DEV float sumsq64(const float* v) {
 // 1 / sqrt(mean + eps) from per-tile partial sums, summed in tile order.
 QHL_DEV float rstd_from_partials(const float* ss, int ntiles, float inv_dim, float eps) {
   float s = 0.f;
-  for (int i = 0; i < ntiles; ++i) s = __fadd_rn(s, ss[i]);
+  constexpr int B = 16;   // loads issued in batches ahead of the in-order sum
+  for (int i0 = 0; i0 < ntiles; i0 += B) {
+    float v[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) v[j] = i0 + j < ntiles ? ss[i0 + j] : 0.f;
+#pragma unroll
+    for (int j = 0; j < B; ++j)
+      if (i0 + j < ntiles) s = __fadd_rn(s, v[j]);
+  }
   return __frcp_rn(__fsqrt_rn(__fadd_rn(__fmul_rn(s, inv_dim), eps)));
 }
 

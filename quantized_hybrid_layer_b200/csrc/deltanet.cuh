@@ -10,7 +10,8 @@
 //     S_i <- alpha S_i + beta (v_i - alpha (S_i . k)) k,   o_i = S_i . q
 //
 // Each warp keeps 4 rows of one head's 128x128 f32 state in registers (lane l
-// holds columns 4l..4l+3) for all NT tokens, so the state is read from HBM once
+// holds columns 4l..4l+3) for all NT tokens (8 warps = 32 rows per CTA, so a
+// CTA owns whole 32-value output blocks), so the state is read from HBM once
 // and written once per token as the snapshot S_t used for exact rollback
 // (SwarmLLM README: batched verify "with exact rollback of the recurrent
 // state").  The state rows are loaded before griddepcontrol.wait, overlapping
@@ -19,7 +20,7 @@
 // same whatever NT is.
 #pragma once
 
-#include "common.cuh"
+#include "qact.cuh"
 
 namespace qhl {
 
@@ -37,8 +38,10 @@ struct DnArgs {
   int ring_size;
   const int* cur;
   const float* s_in;
-  float* o;                // [NT][o_stride], o_stride >= Hv * 128
+  float* o;                // optional f32 output [NT][o_stride], o_stride >= Hv * 128
   int o_stride;
+  uint8_t* qo;             // optional output in block fixed point (the out-projection's input)
+  int qo_stride;
 };
 
 QHL_DEV float dot4(float4 a, float4 b) {
@@ -49,10 +52,11 @@ QHL_DEV float dot4(float4 a, float4 b) {
 }
 
 template <int NT>
-__global__ void __launch_bounds__(128) dn_step_kernel(const DnArgs a) {
+__global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
+  __shared__ float ob[NT][32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x >> 3;                       // 8 CTAs of 16 rows per head
-  const int row0 = (blockIdx.x & 7) * 16 + warp * 4;
+  const int h = blockIdx.x >> 2;                       // 4 CTAs of 32 rows per head
+  const int row0 = (blockIdx.x & 3) * 32 + warp * 4;
   const int g = h / (a.Hv / a.Hk);
   if (threadIdx.x == 0) pdl_launch();
 
@@ -91,9 +95,17 @@ __global__ void __launch_bounds__(128) dn_step_kernel(const DnArgs a) {
       S[r].z = __fmaf_rn(coef, k.z, __fmul_rn(alpha, S[r].z));
       S[r].w = __fmaf_rn(coef, k.w, __fmul_rn(alpha, S[r].w));
       const float o = warp_sum(dot4(S[r], q));
-      if (lane == 0) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
+      if (lane == 0) {
+        ob[t][warp * 4 + r] = o;
+        if (a.o) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
+      }
       reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = S[r];
     }
+  }
+  if (a.qo) {
+    __syncthreads();
+    for (int t = warp; t < NT; t += 8)
+      qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (blockIdx.x & 3), lane);
   }
 }
 

@@ -4,6 +4,16 @@
 namespace qhl {
 namespace {
 
+// Every stage kernel asks for the full shared-memory carveout, so consecutive
+// kernels never need the SM reconfigured and can share it under programmatic
+// dependent launch.
+template <typename K>
+cudaError_t set_carveout(K k, cudaFuncAttribute, int smem) {
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
+}
+
 template <int NT, int EPI>
 cudaError_t one(const GemvArgs& a, int grid, cudaStream_t s, bool pdl) {
   return launch_ex(qgemv_kernel<kQ8_0, NT, EPI>, dim3(grid), dim3(kGemvThreads),
@@ -13,9 +23,9 @@ cudaError_t one(const GemvArgs& a, int grid, cudaStream_t s, bool pdl) {
 template <int NT>
 cudaError_t prep() {
   const int smem = gemv_smem_bytes<kQ8_0, NT>();
-  cudaError_t e = cudaFuncSetAttribute(qgemv_kernel<kQ8_0, NT, EPI_STORE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(qgemv_kernel<kQ8_0, NT, EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(qgemv_kernel<kQ8_0, NT, EPI_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = set_carveout(qgemv_kernel<kQ8_0, NT, EPI_STORE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = set_carveout(qgemv_kernel<kQ8_0, NT, EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = set_carveout(qgemv_kernel<kQ8_0, NT, EPI_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   return e;
 }
 

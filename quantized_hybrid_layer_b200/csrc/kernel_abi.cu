@@ -31,6 +31,8 @@ int cuda_err(const char* what, cudaError_t e) {
 struct GemvScratch {
   bool ready = false;
   int sms = 0;
+  uint8_t* qx = nullptr;    // the input in block fixed point
+  size_t qx_cap = 0;
   float* partials = nullptr;
   int* counters = nullptr;
   int counter_cap = 0;
@@ -40,7 +42,7 @@ struct GemvScratch {
 std::mutex g_mu;
 std::vector<GemvScratch> g_scratch;
 
-int get_scratch(int tiles, int qt, GemvScratch** out) {
+int get_scratch(int tiles, int qt, size_t qx_bytes, GemvScratch** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_err("cudaGetDevice", e);
@@ -65,6 +67,16 @@ int get_scratch(int tiles, int qt, GemvScratch** out) {
     }
     s.counters = c;
     s.counter_cap = tiles;
+  }
+  if (qx_bytes > s.qx_cap) {
+    uint8_t* q = nullptr;
+    if ((e = cudaMalloc(&q, qx_bytes)) != cudaSuccess) return cuda_err("cudaMalloc", e);
+    if (s.qx) {
+      cudaDeviceSynchronize();
+      cudaFree(s.qx);
+    }
+    s.qx = q;
+    s.qx_cap = qx_bytes;
   }
   if (!s.prepared[qt]) {
     if ((e = gemv_prepare(qt)) != cudaSuccess) return cuda_err("gemv_prepare", e);
@@ -115,14 +127,16 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
     return err(STAGE_E_ARG, "qhl_qgemv: packed_dev and x_dev must be 16-byte aligned");
   const int tiles = packed_tiles(rows, false);
   GemvScratch* s = nullptr;
-  int rc = get_scratch(tiles, qtype, &s);
+  int rc = get_scratch(tiles, qtype, (size_t)n_tok * qact_row_bytes(cols), &s);
   if (rc) return rc;
+  cudaError_t e = launch_quantize_rows(x_dev, n_tok, cols, s->qx, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_err("quantize launch", e);
   GemvArgs a = {};
   a.W = static_cast<const uint8_t*>(packed_dev);
   a.tiles = tiles;
   a.chunks = cols / kChunkCols;
-  a.x = x_dev;
-  a.x_stride = cols;
+  a.qx = s->qx;
+  a.qx_stride = (int)qact_row_bytes(cols);
   a.y = y_dev;
   a.y_stride = rows;
   a.out_valid = rows;
@@ -133,7 +147,7 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
   a.err = s->err;
   const long long items = (long long)a.tiles * a.chunks;
   a.workers = (int)(items < (long long)kCtasPerSm * s->sms ? items : (long long)kCtasPerSm * s->sms);
-  cudaError_t e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, static_cast<cudaStream_t>(stream), false);
+  e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, static_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? 0 : cuda_err("qgemv launch", e);
 }
 
@@ -154,7 +168,7 @@ int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float
   d.s_in = s_in_dev;
   d.o = o_dev;
   d.o_stride = Hv * kDnDim;
-  cudaError_t e = launch_dn_step(n_tok, d, Hv * (kDnDim / 16), static_cast<cudaStream_t>(stream), false);
+  cudaError_t e = launch_dn_step(n_tok, d, Hv * (kDnDim / 32), static_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? 0 : cuda_err("deltanet launch", e);
 }
 

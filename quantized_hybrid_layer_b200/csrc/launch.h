@@ -41,8 +41,9 @@ cudaError_t mixers_prepare(int rep);   // rep = query heads per KV head
 cudaError_t launch_dn_step(int nt, const DnArgs& a, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_attn_partial(int nt, const AttnArgs& a, int nchunk, int hkv, cudaStream_t s, bool pdl);
 cudaError_t launch_attn_combine(int nt, const AttnArgs& a, cudaStream_t s, bool pdl);
-cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, float* z, float* ss,
-                               int ss_stride, cudaStream_t s);
+cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, uint8_t* qz, int qz_stride,
+                               float* ss, int ss_stride, cudaStream_t s);
+cudaError_t launch_quantize_rows(const float* x, int n, int cols, uint8_t* qx, cudaStream_t s);
 
 cudaError_t launch_repack(int qt, const uint8_t* a, const uint8_t* b, int rows, int cols, uint8_t* out,
                           cudaStream_t s);

@@ -23,24 +23,50 @@ int gemv_smem(int qt, int nt) { return qt == kQ4_0 ? gemv_smem_4(nt) : gemv_smem
 #define QHL_NT_CASES(X) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
 
 // ---------------------------------------------------------------------------
-// stage input: z = h * gamma (the first layer's RMSNorm weight) and per-tile
-// sums of squares of h, exactly as the residual epilogue of the GEMV writes
-// them, so a stage that starts at layer L gives the same bits as the same
-// layers inside a longer stage.
+// stage input: z = h * gamma (the first layer's RMSNorm weight) in block fixed
+// point and per-tile sums of squares of h, exactly as the residual epilogue of
+// the GEMV writes them, so a stage that starts at layer L gives the same bits
+// as the same layers inside a longer stage.
 template <int NT>
-__global__ void __launch_bounds__(256) stage_input_kernel(const float* h, int H, const float* gamma, float* z,
-                                                          float* ss, int ss_stride) {
+__global__ void __launch_bounds__(256) stage_input_kernel(const float* h, int H, const float* gamma, uint8_t* qz,
+                                                          int qz_stride, float* ss, int ss_stride) {
   __shared__ float sm[NT * 64];
   if (threadIdx.x == 0) pdl_launch();
-  const int tile = blockIdx.x;
+  const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int idx = threadIdx.x; idx < NT * 64; idx += blockDim.x) {
     const int t = idx >> 6, gr = tile * 64 + (idx & 63);
-    const float v = h[(size_t)t * H + gr];
-    z[(size_t)t * H + gr] = __fmul_rn(v, gamma[gr]);
-    sm[idx] = v;
+    sm[idx] = h[(size_t)t * H + gr];
   }
   __syncthreads();
+  for (int p = warp; p < NT * 2; p += 8) {
+    const int t = p >> 1, b = p & 1, gr = tile * 64 + b * 32 + lane;
+    qact_store_block(__fmul_rn(sm[t * 64 + b * 32 + lane], gamma[gr]), qz + (size_t)t * qz_stride, tile * 2 + b, lane);
+  }
   if (threadIdx.x < NT) ss[(size_t)threadIdx.x * ss_stride + tile] = sumsq64(sm + threadIdx.x * 64);
+}
+
+// f32 rows -> block fixed point, one warp per (token, 32-column block).
+__global__ void quantize_rows_kernel(const float* x, int n, int cols, uint8_t* qx) {
+  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31, nb = cols / 32;
+  if (gw >= (long long)n * nb) return;
+  const int t = (int)(gw / nb), b = (int)(gw % nb);
+  qact_store_block(x[(size_t)t * cols + b * 32 + lane], qx + (size_t)t * qact_row_bytes(cols), b, lane);
+}
+
+cudaError_t launch_quantize_rows(const float* x, int n, int cols, uint8_t* qx, cudaStream_t s) {
+  const long long warps = (long long)n * (cols / 32);
+  quantize_rows_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(x, n, cols, qx);
+  return cudaGetLastError();
+}
+
+__global__ void commit_kernel(int* ctrl, int n_accepted, int n_dn, int ring);
+
+// Full shared-memory carveout for every stage kernel (see gemv_q4.cu), and the
+// attention kernel's dynamic shared-memory limit.
+template <typename K>
+static cudaError_t max_carveout(K k) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
 }
 
 cudaError_t mixers_prepare(int rep) {
@@ -48,15 +74,20 @@ cudaError_t mixers_prepare(int rep) {
 #define P(N)                                                                                            \
   if (e == cudaSuccess)                                                                                 \
     e = cudaFuncSetAttribute(attn_partial_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
-                             attn_smem_bytes<N>(rep));
+                             attn_smem_bytes<N>(rep));                                                  \
+  if (e == cudaSuccess) e = max_carveout(attn_partial_kernel<N>);                                       \
+  if (e == cudaSuccess) e = max_carveout(attn_combine_kernel<N>);                                       \
+  if (e == cudaSuccess) e = max_carveout(dn_step_kernel<N>);                                            \
+  if (e == cudaSuccess) e = max_carveout(stage_input_kernel<N>);
   QHL_NT_CASES(P)
 #undef P
+  if (e == cudaSuccess) e = max_carveout(commit_kernel);
   return e;
 }
 
 cudaError_t launch_dn_step(int nt, const DnArgs& a, int grid, cudaStream_t s, bool pdl) {
   switch (nt) {
-#define C(N) case N: return launch_ex(dn_step_kernel<N>, dim3(grid), dim3(128), 0, s, pdl, a);
+#define C(N) case N: return launch_ex(dn_step_kernel<N>, dim3(grid), dim3(256), 0, s, pdl, a);
     QHL_NT_CASES(C)
 #undef C
     default: return cudaErrorInvalidValue;
@@ -78,17 +109,17 @@ cudaError_t launch_attn_partial(int nt, const AttnArgs& a, int nchunk, int hkv, 
 
 cudaError_t launch_attn_combine(int nt, const AttnArgs& a, cudaStream_t s, bool pdl) {
   switch (nt) {
-#define C(N) case N: return launch_ex(attn_combine_kernel<N>, dim3(N * a.Hq), dim3(256), 0, s, pdl, a);
+#define C(N) case N: return launch_ex(attn_combine_kernel<N>, dim3(N * a.Hq), dim3(256), (size_t)3 * a.nchunk * 4, s, pdl, a);
     QHL_NT_CASES(C)
 #undef C
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, float* z, float* ss,
-                               int ss_stride, cudaStream_t s) {
+cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, uint8_t* qz, int qz_stride,
+                               float* ss, int ss_stride, cudaStream_t s) {
   switch (nt) {
-#define C(N) case N: return launch_ex(stage_input_kernel<N>, dim3(H / 64), dim3(256), 0, s, false, h, H, gamma, z, ss, ss_stride);
+#define C(N) case N: return launch_ex(stage_input_kernel<N>, dim3(H / 64), dim3(256), 0, s, false, h, H, gamma, qz, qz_stride, ss, ss_stride);
     QHL_NT_CASES(C)
 #undef C
     default: return cudaErrorInvalidValue;
@@ -130,7 +161,7 @@ __global__ void repack_kernel(int qt, const uint8_t* a, const uint8_t* b, int ro
   } else {
     for (int half = 0; half < 2; ++half) {
       uint8_t* q = base + (((blk * 2 + half) * 2 + h) * 32 + lane) * 16;
-      for (int i = 0; i < 16; ++i) q[i] = valid ? (uint8_t)(sp[2 + 16 * half + i] ^ 0x80) : 0x80;
+      for (int i = 0; i < 16; ++i) q[i] = valid ? sp[2 + 16 * half + i] : 0;
     }
     uint8_t* s = base + 16384 + (blk * 32 + lane) * 4 + h * 2;
     s[0] = valid ? sp[0] : 0;

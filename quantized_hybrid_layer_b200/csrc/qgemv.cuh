@@ -3,32 +3,38 @@
 // y[t][r] = sum_c x[t][c] * W[r][c] for n_tok = NT tokens (1..16), the
 // projection every layer of the stage streams: "every token reads all of the
 // weights once" (SwarmLLM README, paragraph after the peer diagram).  Decode is
-// memory-bound, so the kernel is built to keep HBM busy:
+// memory-bound, so the kernel is built to keep HBM busy and the SM's integer
+// and FP pipes well below their limits:
 //
-//  * Persistent stream-K grid, one CTA per SM.  The (tile, chunk) items of the
+//  * Persistent stream-K grid, two CTAs per SM.  The (tile, chunk) items of the
 //    packed matrix are split into contiguous equal ranges, one per CTA, so every
 //    SM streams the same number of bytes whatever the matrix shape.
 //  * One producer warp per CTA moves items (64 rows x 256 columns, one
-//    contiguous record) into a ring of shared-memory stages with bulk async
-//    copies (cp.async.bulk + mbarrier, L2 evict-first).  The weights never
-//    depend on the previous kernel, so the producer starts before
-//    griddepcontrol.wait: under programmatic dependent launch the next
-//    projection's weights are in flight while the previous kernel drains.
-//  * Eight consumer warps; warp w dequantises block w of each item.  Lane l
-//    owns tile rows l and l + 32, so the x values are warp-uniform broadcast
-//    loads and no cross-lane reduction is needed.  Nibbles/bytes become floats
-//    exactly (mask-or into 2^23, one packed FMA), products are accumulated with
-//    packed f32x2 FMAs, and the per-block f16 scale is applied once per block.
-//  * Reduction order is fixed and independent of NT: per row, blocks in item
-//    order inside a warp, then warps 0..7, then CTAs in grid order (stream-K
-//    partials, combined by whichever CTA finishes a tile last).  Each token's
-//    sum is computed by exactly the same operations whatever NT is, so a
-//    16-token pass is bit-identical to 16 single-token passes.
+//    contiguous record) and the matching x columns into a ring of shared-memory
+//    stages with bulk async copies (cp.async.bulk + mbarrier, L2 evict-first for
+//    weights).  The weights never depend on the previous kernel, so the first
+//    stages are requested before griddepcontrol.wait: under programmatic
+//    dependent launch a projection's weights stream in while the previous
+//    kernel drains.
+//  * Eight consumer warps; warp w handles block w of each item.  Lane l owns
+//    tile rows l and l + 32, so x is read as warp-uniform broadcasts and no
+//    cross-lane reduction is needed.  x arrives in block fixed-point form
+//    (qact.cuh): each block's sum_j q_j X_j is formed exactly in int32 with
+//    byte dot products (dp4a) against the 4-bit (or 8-bit) quants, and one FMA
+//    per block adds d * s * sum to the row's f32 accumulator.
+//  * Reduction order is fixed and independent of NT: per row, exact integer
+//    block sums, blocks in item order inside a warp, then warps 0..7, then CTAs
+//    in grid order (stream-K partials, combined by whichever CTA finishes a tile
+//    last).  Each token's result is produced by the same operations whatever NT
+//    is, so a 16-token pass is bit-identical to 16 single-token passes.
 //  * Fused epilogues: input RMS scale (RMSNorm folded as rstd * sum(z W) with
-//    z = h * gamma written by the producer of h), SwiGLU on paired gate/up
-//    rows, residual add with the next RMSNorm's z and per-tile sum of squares.
+//    z = h * gamma written by the producer of h), SwiGLU on paired gate/up rows
+//    writing the down projection's input in block fixed-point form, and the
+//    residual add writing h, the next RMSNorm's z (block fixed point) and its
+//    per-tile sums of squares.
 #pragma once
 
+#include "qact.cuh"
 #include "qpack.cuh"
 
 namespace qhl {
@@ -38,18 +44,18 @@ enum Epi : int { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_RESID = 2 };
 struct GemvArgs {
   const uint8_t* W;        // packed items, tile-major
   int tiles, chunks;       // item grid: tiles x chunks
-  const float* x;          // [NT][x_stride] input (z for normed inputs)
-  int x_stride;
-  float* y;                // STORE / SWIGLU output; RESID: residual stream (in/out)
+  const uint8_t* qx;       // input in block fixed point: [NT][qx_stride bytes]
+  int qx_stride;
+  float* y;                // STORE: f32 output [NT][y_stride]; RESID: residual stream h (in/out)
   int y_stride;
   int out_valid;           // STORE/RESID: valid rows; SWIGLU: valid features
+  uint8_t* qout;           // SWIGLU: silu(g)*u; RESID: h_new * gamma_next (block fixed point), or null
+  int qout_stride;
   const float* ss_in;      // optional per-tile sums of squares of the pre-norm input: [NT][ss_stride]
   int ss_tiles, ss_stride;
   float inv_dim, eps;      // rstd = 1 / sqrt(sum(ss) * inv_dim + eps)
-  const float* gamma_next; // RESID: next RMSNorm weight (z_out = h_new * gamma_next)
-  float* z_out;
-  int z_stride;
-  float* ss_out;           // RESID: per-tile sum of squares of h_new, [NT][ss_out_stride]
+  const float* gamma_next; // RESID: next RMSNorm weight
+  float* ss_out;           // RESID: per-tile sum of squares of h_new, [NT][ss_out_stride], or null
   int ss_out_stride;
   float* partials;         // stream-K scratch: [2 * workers][NT][64]
   int* counters;           // stream-K tile counters, zero between launches
@@ -63,14 +69,14 @@ constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 // (the split, and hence the summation order, must not depend on NT).
 constexpr int kCtasPerSm = 2;
 
-// A stage holds one item's packed weights followed by the item's x columns for
-// every token ([NT][256] f32).  Up to 2 tokens the ring is small enough for two
-// CTAs of this kernel plus one of the next (under programmatic dependent
+// A stage holds one item's packed weights followed by the item's x chunk for
+// every token ([NT][864] bytes).  Up to 2 tokens the ring is small enough for
+// two CTAs of this kernel plus one of the next (under programmatic dependent
 // launch) to share an SM; up to 4 tokens two CTAs fit; beyond that one CTA per
 // SM runs at a time.
 template <int QT, int NT>
 struct GemvCfg {
-  static constexpr int kStageBytes = QLayout<QT>::kItemBytes + NT * kChunkCols * 4;
+  static constexpr int kStageBytes = QLayout<QT>::kItemBytes + NT * kQChunkBytes;
   static constexpr int kBudget = NT <= 2 ? 72 * 1024 : (NT <= 4 ? 104 * 1024 : 196 * 1024);
   static constexpr int kRaw = (kBudget - kConsumerWarps * NT * 64 * 4 - 512) / kStageBytes;
   static constexpr int kStages = kRaw < 3 ? 3 : (kRaw > 12 ? 12 : kRaw);
@@ -119,81 +125,107 @@ QHL_DEV void load_item(const uint8_t* st, int warp, int lane, ItemRegs<QT>& r) {
   r.sc = *reinterpret_cast<const uint32_t*>(st + QLayout<QT>::kQuantBytes + (warp * 32 + lane) * 4);
 }
 
-// Accumulate one block for both rows and all NT tokens.  Per token and row the
-// operation sequence is fixed: packed FMAs over the block's element pairs in
-// word order, the two lanes added, then one FMA with the block scale.
+// x words of one block: 8 words per byte plane (word k = elements 4k..4k+3).
+struct XBlock { uint32_t hi[8], mid[8], lo[8]; float s; int s_hi, s_ml; };
+
+QHL_DEV void load_xblock(const uint8_t* xt, int warp, XBlock& x) {
+  const uint4* ph = reinterpret_cast<const uint4*>(xt + warp * 32);
+  const uint4* pm = reinterpret_cast<const uint4*>(xt + 256 + warp * 32);
+  const uint4* pl = reinterpret_cast<const uint4*>(xt + 512 + warp * 32);
+  const uint4 h0 = ph[0], h1 = ph[1], m0 = pm[0], m1 = pm[1], l0 = pl[0], l1 = pl[1];
+  x.hi[0] = h0.x; x.hi[1] = h0.y; x.hi[2] = h0.z; x.hi[3] = h0.w;
+  x.hi[4] = h1.x; x.hi[5] = h1.y; x.hi[6] = h1.z; x.hi[7] = h1.w;
+  x.mid[0] = m0.x; x.mid[1] = m0.y; x.mid[2] = m0.z; x.mid[3] = m0.w;
+  x.mid[4] = m1.x; x.mid[5] = m1.y; x.mid[6] = m1.z; x.mid[7] = m1.w;
+  x.lo[0] = l0.x; x.lo[1] = l0.y; x.lo[2] = l0.z; x.lo[3] = l0.w;
+  x.lo[4] = l1.x; x.lo[5] = l1.y; x.lo[6] = l1.z; x.lo[7] = l1.w;
+  x.s = reinterpret_cast<const float*>(xt + 768)[warp];
+  x.s_hi = reinterpret_cast<const int*>(xt + 800)[warp];
+  x.s_ml = reinterpret_cast<const int*>(xt + 832)[warp];
+}
+
+// acc = fma(d * s, 65536 * H + ML, acc): the block's exact integer partial sums
+// turned into one f32 update by a fixed sequence of operations.
+QHL_DEV float block_update(float d, float s, int H, int ML, float acc) {
+  const float v = __fmaf_rn(__int2float_rn(H), 65536.f, __int2float_rn(ML));
+  return __fmaf_rn(__fmul_rn(d, s), v, acc);
+}
+
+// One block for both rows and all NT tokens.
 template <int QT, int NT>
-QHL_DEV void compute_item(const ItemRegs<QT>& r, const float* xcol, float (&r0)[NT], float (&r1)[NT]) {
-  constexpr int x_stride = kChunkCols;   // x chunk in shared memory: [NT][256]
-  float2 a0[NT], a1[NT];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) { a0[t] = make_float2(0.f, 0.f); a1[t] = make_float2(0.f, 0.f); }
+QHL_DEV void compute_item(const ItemRegs<QT>& r, const uint8_t* xs, int warp, float (&r0)[NT], float (&r1)[NT]) {
+  const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(r.sc & 0xFFFFu)));
+  const float d1 = __half2float(__ushort_as_half(static_cast<unsigned short>(r.sc >> 16)));
   if constexpr (QT == kQ4_0) {
+    // low nibbles of word i are elements 4i..4i+3, high nibbles 16+4i..16+4i+3
+    uint32_t qa[8], qb[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float2 p[4], q[4];
-      q4_word(r.a[i], p);
-      q4_word(r.b[i], q);
+      qa[i] = r.a[i] & 0x0F0F0F0Fu;
+      qa[4 + i] = (r.a[i] >> 4) & 0x0F0F0F0Fu;
+      qb[i] = r.b[i] & 0x0F0F0F0Fu;
+      qb[4 + i] = (r.b[i] >> 4) & 0x0F0F0F0Fu;
+    }
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float4* xv = reinterpret_cast<const float4*>(xcol + t * x_stride);
-        const float4 xa = xv[i];
-        const float4 xb = xv[4 + i];
-        const float2 x0 = make_float2(xa.x, xa.y), x1 = make_float2(xa.z, xa.w);
-        const float2 x2 = make_float2(xb.x, xb.y), x3 = make_float2(xb.z, xb.w);
-        a0[t] = ffma2(p[0], x0, a0[t]);
-        a0[t] = ffma2(p[1], x1, a0[t]);
-        a0[t] = ffma2(p[2], x2, a0[t]);
-        a0[t] = ffma2(p[3], x3, a0[t]);
-        a1[t] = ffma2(q[0], x0, a1[t]);
-        a1[t] = ffma2(q[1], x1, a1[t]);
-        a1[t] = ffma2(q[2], x2, a1[t]);
-        a1[t] = ffma2(q[3], x3, a1[t]);
+    for (int t = 0; t < NT; ++t) {
+      XBlock x;
+      load_xblock(xs + t * kQChunkBytes, warp, x);
+      int H0 = 0, M0 = 0, L0 = 0, H1 = 0, M1 = 0, L1 = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {        // q in 0..15: signed x signed is exact for hi
+        H0 = dp4a_ss(qa[k], x.hi[k], H0);
+        M0 = dp4a_uu(qa[k], x.mid[k], M0);
+        L0 = dp4a_uu(qa[k], x.lo[k], L0);
+        H1 = dp4a_ss(qb[k], x.hi[k], H1);
+        M1 = dp4a_uu(qb[k], x.mid[k], M1);
+        L1 = dp4a_uu(qb[k], x.lo[k], L1);
       }
+      // sum_j (q_j - 8) X_j = 65536 (H - 8 sum hi) + (256 M + L - 8 sum ml)
+      r0[t] = block_update(d0, x.s, H0 - 8 * x.s_hi, M0 * 256 + L0 - 8 * x.s_ml, r0[t]);
+      r1[t] = block_update(d1, x.s, H1 - 8 * x.s_hi, M1 * 256 + L1 - 8 * x.s_ml, r1[t]);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float2 p[2], q[2];
-      q8_word(r.a[i], p);
-      q8_word(r.b[i], q);
+    for (int t = 0; t < NT; ++t) {
+      XBlock x;
+      load_xblock(xs + t * kQChunkBytes, warp, x);
+      int H0 = 0, M0 = 0, L0 = 0, H1 = 0, M1 = 0, L1 = 0;
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float4 xa = reinterpret_cast<const float4*>(xcol + t * x_stride)[i];
-        const float2 x0 = make_float2(xa.x, xa.y), x1 = make_float2(xa.z, xa.w);
-        a0[t] = ffma2(p[0], x0, a0[t]);
-        a0[t] = ffma2(p[1], x1, a0[t]);
-        a1[t] = ffma2(q[0], x0, a1[t]);
-        a1[t] = ffma2(q[1], x1, a1[t]);
+      for (int k = 0; k < 8; ++k) {        // word k holds signed quants 4k..4k+3
+        H0 = dp4a_ss(r.a[k], x.hi[k], H0);
+        M0 = dp4a_su(r.a[k], x.mid[k], M0);
+        L0 = dp4a_su(r.a[k], x.lo[k], L0);
+        H1 = dp4a_ss(r.b[k], x.hi[k], H1);
+        M1 = dp4a_su(r.b[k], x.mid[k], M1);
+        L1 = dp4a_su(r.b[k], x.lo[k], L1);
       }
+      r0[t] = block_update(d0, x.s, H0, M0 * 256 + L0, r0[t]);
+      r1[t] = block_update(d1, x.s, H1, M1 * 256 + L1, r1[t]);
     }
-  }
-  const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(r.sc & 0xFFFFu)));
-  const float d1 = __half2float(__ushort_as_half(static_cast<unsigned short>(r.sc >> 16)));
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    r0[t] = __fmaf_rn(d0, __fadd_rn(a0[t].x, a0[t].y), r0[t]);
-    r1[t] = __fmaf_rn(d1, __fadd_rn(a1[t].x, a1[t].y), r1[t]);
   }
 }
 
 // Epilogue for one finished tile; vals = [NT][64] final sums in shared memory.
+// Called by all 256 consumer threads.
 template <int EPI, int NT>
 QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float* rstd, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
   if constexpr (EPI == EPI_STORE) {
     for (int idx = tid; idx < NT * 64; idx += 256) {
       const int t = idx >> 6, row = idx & 63, gr = tile * 64 + row;
       if (gr < a.out_valid) a.y[(size_t)t * a.y_stride + gr] = __fmul_rn(vals[idx], rstd[t]);
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
-    for (int idx = tid; idx < NT * 32; idx += 256) {
-      const int t = idx >> 5, r = idx & 31, f = tile * 32 + r;
+    // tile rows 0..31 are gate rows of features tile*32.., rows 32..63 the matching up rows
+    for (int t = warp; t < NT; t += kConsumerWarps) {
+      const int f = tile * 32 + lane;
+      float u = 0.f;
       if (f < a.out_valid) {
-        const float g = __fmul_rn(vals[t * 64 + r], rstd[t]);
-        const float u = __fmul_rn(vals[t * 64 + 32 + r], rstd[t]);
-        const float s = __fdiv_rn(g, __fadd_rn(1.f, expf(-g)));   // silu(g) = g * sigmoid(g)
-        a.y[(size_t)t * a.y_stride + f] = __fmul_rn(s, u);
+        const float g = __fmul_rn(vals[t * 64 + lane], rstd[t]);
+        const float up = __fmul_rn(vals[t * 64 + 32 + lane], rstd[t]);
+        u = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), up);   // silu(g) * up
       }
+      qact_store_block(u, a.qout + (size_t)t * a.qout_stride, tile, lane);
     }
   } else {
     for (int idx = tid; idx < NT * 64; idx += 256) {
@@ -203,14 +235,18 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float
         float* hp = a.y + (size_t)t * a.y_stride + gr;
         hn = __fadd_rn(*hp, vals[idx]);
         *hp = hn;
-        if (a.z_out) a.z_out[(size_t)t * a.z_stride + gr] = __fmul_rn(hn, a.gamma_next[gr]);
       }
       vals[idx] = hn;
     }
-    if (a.ss_out) {
-      named_sync(1, 256);
-      if (tid < NT) a.ss_out[(size_t)tid * a.ss_out_stride + tile] = sumsq64(vals + tid * 64);
+    named_sync(1, 256);
+    if (a.qout) {
+      for (int p = warp; p < NT * 2; p += kConsumerWarps) {
+        const int t = p >> 1, b = p & 1, gr = tile * 64 + b * 32 + lane;
+        const float z = gr < a.out_valid ? __fmul_rn(vals[t * 64 + b * 32 + lane], a.gamma_next[gr]) : 0.f;
+        qact_store_block(z, a.qout + (size_t)t * a.qout_stride, tile * 2 + b, lane);
+      }
     }
+    if (a.ss_out && tid < NT) a.ss_out[(size_t)tid * a.ss_out_stride + tile] = sumsq64(vals + tid * 64);
   }
 }
 
@@ -219,7 +255,6 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
   constexpr int S = GemvCfg<QT, NT>::kStages;
   constexpr int IB = QLayout<QT>::kItemBytes;
   constexpr int SB = GemvCfg<QT, NT>::kStageBytes;
-  constexpr int XB = kChunkCols * 4;      // bytes of one token's x chunk
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* stages = smem;
   float* red = reinterpret_cast<float*>(smem + S * SB);                 // [8][NT][64]
@@ -234,6 +269,7 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
   const long long n_items = (long long)a.tiles * a.chunks;
   const long long i0 = sk_begin(cta, n_items, a.workers);
   const long long i1 = sk_begin(cta + 1, n_items, a.workers);
+  const int n_local = (int)(i1 - i0);
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -251,17 +287,15 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
     // previous kernel) follow once the dependency is resolved.
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      const int n_local = (int)(i1 - i0);
       const int pre = n_local < S ? n_local : S;
       const int c0 = (int)(i0 % a.chunks);
       auto issue_x = [&](int k, int s) {
-        // chunk of local item k: (c0 + k) mod chunks, without 64-bit division
-        int c = c0 + k;
+        int c = c0 + k;                    // chunk of local item k, without 64-bit division
         while (c >= a.chunks) c -= a.chunks;
         const uint32_t full = smem_u32(&bars[s]);
         for (int t = 0; t < NT; ++t)
-          bulk_g2s_plain(smem_u32(stages + s * SB + IB + t * XB), a.x + (size_t)t * a.x_stride + (size_t)c * kChunkCols,
-                         XB, full);
+          bulk_g2s_plain(smem_u32(stages + s * SB + IB + t * kQChunkBytes),
+                         a.qx + (size_t)t * a.qx_stride + (size_t)c * kQChunkBytes, kQChunkBytes, full);
       };
       for (int k = 0; k < pre; ++k) {
         const uint32_t full = smem_u32(&bars[k]);
@@ -283,7 +317,7 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
   }
 
   // ---------------- consumers ------------------------------------------------
-  pdl_wait();   // x, ss_in, the residual stream and the scratch come from earlier kernels
+  pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
   if (tid < NT)
     rstd[tid] = a.ss_in ? rstd_from_partials(a.ss_in + (size_t)tid * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps) : 1.f;
 
@@ -315,19 +349,23 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
       gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
     } else {
       // stream-K: publish this CTA's partial; the last contributor finishes the tile
+      // (release: the barrier orders every thread's stores before thread 0's
+      // fence and counter increment; acquire: the last arriver's fence after
+      // its increment, then the barrier, orders the partial loads after it)
       float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * 64;
       for (int idx = tid; idx < NT * 64; idx += 256) mine[idx] = red[idx];
-      __threadfence();
       named_sync(1, 256);
       const long long cf = sk_owner(t_lo, n_items, a.workers);
       const long long cl = sk_owner(t_hi - 1, n_items, a.workers);
       if (tid == 0) {
+        __threadfence();
         const int old = atomicAdd(&a.counters[tl], 1);
-        *flag = (old == (int)(cl - cf)) ? 1 : 0;
+        const int last = (old == (int)(cl - cf)) ? 1 : 0;
+        if (last) __threadfence();
+        *flag = last;
       }
       named_sync(1, 256);
       if (*flag) {
-        __threadfence();
         for (int idx = tid; idx < NT * 64; idx += 256) {
           float v = 0.f;
           for (long long c = cf; c <= cl; ++c) {
@@ -347,7 +385,6 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
   };
 
   named_sync(1, 256);   // rstd visible
-  const int n_local = (int)(i1 - i0);
   int chunk = (int)(i0 - (long long)tile * a.chunks);
   int s = 0;
   uint32_t phase = 0;
@@ -361,7 +398,7 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
     ItemRegs<QT> regs;
     const uint8_t* st = stages + s * SB;
     load_item<QT>(st, warp, lane, regs);
-    compute_item<QT, NT>(regs, reinterpret_cast<const float*>(st + IB) + warp * 32, r0, r1);
+    compute_item<QT, NT>(regs, st + IB, warp, r0, r1);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&bars[S + s]));   // stage free for the producer
     ++chunk;
@@ -370,10 +407,10 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
       phase ^= 1u;
     }
   }
-  if (i1 > i0) flush(tile);
+  if (n_local > 0) flush(tile);
   if (timed_out && lane == 0) {
     // error path: let any copy still in flight land before the CTA exits
-    for (int s = 0; s < S; ++s) mbar_wait(smem_u32(&bars[s]), 0, nullptr);
+    for (int q = 0; q < S; ++q) mbar_wait(smem_u32(&bars[q]), 0, nullptr);
   }
 }
 

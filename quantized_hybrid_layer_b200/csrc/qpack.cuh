@@ -11,9 +11,8 @@
 //
 //  Q4_0 item (9216 B):  nibbles  [block 8][h 2][lane 32][16 B]   (GGUF byte order kept)
 //                       scales   [block 8][lane 32][h 2] binary16
-//  Q8_0 item (17408 B): quants   [block 8][half 2][h 2][lane 32][16 B]  bytes 16*half.. of
-//                                the block, stored offset-binary (q + 128) so a byte
-//                                converts to float with one mask-or
+//  Q8_0 item (17408 B): quants   [block 8][half 2][h 2][lane 32][16 B]  signed bytes
+//                                16*half .. 16*half+15 of the block
 //                       scales   [block 8][lane 32][h 2] binary16
 //
 // A Q4_0 block keeps its GGUF meaning: element j (j < 16) is the low nibble of
@@ -80,12 +79,14 @@ QHL_DEV void q4_word(uint32_t w, float2 p[4]) {
   p[3] = ffma2(make_float2(magic_field<0x00F0u>(w2, m), magic_field<0xF000u>(w2, m)), s_hi, c_hi);
 }
 
-// Q8_0 (offset-binary bytes): word i holds elements 4i .. 4i+3.
-// p[0] = (e4i, e4i+1), p[1] = (e4i+2, e4i+3) as signed integers.
-QHL_DEV void q8_word(uint32_t w, float2 p[2]) {
+// Q8_0: word i holds signed elements 4i .. 4i+3.
+// p[0] = (e4i, e4i+1), p[1] = (e4i+2, e4i+3) as signed integers (the sign
+// bits are flipped to offset binary, q + 128, before the mask-or).
+QHL_DEV void q8_word(uint32_t w_signed, float2 p[2]) {
   const float2 s = make_float2(1.0f, 0.00390625f);
   const float2 c = make_float2(-8388736.0f, -32896.0f);        // -(2^23+128), -(2^15+128)
   const uint32_t m = kMagic;
+  const uint32_t w = w_signed ^ 0x80808080u;
   const uint32_t w2 = w >> 16;
   p[0] = ffma2(make_float2(magic_field<0x00FFu>(w, m), magic_field<0xFF00u>(w, m)), s, c);
   p[1] = ffma2(make_float2(magic_field<0x00FFu>(w2, m), magic_field<0xFF00u>(w2, m)), s, c);

@@ -54,7 +54,9 @@ def test_single_q4_0_gemv_1024(q):
     ref = oracle.qgemv(Q4_0, W, x)
     err = rel_err_rows(y, ref)
     assert max(err) <= TOL, err
-    assert max(err) <= 1e-5            # f32 accumulation of 1024 terms: far inside the bound
+    # x enters as 16-bit block fixed point (step <= 2^-15 of the block max): the
+    # error stays far inside the bound
+    assert max(err) <= 2e-4
 
 
 @pytest.mark.parametrize("qtype", [Q4_0, Q8_0])
