@@ -222,6 +222,26 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
 int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float* s_in_dev,
                       float* snaps_dev, float* o_dev, void* stream);
 
+/* The GEMV of qhl_qgemv for callers that cannot allocate device memory at
+ * call time: a process whose memory pool already owns the whole GPU, or a
+ * latency-critical loop that must not pay for cudaMalloc / cudaFree (which can
+ * synchronise the device).  The pages have no counterpart of this call; it
+ * exists for such callers only.  Same arguments and results as qhl_qgemv (same
+ * kernels, so the outputs are identical), but every piece of scratch lives in
+ * one static device array of about 3.6 MiB that each GPU loading this library
+ * holds until the process exits; the call itself allocates nothing.  Limits:
+ * n_tok * (cols / 256) * 864 bytes must not exceed 1 MiB (for example cols up to
+ * 19200 at 16 tokens, 310528 at 1 token), rows at most 1048576, and the device
+ * at most 160 SMs; larger problems return STAGE_E_ARG (STAGE_E_UNSUPPORTED for
+ * the SM count) before any device work.  The first call on a device looks up
+ * the array's device address and sets kernel attributes; make that first call
+ * before any stream capture.  All calls share the one array, which keeps the
+ * last call's contents (the tile counters are cleared by every call): calls
+ * that overlap on the GPU, e.g. on two streams of the same device, race and
+ * must be serialised by the caller. */
+int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* packed_dev, const float* x_dev, int n_tok,
+                      float* y_dev, void* stream);
+
 /* Message of the last failed qhl_* call on this host thread ("" if none). */
 const char* qhl_last_error(void);
 

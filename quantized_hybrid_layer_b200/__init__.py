@@ -34,7 +34,7 @@ EXPORTS = (
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
     "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_weight_bytes", "stage_last_error",
     "stage_free", "qhl_packed_bytes", "qhl_repack", "qhl_dequant", "qhl_qgemv", "qhl_deltanet_step",
-    "qhl_last_error",
+    "qhl_qgemv_noalloc", "qhl_last_error",
 )
 
 
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
             "qhl_dequant": (i, [i, i, i, vp, i, i, i, vp, vp]),
             "qhl_qgemv": (i, [i, i, i, vp, vp, i, vp, vp]),
             "qhl_deltanet_step": (i, [i, i, vp, i, vp, vp, vp, vp]),
+            "qhl_qgemv_noalloc": (i, [i, i, i, vp, vp, i, vp, vp]),
             "qhl_last_error": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -271,6 +272,13 @@ def qhl_dequant(qtype: int, rows: int, cols: int, packed, row0: int, nrows: int,
 def qhl_qgemv(qtype: int, rows: int, cols: int, packed, x, y, stream=None):
     n = x.shape[0]
     _check_qhl(lib().qhl_qgemv(qtype, rows, cols, _ptr(packed), _ptr(x), n, _ptr(y), _stream(stream)))
+
+
+def qhl_qgemv_noalloc(qtype: int, rows: int, cols: int, packed, x, y, stream=None):
+    """qhl_qgemv for callers that cannot allocate device memory: its scratch is a
+    fixed static device array, so the call allocates nothing (limits in qhl_stage.h)."""
+    n = x.shape[0]
+    _check_qhl(lib().qhl_qgemv_noalloc(qtype, rows, cols, _ptr(packed), _ptr(x), n, _ptr(y), _stream(stream)))
 
 
 def qhl_deltanet_step(Hk: int, Hv: int, y, s_in, snaps, o, stream=None):
