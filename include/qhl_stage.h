@@ -166,6 +166,25 @@ stage_status stage_set_kv_len(stage_t* st, int kv_len);
  * repacked weights dequantise bit-exactly. */
 stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst);
 
+/* How a pass runs on the device.
+ *   STAGE_PASS_PERSISTENT (default): one cooperative kernel runs the whole pass
+ *     (stage input, then every layer's projections and mixer), its phases
+ *     separated by grid-wide barriers, its CTAs streaming the next projection's
+ *     weights across phase boundaries.  Used for n_tok 1..4 when two CTAs per
+ *     SM are resident and the mixers' scratch fits (attention context of at
+ *     most ~1700 chunks of 64 rows at n_tok 1); other passes fall back to
+ *     kernels.
+ *   STAGE_PASS_KERNELS: one kernel per step, all recorded in a CUDA graph.
+ * Both run the same units with the same split and reduction order, so they
+ * give bit-identical results.  Refused while a pass is pending; waits for the
+ * stage's stream and drops the recorded graphs. */
+typedef enum { STAGE_PASS_KERNELS = 0, STAGE_PASS_PERSISTENT = 1 } stage_pass_mode;
+stage_status stage_set_pass_mode(stage_t* st, int mode);
+
+/* 1 if an n_tok-token pass would run as the persistent kernel, 0 if as a chain
+ * of kernels, -1 for a NULL stage or n_tok outside 1..16. */
+int stage_pass_persistent(stage_t* st, int n_tok);
+
 /* Bytes of weight storage the stage streams per pass (packed quants + scales). */
 size_t stage_weight_bytes(const stage_t* st);
 

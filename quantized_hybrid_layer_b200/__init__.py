@@ -32,10 +32,14 @@ STATUS = {
 EXPORTS = (
     "stage_load", "stage_forward", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
-    "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_weight_bytes", "stage_last_error",
+    "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_set_pass_mode", "stage_pass_persistent",
+    "stage_weight_bytes", "stage_last_error",
     "stage_free", "qhl_packed_bytes", "qhl_repack", "qhl_dequant", "qhl_qgemv", "qhl_deltanet_step",
     "qhl_qgemv_noalloc", "qhl_last_error",
 )
+
+
+PASS_KERNELS, PASS_PERSISTENT = 0, 1
 
 
 class StageError(RuntimeError):
@@ -86,6 +90,8 @@ def lib() -> ctypes.CDLL:
             "stage_set_kv": (i, [vp, i, vp, vp, sz]),
             "stage_set_kv_len": (i, [vp, i]),
             "stage_debug_dequant": (i, [vp, ctypes.c_char_p, i, vp]),
+            "stage_set_pass_mode": (i, [vp, i]),
+            "stage_pass_persistent": (i, [vp, i]),
             "stage_weight_bytes": (sz, [vp]),
             "stage_last_error": (ctypes.c_char_p, [vp]),
             "stage_free": (None, [vp]),
@@ -175,6 +181,15 @@ class Stage:
     @property
     def pending(self) -> int:
         return lib().stage_pending(self._h)
+
+    def set_pass_mode(self, mode: int):
+        """PASS_PERSISTENT (one cooperative kernel per pass where eligible) or
+        PASS_KERNELS (one kernel per step)."""
+        self._check(lib().stage_set_pass_mode(self._h, mode))
+
+    def pass_persistent(self, n_tok: int) -> bool:
+        """Whether an n_tok pass runs as the persistent kernel."""
+        return lib().stage_pass_persistent(self._h, n_tok) == 1
 
     @property
     def weight_bytes(self) -> int:

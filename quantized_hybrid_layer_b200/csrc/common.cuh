@@ -65,6 +65,12 @@ QHL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
   return false;
 }
 
+// Error path of a kernel that gave up waiting: idle ~200 us so that bulk copies
+// already issued into this CTA's shared memory land before the CTA leaves.
+QHL_DEV void drain_inflight_copies() {
+  for (int i = 0; i < 200; ++i) __nanosleep(1000);
+}
+
 // ---- bulk copies (non-tensor TMA) -----------------------------------------
 QHL_DEV uint64_t policy_evict_first() {
   uint64_t p;
@@ -127,18 +133,21 @@ QHL_DEV float sumsq64(const float* v) {
   return s;
 }
 
-// 1 / sqrt(mean + eps) from per-tile partial sums, summed in tile order.
-QHL_DEV float rstd_from_partials(const float* ss, int ntiles, float inv_dim, float eps) {
+// 1 / sqrt(mean + eps) from per-tile partial sums, computed by one warp: lane
+// l sums tiles l, l + 32, .. in order, then an xor butterfly (every lane gets
+// the same bits).  One round of loads instead of a chain; the summation order
+// is fixed by ntiles alone.
+QHL_DEV float rstd_warp(const float* ss, int ntiles, float inv_dim, float eps, int lane) {
+  constexpr int B = 8;   // up to 256 tiles in one round of loads
+  float v[B];
+#pragma unroll
+  for (int j = 0; j < B; ++j) v[j] = lane + 32 * j < ntiles ? __ldcg(ss + lane + 32 * j) : 0.f;
   float s = 0.f;
-  constexpr int B = 16;   // loads issued in batches ahead of the in-order sum
-  for (int i0 = 0; i0 < ntiles; i0 += B) {
-    float v[B];
 #pragma unroll
-    for (int j = 0; j < B; ++j) v[j] = i0 + j < ntiles ? ss[i0 + j] : 0.f;
-#pragma unroll
-    for (int j = 0; j < B; ++j)
-      if (i0 + j < ntiles) s = __fadd_rn(s, v[j]);
-  }
+  for (int j = 0; j < B; ++j)
+    if (lane + 32 * j < ntiles) s = __fadd_rn(s, v[j]);
+  for (int i = lane + 32 * B; i < ntiles; i += 32) s = __fadd_rn(s, __ldcg(ss + i));
+  s = warp_sum(s);
   return __frcp_rn(__fsqrt_rn(__fadd_rn(__fmul_rn(s, inv_dim), eps)));
 }
 

@@ -51,15 +51,15 @@ QHL_DEV float dot4(float4 a, float4 b) {
   return __fmaf_rn(a.w, b.w, s);
 }
 
+// One unit: 32 rows of value head `unit / 4` (8 warps x 4 rows), all NT tokens.
+// ob: shared [NT][32] for the unit's outputs.  q, k, v, b, a are read through
+// L2 (they may have been written earlier in the same kernel by another CTA).
 template <int NT>
-__global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
-  __shared__ float ob[NT][32];
+QHL_DEV void dn_unit(const DnArgs& a, int unit, float (*ob)[32]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x >> 2;                       // 4 CTAs of 32 rows per head
-  const int row0 = (blockIdx.x & 3) * 32 + warp * 4;
+  const int h = unit >> 2;                       // 4 units of 32 rows per head
+  const int row0 = (unit & 3) * 32 + warp * 4;
   const int g = h / (a.Hv / a.Hk);
-  if (threadIdx.x == 0) pdl_launch();
-
   const int cur = a.cur ? *a.cur : 0;
   const float* s_in = a.cur ? a.ring + (size_t)cur * a.state_elems : a.s_in;
   float4 S[4];
@@ -67,29 +67,30 @@ __global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
   for (int r = 0; r < 4; ++r)
     S[r] = __ldg(reinterpret_cast<const float4*>(s_in + ((size_t)h * kDnDim + row0 + r) * kDnDim) + lane);
 
-  pdl_wait();
-
   const int off_k = a.Hk * kDnDim;
   const int off_v = 2 * a.Hk * kDnDim;
   const int off_b = off_v + a.Hv * kDnDim;
   const int off_a = off_b + a.Hv;
   for (int t = 0; t < NT; ++t) {
     const float* yt = a.y + (size_t)t * a.y_stride;
-    float4 q = *(reinterpret_cast<const float4*>(yt + g * kDnDim) + lane);
-    float4 k = *(reinterpret_cast<const float4*>(yt + off_k + g * kDnDim) + lane);
+    float4 q = __ldcg(reinterpret_cast<const float4*>(yt + g * kDnDim) + lane);
+    float4 k = __ldcg(reinterpret_cast<const float4*>(yt + off_k + g * kDnDim) + lane);
+    float v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) v[r] = __ldcg(yt + off_v + h * kDnDim + row0 + r);
+    const float bb = __ldcg(yt + off_b + h), aa = __ldcg(yt + off_a + h);
     const float rq = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(q, q)), 1e-6f)));
     const float rk = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(k, k)), 1e-6f)));
     q = make_float4(__fmul_rn(q.x, rq), __fmul_rn(q.y, rq), __fmul_rn(q.z, rq), __fmul_rn(q.w, rq));
     k = make_float4(__fmul_rn(k.x, rk), __fmul_rn(k.y, rk), __fmul_rn(k.z, rk), __fmul_rn(k.w, rk));
-    const float beta = sigmoidf_(yt[off_b + h]);     // sigmoid(b)
-    const float alpha = sigmoidf_(-yt[off_a + h]);   // exp(-softplus(a)) = sigmoid(-a)
+    const float beta = sigmoidf_(bb);      // sigmoid(b)
+    const float alpha = sigmoidf_(-aa);    // exp(-softplus(a)) = sigmoid(-a)
     float* dst = a.cur ? a.ring + (size_t)((cur + 1 + t) % a.ring_size) * a.state_elems
                        : a.ring + (size_t)t * a.state_elems;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float v = yt[off_v + h * kDnDim + row0 + r];
       const float kS = warp_sum(dot4(S[r], k));
-      const float coef = __fmul_rn(beta, __fsub_rn(v, __fmul_rn(alpha, kS)));
+      const float coef = __fmul_rn(beta, __fsub_rn(v[r], __fmul_rn(alpha, kS)));
       S[r].x = __fmaf_rn(coef, k.x, __fmul_rn(alpha, S[r].x));
       S[r].y = __fmaf_rn(coef, k.y, __fmul_rn(alpha, S[r].y));
       S[r].z = __fmaf_rn(coef, k.z, __fmul_rn(alpha, S[r].z));
@@ -102,11 +103,19 @@ __global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
       reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = S[r];
     }
   }
-  if (a.qo) {
-    __syncthreads();
+  named_sync(1, 256);
+  if (a.qo)
     for (int t = warp; t < NT; t += 8)
-      qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (blockIdx.x & 3), lane);
-  }
+      qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (unit & 3), lane);
+  named_sync(1, 256);   // ob reusable by the caller
+}
+
+template <int NT>
+__global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
+  __shared__ float ob[NT][32];
+  if (threadIdx.x == 0) pdl_launch();
+  pdl_wait();
+  dn_unit<NT>(a, blockIdx.x, ob);
 }
 
 }  // namespace qhl

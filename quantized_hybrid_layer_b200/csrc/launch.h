@@ -9,6 +9,8 @@
 
 #include "attention.cuh"
 #include "deltanet.cuh"
+#include "input.cuh"
+#include "pass.cuh"
 #include "qgemv.cuh"
 
 namespace qhl {
@@ -52,6 +54,20 @@ cudaError_t launch_dequant(int qt, const uint8_t* packed, int rows, int cols, in
 cudaError_t launch_rope_table(float2* tab, int max_ctx, int rope_dims, double theta, cudaStream_t s);
 cudaError_t launch_commit(int* ctrl, int n_accepted, int n_dn, int ring, cudaStream_t s);
 cudaError_t launch_set_int(int* p, int v, cudaStream_t s);
+
+// Persistent pass (pass.cuh), instantiated in pass_q4.cu / pass_q8.cu.
+extern template struct PassOps<kQ4_0>;
+extern template struct PassOps<kQ8_0>;
+inline cudaError_t pass_prepare(int qt) { return qt == kQ4_0 ? PassOps<kQ4_0>::prepare() : PassOps<kQ8_0>::prepare(); }
+inline cudaError_t pass_occupancy(int qt, int nt, int* blocks) {
+  return qt == kQ4_0 ? PassOps<kQ4_0>::occupancy(nt, blocks) : PassOps<kQ8_0>::occupancy(nt, blocks);
+}
+inline int pass_mix_bytes(int qt, int nt) {
+  return qt == kQ4_0 ? PassOps<kQ4_0>::mix_bytes(nt) : PassOps<kQ8_0>::mix_bytes(nt);
+}
+inline cudaError_t launch_pass(int qt, int nt, const PassArgs& p, cudaStream_t s) {
+  return qt == kQ4_0 ? PassOps<kQ4_0>::launch(nt, p, s) : PassOps<kQ8_0>::launch(nt, p, s);
+}
 
 // packed-layout geometry
 inline int packed_tiles(int rows, bool paired) { return paired ? (rows + 31) / 32 : (rows + 63) / 64; }

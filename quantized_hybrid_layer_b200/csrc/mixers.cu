@@ -32,17 +32,7 @@ __global__ void __launch_bounds__(256) stage_input_kernel(const float* h, int H,
                                                           int qz_stride, float* ss, int ss_stride) {
   __shared__ float sm[NT * 64];
   if (threadIdx.x == 0) pdl_launch();
-  const int tile = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int idx = threadIdx.x; idx < NT * 64; idx += blockDim.x) {
-    const int t = idx >> 6, gr = tile * 64 + (idx & 63);
-    sm[idx] = h[(size_t)t * H + gr];
-  }
-  __syncthreads();
-  for (int p = warp; p < NT * 2; p += 8) {
-    const int t = p >> 1, b = p & 1, gr = tile * 64 + b * 32 + lane;
-    qact_store_block(__fmul_rn(sm[t * 64 + b * 32 + lane], gamma[gr]), qz + (size_t)t * qz_stride, tile * 2 + b, lane);
-  }
-  if (threadIdx.x < NT) ss[(size_t)threadIdx.x * ss_stride + tile] = sumsq64(sm + threadIdx.x * 64);
+  input_unit<NT>(h, H, gamma, qz, qz_stride, ss, ss_stride, blockIdx.x, sm);
 }
 
 // f32 rows -> block fixed point, one warp per (token, 32-column block).

@@ -233,7 +233,7 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float
       float hn = 0.f;
       if (gr < a.out_valid) {
         float* hp = a.y + (size_t)t * a.y_stride + gr;
-        hn = __fadd_rn(*hp, vals[idx]);
+        hn = __fadd_rn(__ldcg(hp), vals[idx]);   // through L2: h may come from another CTA of the same kernel
         *hp = hn;
       }
       vals[idx] = hn;
@@ -248,6 +248,117 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float
     }
     if (a.ss_out && tid < NT) a.ss_out[(size_t)tid * a.ss_out_stride + tile] = sumsq64(vals + tid * 64);
   }
+}
+
+// Consumer side of one GEMV for CTA `cta` (the 256 threads of warps 0..7):
+// takes this CTA's stream-K items, in order, from the shared-memory ring
+// (`slot` / `phase` carry the ring position across calls), accumulates,
+// and finishes every tile it touches (directly or through the stream-K
+// partials).  `red` = [8][NT][64] f32, `rstd` = [16] f32, `flag` = one int.
+template <int QT, int NT, int EPI, int S>
+QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t* bars, float* red, float* rstd,
+                          int* flag, int& slot, uint32_t& phase, bool& timed_out) {
+  constexpr int IB = QLayout<QT>::kItemBytes;
+  constexpr int SB = IB + NT * kQChunkBytes;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long n_items = (long long)a.tiles * a.chunks;
+  const long long i0 = sk_begin(cta, n_items, a.workers);
+  const long long i1 = sk_begin(cta + 1, n_items, a.workers);
+  const int n_local = cta < a.workers ? (int)(i1 - i0) : 0;
+
+  if (n_local == 0) return;
+  // the input's RMS scale, one warp per token; only the epilogue reads it,
+  // after the first flush's barriers
+  for (int t = warp; t < NT; t += kConsumerWarps) {
+    const float r = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
+    if (lane == 0) rstd[t] = r;
+  }
+
+  float r0[NT], r1[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) { r0[t] = 0.f; r1[t] = 0.f; }
+  int tile = (int)(i0 / a.chunks);
+  const int first_tile = tile;
+
+  auto flush = [&](int tl) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      red[(warp * NT + t) * 64 + lane] = r0[t];
+      red[(warp * NT + t) * 64 + 32 + lane] = r1[t];
+      r0[t] = 0.f;
+      r1[t] = 0.f;
+    }
+    named_sync(1, 256);
+    for (int idx = tid; idx < NT * 64; idx += 256) {
+      float v = red[idx];
+#pragma unroll
+      for (int w = 1; w < kConsumerWarps; ++w) v = __fadd_rn(v, red[w * NT * 64 + idx]);
+      red[idx] = v;
+    }
+    named_sync(1, 256);
+    const long long t_lo = (long long)tl * a.chunks, t_hi = t_lo + a.chunks;
+    if (t_lo >= i0 && t_hi <= i1) {
+      gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
+    } else {
+      // stream-K: publish this CTA's partial; the last contributor finishes the tile
+      // (release: the barrier orders every thread's stores before thread 0's
+      // fence and counter increment; acquire: the last arriver's fence after
+      // its increment, then the barrier, orders the partial loads after it)
+      float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * 64;
+      for (int idx = tid; idx < NT * 64; idx += 256) mine[idx] = red[idx];
+      named_sync(1, 256);
+      const long long cf = sk_owner(t_lo, n_items, a.workers);
+      const long long cl = sk_owner(t_hi - 1, n_items, a.workers);
+      if (tid == 0) {
+        __threadfence();
+        const int old = atomicAdd(&a.counters[tl], 1);
+        const int last = (old == (int)(cl - cf)) ? 1 : 0;
+        if (last) __threadfence();
+        *flag = last;
+      }
+      named_sync(1, 256);
+      if (*flag) {
+        for (int idx = tid; idx < NT * 64; idx += 256) {
+          float v = 0.f;
+          for (long long c = cf; c <= cl; ++c) {
+            const int ft = (int)(sk_begin(c, n_items, a.workers) / a.chunks);
+            const float* pc = a.partials + (size_t)(2 * c + (tl == ft ? 0 : 1)) * NT * 64;
+            const float pv = __ldcg(pc + idx);
+            v = (c == cf) ? pv : __fadd_rn(v, pv);
+          }
+          red[idx] = v;
+        }
+        named_sync(1, 256);
+        gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
+        if (tid == 0) a.counters[tl] = 0;
+      }
+    }
+    named_sync(1, 256);
+  };
+
+  int chunk = (int)(i0 - (long long)tile * a.chunks);
+  for (int k = 0; k < n_local; ++k) {
+    if (chunk == a.chunks) {
+      flush(tile);
+      ++tile;
+      chunk = 0;
+    }
+    // after one timed-out wait the rest of the call runs without waiting (the
+    // error is recorded; results are garbage, but the kernel ends promptly)
+    if (!timed_out && !mbar_wait(smem_u32(&bars[slot]), phase, a.err)) timed_out = true;
+    ItemRegs<QT> regs;
+    const uint8_t* st = stages + slot * SB;
+    load_item<QT>(st, warp, lane, regs);
+    compute_item<QT, NT>(regs, st + IB, warp, r0, r1);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars[S + slot]));   // stage free for the producer
+    ++chunk;
+    if (++slot == S) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  flush(tile);
 }
 
 template <int QT, int NT, int EPI>
@@ -318,100 +429,11 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
 
   // ---------------- consumers ------------------------------------------------
   pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
-  if (tid < NT)
-    rstd[tid] = a.ss_in ? rstd_from_partials(a.ss_in + (size_t)tid * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps) : 1.f;
-
-  float r0[NT], r1[NT];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) { r0[t] = 0.f; r1[t] = 0.f; }
-  bool timed_out = false;
-  int tile = (int)(i0 / a.chunks);
-  const int first_tile = tile;
-
-  auto flush = [&](int tl) {
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      red[(warp * NT + t) * 64 + lane] = r0[t];
-      red[(warp * NT + t) * 64 + 32 + lane] = r1[t];
-      r0[t] = 0.f;
-      r1[t] = 0.f;
-    }
-    named_sync(1, 256);
-    for (int idx = tid; idx < NT * 64; idx += 256) {
-      float v = red[idx];
-#pragma unroll
-      for (int w = 1; w < kConsumerWarps; ++w) v = __fadd_rn(v, red[w * NT * 64 + idx]);
-      red[idx] = v;
-    }
-    named_sync(1, 256);
-    const long long t_lo = (long long)tl * a.chunks, t_hi = t_lo + a.chunks;
-    if (t_lo >= i0 && t_hi <= i1) {
-      gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
-    } else {
-      // stream-K: publish this CTA's partial; the last contributor finishes the tile
-      // (release: the barrier orders every thread's stores before thread 0's
-      // fence and counter increment; acquire: the last arriver's fence after
-      // its increment, then the barrier, orders the partial loads after it)
-      float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * 64;
-      for (int idx = tid; idx < NT * 64; idx += 256) mine[idx] = red[idx];
-      named_sync(1, 256);
-      const long long cf = sk_owner(t_lo, n_items, a.workers);
-      const long long cl = sk_owner(t_hi - 1, n_items, a.workers);
-      if (tid == 0) {
-        __threadfence();
-        const int old = atomicAdd(&a.counters[tl], 1);
-        const int last = (old == (int)(cl - cf)) ? 1 : 0;
-        if (last) __threadfence();
-        *flag = last;
-      }
-      named_sync(1, 256);
-      if (*flag) {
-        for (int idx = tid; idx < NT * 64; idx += 256) {
-          float v = 0.f;
-          for (long long c = cf; c <= cl; ++c) {
-            const int ft = (int)(sk_begin(c, n_items, a.workers) / a.chunks);
-            const float* pc = a.partials + (size_t)(2 * c + (tl == ft ? 0 : 1)) * NT * 64;
-            const float pv = __ldcg(pc + idx);
-            v = (c == cf) ? pv : __fadd_rn(v, pv);
-          }
-          red[idx] = v;
-        }
-        named_sync(1, 256);
-        gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
-        if (tid == 0) a.counters[tl] = 0;
-      }
-    }
-    named_sync(1, 256);
-  };
-
-  named_sync(1, 256);   // rstd visible
-  int chunk = (int)(i0 - (long long)tile * a.chunks);
-  int s = 0;
+  int slot = 0;
   uint32_t phase = 0;
-  for (int k = 0; k < n_local; ++k) {
-    if (chunk == a.chunks) {
-      flush(tile);
-      ++tile;
-      chunk = 0;
-    }
-    if (!mbar_wait(smem_u32(&bars[s]), phase, a.err)) timed_out = true;
-    ItemRegs<QT> regs;
-    const uint8_t* st = stages + s * SB;
-    load_item<QT>(st, warp, lane, regs);
-    compute_item<QT, NT>(regs, st + IB, warp, r0, r1);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&bars[S + s]));   // stage free for the producer
-    ++chunk;
-    if (++s == S) {
-      s = 0;
-      phase ^= 1u;
-    }
-  }
-  if (n_local > 0) flush(tile);
-  if (timed_out && lane == 0) {
-    // error path: let any copy still in flight land before the CTA exits
-    for (int q = 0; q < S; ++q) mbar_wait(smem_u32(&bars[q]), 0, nullptr);
-  }
+  bool timed_out = false;
+  gemv_consume<QT, NT, EPI, S>(a, cta, stages, bars, red, rstd, flag, slot, phase, timed_out);
+  if (timed_out && tid == 0) drain_inflight_copies();   // error path
 }
 
 }  // namespace qhl

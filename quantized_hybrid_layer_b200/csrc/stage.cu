@@ -92,6 +92,10 @@ struct stage {
   int committed = 0, pending_n = 0, pending_pos = 0;
   std::vector<int> cur;
   cudaGraphExec_t exec[kMaxTok + 1] = {};
+  // persistent pass: per-layer step arguments on the device, grid-barrier counter
+  PassLayer* pass_layers = nullptr;
+  unsigned* bar = nullptr;
+  int pass_mode = STAGE_PASS_PERSISTENT;
   size_t weight_bytes = 0;
   std::string last_error;
 };
@@ -169,122 +173,193 @@ GemvArgs gemv_base(const stage* st) {
   return a;
 }
 
-cudaError_t run_gemv(const stage* st, int n, int epi, GemvArgs& a, cudaStream_t s) {
+void set_workers(const stage* st, GemvArgs& a) {
   const long long items = (long long)a.tiles * a.chunks;
   a.workers = (int)std::min<long long>((long long)kCtasPerSm * st->sms, items);
-  return launch_gemv(st->cfg.qtype, n, epi, a, a.workers, s, kUsePdl);
 }
 
-// Record one pass of n tokens onto stream s (being captured).
-cudaError_t record_pass(stage* st, int n, cudaStream_t s) {
+// Arguments of every step of layer i (shared by both execution paths, so they
+// run the same units with the same split).
+PassLayer layer_args(const stage* st, size_t i) {
   const stage_config& c = st->cfg;
   const int H = c.hidden, F = c.ffn;
-  cudaError_t e = launch_stage_input(n, st->h, H, st->layers[0].norm1, st->qz, st->qz_stride, st->ss,
-                                     st->ss_stride, s);
-  if (e != cudaSuccess) return e;
-  for (size_t i = 0; i < st->layers.size(); ++i) {
-    const Layer& L = st->layers[i];
-    const float* next_norm1 = i + 1 < st->layers.size() ? st->layers[i + 1].norm1 : nullptr;
-    // mixer in-projection with the RMSNorm1 scale folded into the epilogue
-    GemvArgs a = gemv_base(st);
-    a.W = L.w_in;
-    a.tiles = L.in_tiles;
-    a.chunks = H / kChunkCols;
-    a.qx = st->qz;
-    a.qx_stride = st->qz_stride;
-    a.y = st->y;
-    a.y_stride = st->y_stride;
-    a.out_valid = L.in_rows;
-    a.ss_in = st->ss;
-    a.ss_tiles = H / 64;
-    a.ss_stride = st->ss_stride;
-    if ((e = run_gemv(st, n, EPI_STORE, a, s)) != cudaSuccess) return e;
-    if (!L.attn) {
-      DnArgs d = {};
-      d.y = st->y;
-      d.y_stride = st->y_stride;
-      d.Hk = c.dn_k_heads;
-      d.Hv = c.dn_v_heads;
-      d.ring = L.ring;
-      d.state_elems = st->state_elems;
-      d.ring_size = kRing;
-      d.cur = st->ctrl + 1 + L.dn_slot;
-      d.qo = st->qo;
-      d.qo_stride = st->qo_stride;
-      if ((e = launch_dn_step(n, d, c.dn_v_heads * (kDnDim / 32), s, kUsePdl)) != cudaSuccess) return e;
-    } else {
-      AttnArgs at = {};
-      at.y = st->y;
-      at.y_stride = st->y_stride;
-      at.Hq = c.att_q_heads;
-      at.Hkv = c.att_kv_heads;
-      at.K = L.K;
-      at.V = L.V;
-      at.max_ctx = c.max_ctx;
-      at.kv_len = st->ctrl;
-      at.gq = L.qn;
-      at.gk = L.kn;
-      at.rope = st->rope;
-      at.eps = c.eps;
-      at.pm = st->pm;
-      at.pl = st->pl;
-      at.po = st->po;
-      at.nchunk = st->nchunk;
-      at.qout = st->qo;
-      at.qout_stride = st->qo_stride;
-      if ((e = launch_attn_partial(n, at, st->nchunk, c.att_kv_heads, s, kUsePdl)) != cudaSuccess) return e;
-      if ((e = launch_attn_combine(n, at, s, kUsePdl)) != cudaSuccess) return e;
-    }
-    // out-projection + residual; z = h * norm2 (block fixed point) and its tile sums of squares
-    a = gemv_base(st);
-    a.W = L.w_out;
-    a.tiles = H / 64;
-    a.chunks = L.out_cols / kChunkCols;
-    a.qx = st->qo;
-    a.qx_stride = st->qo_stride;
-    a.y = st->h;
-    a.y_stride = H;
-    a.out_valid = H;
-    a.gamma_next = L.norm2;
+  const Layer& L = st->layers[i];
+  const float* next_norm1 = i + 1 < st->layers.size() ? st->layers[i + 1].norm1 : nullptr;
+  PassLayer P = {};
+  P.attn = L.attn ? 1 : 0;
+  // mixer in-projection with the RMSNorm1 scale folded into the epilogue
+  GemvArgs a = gemv_base(st);
+  a.W = L.w_in;
+  a.tiles = L.in_tiles;
+  a.chunks = H / kChunkCols;
+  a.qx = st->qz;
+  a.qx_stride = st->qz_stride;
+  a.y = st->y;
+  a.y_stride = st->y_stride;
+  a.out_valid = L.in_rows;
+  a.ss_in = st->ss;
+  a.ss_tiles = H / 64;
+  a.ss_stride = st->ss_stride;
+  set_workers(st, a);
+  P.g[0] = a;
+  if (!L.attn) {
+    DnArgs& d = P.dn;
+    d.y = st->y;
+    d.y_stride = st->y_stride;
+    d.Hk = c.dn_k_heads;
+    d.Hv = c.dn_v_heads;
+    d.ring = L.ring;
+    d.state_elems = st->state_elems;
+    d.ring_size = kRing;
+    d.cur = st->ctrl + 1 + L.dn_slot;
+    d.qo = st->qo;
+    d.qo_stride = st->qo_stride;
+  } else {
+    AttnArgs& at = P.at;
+    at.y = st->y;
+    at.y_stride = st->y_stride;
+    at.Hq = c.att_q_heads;
+    at.Hkv = c.att_kv_heads;
+    at.K = L.K;
+    at.V = L.V;
+    at.max_ctx = c.max_ctx;
+    at.kv_len = st->ctrl;
+    at.gq = L.qn;
+    at.gk = L.kn;
+    at.rope = st->rope;
+    at.eps = c.eps;
+    at.pm = st->pm;
+    at.pl = st->pl;
+    at.po = st->po;
+    at.nchunk = st->nchunk;
+    at.qout = st->qo;
+    at.qout_stride = st->qo_stride;
+  }
+  // out-projection + residual; z = h * norm2 (block fixed point) and its tile sums of squares
+  a = gemv_base(st);
+  a.W = L.w_out;
+  a.tiles = H / 64;
+  a.chunks = L.out_cols / kChunkCols;
+  a.qx = st->qo;
+  a.qx_stride = st->qo_stride;
+  a.y = st->h;
+  a.y_stride = H;
+  a.out_valid = H;
+  a.gamma_next = L.norm2;
+  a.qout = st->qz;
+  a.qout_stride = st->qz_stride;
+  a.ss_out = st->ss;
+  a.ss_out_stride = st->ss_stride;
+  set_workers(st, a);
+  P.g[1] = a;
+  // gate/up with the RMSNorm2 scale and the SwiGLU epilogue
+  a = gemv_base(st);
+  a.W = L.w_gu;
+  a.tiles = (F + 31) / 32;
+  a.chunks = H / kChunkCols;
+  a.qx = st->qz;
+  a.qx_stride = st->qz_stride;
+  a.out_valid = F;
+  a.qout = st->qu;
+  a.qout_stride = st->qu_stride;
+  a.ss_in = st->ss;
+  a.ss_tiles = H / 64;
+  a.ss_stride = st->ss_stride;
+  set_workers(st, a);
+  P.g[2] = a;
+  // down + residual; z for the next layer's RMSNorm1
+  a = gemv_base(st);
+  a.W = L.w_down;
+  a.tiles = H / 64;
+  a.chunks = F / kChunkCols;
+  a.qx = st->qu;
+  a.qx_stride = st->qu_stride;
+  a.y = st->h;
+  a.y_stride = H;
+  a.out_valid = H;
+  if (next_norm1) {
+    a.gamma_next = next_norm1;
     a.qout = st->qz;
     a.qout_stride = st->qz_stride;
     a.ss_out = st->ss;
     a.ss_out_stride = st->ss_stride;
-    if ((e = run_gemv(st, n, EPI_RESID, a, s)) != cudaSuccess) return e;
-    // gate/up with the RMSNorm2 scale and the SwiGLU epilogue
-    a = gemv_base(st);
-    a.W = L.w_gu;
-    a.tiles = (F + 31) / 32;
-    a.chunks = H / kChunkCols;
-    a.qx = st->qz;
-    a.qx_stride = st->qz_stride;
-    a.out_valid = F;
-    a.qout = st->qu;
-    a.qout_stride = st->qu_stride;
-    a.ss_in = st->ss;
-    a.ss_tiles = H / 64;
-    a.ss_stride = st->ss_stride;
-    if ((e = run_gemv(st, n, EPI_SWIGLU, a, s)) != cudaSuccess) return e;
-    // down + residual; z for the next layer's RMSNorm1
-    a = gemv_base(st);
-    a.W = L.w_down;
-    a.tiles = H / 64;
-    a.chunks = F / kChunkCols;
-    a.qx = st->qu;
-    a.qx_stride = st->qu_stride;
-    a.y = st->h;
-    a.y_stride = H;
-    a.out_valid = H;
-    if (next_norm1) {
-      a.gamma_next = next_norm1;
-      a.qout = st->qz;
-      a.qout_stride = st->qz_stride;
-      a.ss_out = st->ss;
-      a.ss_out_stride = st->ss_stride;
+  }
+  set_workers(st, a);
+  P.g[3] = a;
+  return P;
+}
+
+// Record one pass of n tokens onto stream s (being captured) as a chain of
+// kernels: stage input, then per layer in-projection, mixer, out-projection,
+// gate/up, down.
+cudaError_t record_kernels(stage* st, int n, cudaStream_t s) {
+  const stage_config& c = st->cfg;
+  const int qt = c.qtype;
+  cudaError_t e = launch_stage_input(n, st->h, c.hidden, st->layers[0].norm1, st->qz, st->qz_stride, st->ss,
+                                     st->ss_stride, s);
+  if (e != cudaSuccess) return e;
+  for (size_t i = 0; i < st->layers.size(); ++i) {
+    const PassLayer P = layer_args(st, i);
+    if ((e = launch_gemv(qt, n, EPI_STORE, P.g[0], P.g[0].workers, s, kUsePdl)) != cudaSuccess) return e;
+    if (!P.attn) {
+      if ((e = launch_dn_step(n, P.dn, c.dn_v_heads * (kDnDim / 32), s, kUsePdl)) != cudaSuccess) return e;
+    } else {
+      if ((e = launch_attn_partial(n, P.at, st->nchunk, c.att_kv_heads, s, kUsePdl)) != cudaSuccess) return e;
+      if ((e = launch_attn_combine(n, P.at, s, kUsePdl)) != cudaSuccess) return e;
     }
-    if ((e = run_gemv(st, n, EPI_RESID, a, s)) != cudaSuccess) return e;
+    if ((e = launch_gemv(qt, n, EPI_RESID, P.g[1], P.g[1].workers, s, kUsePdl)) != cudaSuccess) return e;
+    if ((e = launch_gemv(qt, n, EPI_SWIGLU, P.g[2], P.g[2].workers, s, kUsePdl)) != cudaSuccess) return e;
+    if ((e = launch_gemv(qt, n, EPI_RESID, P.g[3], P.g[3].workers, s, kUsePdl)) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// Whether the n-token pass can run as one persistent kernel: n within the
+// instantiated range, two CTAs per SM resident, and the mixers' scratch within
+// the kernel's shared memory.
+bool pass_eligible(const stage* st, int n) {
+  if (n > kPassMaxTok || !st->pass_layers) return false;
+  const int qt = st->cfg.qtype;
+  int blocks = 0;
+  if (pass_occupancy(qt, n, &blocks) != cudaSuccess || blocks < 2) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  const int rep = st->cfg.att_q_heads / st->cfg.att_kv_heads;
+  const int mix = pass_mix_bytes(qt, n);
+  const int need = std::max({n * 64 * 4, n * 32 * 4, st->nchunk * 3 * 4, st->nchunk ? attn_smem_bytes(n, rep) : 0});
+  return need <= mix;
+}
+
+// Record one pass of n tokens as one cooperative persistent kernel (pass.cuh)
+// after zeroing its grid-barrier counter.
+cudaError_t record_persistent(stage* st, int n, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(st->bar, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  const stage_config& c = st->cfg;
+  PassArgs p = {};
+  p.layers = st->pass_layers;
+  p.n_layers = (int)st->layers.size();
+  p.h = st->h;
+  p.H = c.hidden;
+  p.gamma0 = st->layers[0].norm1;
+  p.qz = st->qz;
+  p.qz_stride = st->qz_stride;
+  p.ss = st->ss;
+  p.ss_stride = st->ss_stride;
+  p.kv_len = st->ctrl;
+  p.bar = st->bar;
+  p.grid = kCtasPerSm * st->sms;
+  p.dn_units = c.dn_v_heads * (kDnDim / 32);
+  p.Hq = c.att_q_heads;
+  p.Hkv = c.att_kv_heads;
+  p.err = st->err;
+  return launch_pass(c.qtype, n, p, s);
+}
+
+cudaError_t record_pass(stage* st, int n, cudaStream_t s) {
+  if (st->pass_mode == STAGE_PASS_PERSISTENT && pass_eligible(st, n)) return record_persistent(st, n, s);
+  return record_kernels(st, n, s);
 }
 
 stage_status build_graph(stage* st, int n) {
@@ -513,6 +588,24 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
       (e = cudaMemset(st->h, 0, (size_t)kMaxTok * H * 4)) != cudaSuccess)
     return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
   st->cur.assign(st->n_dn, 0);
+
+  // --- persistent pass: step arguments of every layer, phase numbering -------
+  if ((e = pass_prepare(qt)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("pass_prepare", e)));
+  {
+    std::vector<PassLayer> pl(st->layers.size());
+    int phase = 1;   // phase 0: stage input
+    for (size_t i = 0; i < pl.size(); ++i) {
+      pl[i] = layer_args(st, i);
+      pl[i].phase_in = phase;
+      phase += pl[i].attn ? 6 : 5;   // in-proj, mixer (attention: partials + combine), out, gate/up, down
+    }
+    if ((s = dalloc_t(st, &st->pass_layers, pl.size() * sizeof(PassLayer))) != STAGE_OK ||
+        (s = dalloc_t(st, &st->bar, 16)) != STAGE_OK)
+      return bail(s);
+    if ((e = cudaMemcpy(st->pass_layers, pl.data(), pl.size() * sizeof(PassLayer), cudaMemcpyHostToDevice)) !=
+        cudaSuccess)
+      return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemcpy pass layers", e)));
+  }
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("load sync", e)));
   *out = st;
   return STAGE_OK;
@@ -666,6 +759,26 @@ stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float
   cudaFree(tmp);
   if (e != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg("dequant", e));
   return STAGE_OK;
+}
+
+stage_status stage_set_pass_mode(stage_t* st, int mode) {
+  if (!st) return STAGE_E_ARG;
+  if (mode != STAGE_PASS_KERNELS && mode != STAGE_PASS_PERSISTENT) return fail(st, STAGE_E_ARG, "unknown pass mode");
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  if (mode == st->pass_mode) return STAGE_OK;
+  CK(cudaStreamSynchronize(st->stream));
+  for (auto& g : st->exec)
+    if (g) {
+      CK(cudaGraphExecDestroy(g));
+      g = nullptr;
+    }
+  st->pass_mode = mode;
+  return STAGE_OK;
+}
+
+int stage_pass_persistent(stage_t* st, int n_tok) {
+  if (!st || n_tok < 1 || n_tok > kMaxTok) return -1;
+  return st->pass_mode == STAGE_PASS_PERSISTENT && pass_eligible(st, n_tok) ? 1 : 0;
 }
 
 size_t stage_weight_bytes(const stage_t* st) { return st ? st->weight_bytes : 0; }

@@ -233,3 +233,50 @@ def test_load_rejects_missing_or_misshaped_tensors(q):
     assert e.value.code == -5
     st = q.stage_load(cfg, t, 3, 4)                         # an attention-only stage loads
     st.free()
+
+
+@pytest.mark.parametrize("qtype,ns", [(Q4_0, (1, 2, 3, 4)), (Q8_0, (1, 3))])
+def test_persistent_pass_equals_kernel_chain(q, qtype, ns):
+    """The one-kernel persistent pass and the chain of per-step kernels run the
+    same units with the same split: outputs and committed states are
+    bit-identical."""
+    import torch
+    seed = 7
+    st, _, _ = make_pair(FULL, qtype, seed, 0, 4, MAX_CTX, CTX, with_oracle=False)
+    try:
+        assert not st.pass_persistent(16)
+        S0 = _states(st, 0, 4)
+        kv0 = {l: st.get_kv(l) for l in attn_layers(0, 4)}
+        for n in ns:
+            st.set_pass_mode(q.PASS_PERSISTENT)
+            assert st.pass_persistent(n), n
+            h = synth.hidden(FULL, seed, n, n)
+            res = {}
+            for mode in (q.PASS_PERSISTENT, q.PASS_KERNELS):
+                st.set_pass_mode(mode)
+                out = run(st, h, CTX)
+                st.commit(n)
+                res[mode] = (out, _states(st, 0, 4), {l: st.get_kv(l) for l in attn_layers(0, 4)})
+                for l, S in S0.items():                       # back to the starting state
+                    st.set_dn_state(l, S)
+                for l, (K, V) in kv0.items():
+                    st.set_kv(l, K, V)
+                st.set_kv_len(CTX)
+            out_p, S_p, kv_p = res[q.PASS_PERSISTENT]
+            out_k, S_k, kv_k = res[q.PASS_KERNELS]
+            assert np.array_equal(out_p, out_k), n
+            for l in S_p:
+                assert np.array_equal(S_p[l], S_k[l]), (n, l)
+            for l in kv_p:
+                assert np.array_equal(kv_p[l][0], kv_k[l][0]) and np.array_equal(kv_p[l][1], kv_k[l][1]), (n, l)
+        st.set_pass_mode(q.PASS_PERSISTENT)
+        st.forward(torch.zeros((1, FULL.hidden), device="cuda"), CTX)
+        with pytest.raises(q.StageError) as e:
+            st.set_pass_mode(q.PASS_KERNELS)          # refused while a pass is pending
+        assert e.value.code == -2
+        st.rollback()
+        with pytest.raises(q.StageError) as e:
+            st.set_pass_mode(5)
+        assert e.value.code == -1
+    finally:
+        st.free()
