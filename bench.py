@@ -127,9 +127,11 @@ def pass_bytes(shape, qtype, layers, ctx: int, n_tok: int = 1) -> dict:
     return {"weights": w, "kv": kv, "state": state, "total": w + kv + state}
 
 
-def launches_per_pass(shape, layers) -> int:
-    """Kernels the stage launches per pass: input + per layer (in-proj, mixer
-    kernel(s), out-proj, gate/up, down)."""
+def launches_per_pass(shape, layers, persistent: bool) -> int:
+    """Kernels the stage launches per pass: one persistent kernel, or input +
+    per layer (in-proj, mixer kernel(s), out-proj, gate/up, down)."""
+    if persistent:
+        return 1
     n = 1
     for l in layers:
         n += 6 if shape.is_attention(l) else 5
@@ -146,7 +148,7 @@ def measured_peaks() -> dict:
 
 def kernel_sources_sha() -> str:
     h = hashlib.sha256()
-    for f in ("qgemv.cuh", "qpack.cuh", "common.cuh"):
+    for f in ("qgemv.cuh", "qpack.cuh", "qact.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "quantized_hybrid_layer_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -328,6 +330,8 @@ def run_ours(args, rank, world, local, pg):
     cfg = q.config_from_shape(shape, qtype, max_ctx)
     with torch.cuda.stream(stream):
         st = q.stage_load(cfg, tensors, 0, args.layers, stream=stream)
+        st.set_pass_mode(q.PASS_PERSISTENT if args.pass_mode == "persistent" else q.PASS_KERNELS)
+        persistent = st.pass_persistent(1)
         for l in layers:
             if shape.is_attention(l):
                 K, V = synth.kv_prefill(shape, SEED, l, CTX0, max_ctx)
@@ -449,7 +453,8 @@ def run_ours(args, rank, world, local, pg):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (launches_per_pass(shape, layers) + 1) * args.steps,
+        "gpu_launches": (launches_per_pass(shape, layers, persistent) + 1) * args.steps,
+        "pass_mode": "persistent" if persistent else "kernels",
         "clocks": clk,
     }
     return res
@@ -507,11 +512,30 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-roofline", action="store_true")
+    ap.add_argument("--pass-mode", choices=("kernels", "persistent"), default="kernels",
+                    help="one kernel per step (CUDA graph) or the one-kernel persistent pass")
+    ap.add_argument("--only-kernel-roofline", action="store_true",
+                    help="time only the dominant kernel alone (the GEMV roofline leg) and print it")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local, pg = dist_setup(args.gpus)
     try:
+        if args.only_kernel_roofline:
+            import torch
+
+            import quantized_hybrid_layer_b200 as q
+            q.lib()
+            dev = torch.device("cuda", local)
+            torch.cuda.set_device(dev)
+            peaks = measured_peaks()
+            hbm = peaks.get("hbm_gbs")
+            roof = gemv_roofline(q, torch, dev, torch.cuda.Stream(device=dev), FULL,
+                                 Q4_0 if args.qtype == "q4_0" else Q8_0, hbm or FALLBACK_HBM_GBS,
+                                 "measured" if hbm else "fallback")
+            if rank == 0:
+                print(json.dumps({"roofline": roof}), flush=True)
+            return
         if args.impl == "reference":
             res = run_reference(args, rank, world, pg)
         else:

@@ -185,6 +185,19 @@ stage_status stage_set_pass_mode(stage_t* st, int mode);
  * of kernels, -1 for a NULL stage or n_tok outside 1..16. */
 int stage_pass_persistent(stage_t* st, int n_tok);
 
+/* Phase trace of the persistent pass (a profiling aid; off by default).
+ * stage_set_trace(st, 1) makes every later persistent pass record, per CTA and
+ * phase, the global-timer time (ns) at which the CTA's consumers started the
+ * phase (past the grid barrier) and finished it; phase 0 is the stage input,
+ * then per layer in-projection, mixer (attention: partials, combine),
+ * out-projection, gate/up, down.  Toggling waits for the stream and drops the
+ * recorded graphs; refused while a pass is pending.
+ * stage_get_trace copies the last pass's record, u64 [grid][n_phases][2], to
+ * host_dst (count = grid * n_phases * 2; host_dst NULL only reports the sizes
+ * through grid / n_phases); STAGE_E_STATE if tracing is off. */
+stage_status stage_set_trace(stage_t* st, int enable);
+stage_status stage_get_trace(stage_t* st, unsigned long long* host_dst, size_t count, int* grid, int* n_phases);
+
 /* Bytes of weight storage the stage streams per pass (packed quants + scales). */
 size_t stage_weight_bytes(const stage_t* st);
 
@@ -226,6 +239,7 @@ int qhl_dequant(int qtype, int rows, int cols, const void* packed_dev, int paire
 /* y = x W^T for n_tok tokens (1..16): x_dev f32 [n_tok, cols], y_dev f32
  * [n_tok, rows], W packed (not paired).  Reduction order is fixed and
  * independent of n_tok (a batched call equals n_tok single calls bit for bit).
+ * At most 2^31 - 1 packed items (ceil(rows/64) * cols/256), else STAGE_E_ARG.
  * Uses library-owned scratch (stream-K partials and tile counters, allocated
  * on first use per device and grown on demand); concurrent calls on different
  * streams of the same device must not overlap. */

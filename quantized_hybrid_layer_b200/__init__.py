@@ -33,6 +33,7 @@ EXPORTS = (
     "stage_load", "stage_forward", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
     "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_set_pass_mode", "stage_pass_persistent",
+    "stage_set_trace", "stage_get_trace",
     "stage_weight_bytes", "stage_last_error",
     "stage_free", "qhl_packed_bytes", "qhl_repack", "qhl_dequant", "qhl_qgemv", "qhl_deltanet_step",
     "qhl_qgemv_noalloc", "qhl_last_error",
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
             "stage_debug_dequant": (i, [vp, ctypes.c_char_p, i, vp]),
             "stage_set_pass_mode": (i, [vp, i]),
             "stage_pass_persistent": (i, [vp, i]),
+            "stage_set_trace": (i, [vp, i]),
+            "stage_get_trace": (i, [vp, vp, sz, ctypes.POINTER(i), ctypes.POINTER(i)]),
             "stage_weight_bytes": (sz, [vp]),
             "stage_last_error": (ctypes.c_char_p, [vp]),
             "stage_free": (None, [vp]),
@@ -190,6 +193,18 @@ class Stage:
     def pass_persistent(self, n_tok: int) -> bool:
         """Whether an n_tok pass runs as the persistent kernel."""
         return lib().stage_pass_persistent(self._h, n_tok) == 1
+
+    def set_trace(self, enable: bool):
+        """Record per-CTA phase times of later persistent passes."""
+        self._check(lib().stage_set_trace(self._h, 1 if enable else 0))
+
+    def get_trace(self) -> np.ndarray:
+        """The last persistent pass's record: u64 ns [grid, n_phases, 2] (start, end)."""
+        g, n = ctypes.c_int(0), ctypes.c_int(0)
+        self._check(lib().stage_get_trace(self._h, None, 0, ctypes.byref(g), ctypes.byref(n)))
+        out = np.zeros((g.value, n.value, 2), dtype=np.uint64)
+        self._check(lib().stage_get_trace(self._h, out.ctypes.data, out.size, ctypes.byref(g), ctypes.byref(n)))
+        return out
 
     @property
     def weight_bytes(self) -> int:

@@ -166,7 +166,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
   uint4 kw[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    kw[i] = key < nkeys ? __ldcg(reinterpret_cast<const uint4*>(a.K + (head_base + k0 + key) * kAttDim) + 4 * i + r4)
+    kw[i] = key < nkeys ? ld_cg_once(reinterpret_cast<const uint4*>(a.K + (head_base + k0 + key) * kAttDim) + 4 * i + r4)
                         : make_uint4(0u, 0u, 0u, 0u);
 
   // scores q.k / 16 (1 / sqrt(256)); per (query, key): each lane's 64 dims in
@@ -205,13 +205,14 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
       if (j0 + jj < njobs && r4 == 0 && key < nkeys) sc[(j0 + jj) * kAttChunk + key] = __fmul_rn(s, 1.f / 16.f);
     }
   }
-  // V rows, issued before the softmax so their latency overlaps it
+  // V rows, issued before the softmax so their latency overlaps it (volatile
+  // loads: the compiler may neither repeat them later nor move them)
   const int pair = tid & 127, half = tid >> 7;
   uint32_t vr[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int kk = half * 32 + i;
-    vr[i] = kk < nkeys ? __ldcg(reinterpret_cast<const uint32_t*>(a.V + (head_base + k0 + kk) * kAttDim) + pair) : 0u;
+    vr[i] = kk < nkeys ? ld_cg_once(reinterpret_cast<const uint32_t*>(a.V + (head_base + k0 + kk) * kAttDim) + pair) : 0u;
   }
   named_sync(1, 256);
 
@@ -238,13 +239,15 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
   named_sync(1, 256);
 
   // exp-weighted V: per (query, dim) the keys of each half in order, then
-  // half 0 + half 1; 8 queries at a time (vec_all holds half 1's sums)
-  float* part = vec_all;   // [8][256]
-  for (int j0 = 0; j0 < njobs; j0 += 8) {
-    float o0[8], o1[8];
-    int nk[8];
+  // half 0 + half 1; 4 queries at a time (vec_all holds half 1's sums), so
+  // the V rows stay in registers across the batches
+  constexpr int JB = 4;
+  float* part = vec_all;   // [JB][256]
+  for (int j0 = 0; j0 < njobs; j0 += JB) {
+    float o0[JB], o1[JB];
+    int nk[JB];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
+    for (int jj = 0; jj < JB; ++jj) {
       o0[jj] = 0.f;
       o1[jj] = 0.f;
       nk[jj] = j0 + jj < njobs ? min(kAttChunk, pos + (j0 + jj) / rep + 1 - k0) : 0;
@@ -255,7 +258,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
       const float vlo = __half2float(__ushort_as_half(static_cast<unsigned short>(vr[i] & 0xFFFFu)));
       const float vhi = __half2float(__ushort_as_half(static_cast<unsigned short>(vr[i] >> 16)));
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
+      for (int jj = 0; jj < JB; ++jj) {
         if (kk < nk[jj]) {
           const float pr = sc[(j0 + jj) * kAttChunk + kk];
           o0[jj] = __fmaf_rn(pr, vlo, o0[jj]);
@@ -265,13 +268,13 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
     }
     if (half == 1) {
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj)
+      for (int jj = 0; jj < JB; ++jj)
         reinterpret_cast<float2*>(part + jj * kAttDim)[pair] = make_float2(o0[jj], o1[jj]);
     }
     named_sync(1, 256);
     if (half == 0) {
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
+      for (int jj = 0; jj < JB; ++jj) {
         const int job = j0 + jj;
         if (job < njobs && nk[jj] > 0) {
           const int t = job / rep, j = job - t * rep;
@@ -329,7 +332,7 @@ QHL_DEV void combine_unit(const AttnArgs& a, int t, int head, int pos, float* cs
   for (int c0 = 0; c0 < nc; c0 += B) {
     float v[B];
 #pragma unroll
-    for (int j = 0; j < B; ++j) v[j] = c0 + j < nc ? __ldcg(po + (size_t)(c0 + j) * kAttDim) : 0.f;
+    for (int j = 0; j < B; ++j) v[j] = c0 + j < nc ? ld_cg_once(po + (size_t)(c0 + j) * kAttDim) : 0.f;
 #pragma unroll
     for (int j = 0; j < B; ++j)
       if (c0 + j < nc) O = __fmaf_rn(v[j], cw[c0 + j], O);

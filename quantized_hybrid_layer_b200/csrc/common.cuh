@@ -65,6 +65,31 @@ QHL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
   return false;
 }
 
+// Loads through L2 that the compiler issues exactly where written, once: a
+// batch of them stays a batch (one memory round trip) instead of being sunk to
+// each value's first use, as register pressure can otherwise make it do.
+QHL_DEV uint32_t ld_cg_once(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+QHL_DEV uint4 ld_cg_once(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+QHL_DEV float ld_cg_once(const float* p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+QHL_DEV float2 ld_cg_once(const float2* p) {
+  float2 v;
+  asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+  return v;
+}
+
 // Error path of a kernel that gave up waiting: idle ~200 us so that bulk copies
 // already issued into this CTA's shared memory land before the CTA leaves.
 QHL_DEV void drain_inflight_copies() {
@@ -141,7 +166,7 @@ QHL_DEV float rstd_warp(const float* ss, int ntiles, float inv_dim, float eps, i
   constexpr int B = 8;   // up to 256 tiles in one round of loads
   float v[B];
 #pragma unroll
-  for (int j = 0; j < B; ++j) v[j] = lane + 32 * j < ntiles ? __ldcg(ss + lane + 32 * j) : 0.f;
+  for (int j = 0; j < B; ++j) v[j] = lane + 32 * j < ntiles ? ld_cg_once(ss + lane + 32 * j) : 0.f;
   float s = 0.f;
 #pragma unroll
   for (int j = 0; j < B; ++j)

@@ -16,7 +16,7 @@ cudaError_t set_carveout(K k, cudaFuncAttribute, int smem) {
 
 template <int NT, int EPI>
 cudaError_t one(const GemvArgs& a, int grid, cudaStream_t s, bool pdl) {
-  return launch_ex(qgemv_kernel<kQ8_0, NT, EPI>, dim3(grid), dim3(kGemvThreads),
+  return launch_ex(qgemv_kernel<kQ8_0, NT, EPI>, dim3(grid), dim3(kGemvCtaThreads),
                    (size_t)gemv_smem_bytes<kQ8_0, NT>(), s, pdl, a);
 }
 

@@ -125,6 +125,8 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
     return err(STAGE_E_ARG, "qhl_qgemv: bad argument");
   if (reinterpret_cast<uintptr_t>(packed_dev) % 16 || reinterpret_cast<uintptr_t>(x_dev) % 16)
     return err(STAGE_E_ARG, "qhl_qgemv: packed_dev and x_dev must be 16-byte aligned");
+  if ((long long)packed_tiles(rows, false) * (cols / kChunkCols) >= (1LL << 31))
+    return err(STAGE_E_ARG, "qhl_qgemv: more than 2^31 - 1 packed items");
   const int tiles = packed_tiles(rows, false);
   GemvScratch* s = nullptr;
   int rc = get_scratch(tiles, qtype, (size_t)n_tok * qact_row_bytes(cols), &s);
@@ -145,8 +147,7 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
   a.partials = s->partials;
   a.counters = s->counters;
   a.err = s->err;
-  const long long items = (long long)a.tiles * a.chunks;
-  a.workers = (int)(items < (long long)kCtasPerSm * s->sms ? items : (long long)kCtasPerSm * s->sms);
+  a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * s->sms);
   e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, static_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? 0 : cuda_err("qgemv launch", e);
 }

@@ -69,6 +69,20 @@ inline cudaError_t launch_pass(int qt, int nt, const PassArgs& p, cudaStream_t s
   return qt == kQ4_0 ? PassOps<kQ4_0>::launch(nt, p, s) : PassOps<kQ8_0>::launch(nt, p, s);
 }
 
+// CTAs that own items of a tiles x chunks GEMV on `cap` co-resident CTAs.
+// When the CTAs can own whole tiles -- a divisor of `tiles` no smaller than
+// 85% of `cap` -- no tile is split and no stream-K fix-up runs (the gate/up
+// projection of the 27B shape: 544 tiles on 272 of 296 CTAs); otherwise a
+// balanced stream-K split over min(cap, items) CTAs.  Depends on the shape
+// and `cap` only, never on the token count.
+inline int gemv_workers(int tiles, int chunks, int cap) {
+  if (tiles >= cap)
+    for (int w = cap; w * 100 >= cap * 85; --w)
+      if (tiles % w == 0) return w;
+  const long long items = (long long)tiles * chunks;
+  return (int)(items < cap ? items : cap);
+}
+
 // packed-layout geometry
 inline int packed_tiles(int rows, bool paired) { return paired ? (rows + 31) / 32 : (rows + 63) / 64; }
 inline size_t packed_bytes(int qt, int rows, int cols, bool paired) {

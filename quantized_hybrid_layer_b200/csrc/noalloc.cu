@@ -62,6 +62,8 @@ extern "C" int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* pack
     return fail(STAGE_E_ARG, "bad argument");
   if (reinterpret_cast<uintptr_t>(packed_dev) % 16 || reinterpret_cast<uintptr_t>(x_dev) % 16)
     return fail(STAGE_E_ARG, "packed_dev and x_dev must be 16-byte aligned");
+  if ((long long)packed_tiles(rows, false) * (cols / kChunkCols) >= (1LL << 31))
+    return fail(STAGE_E_ARG, "more than 2^31 - 1 packed items");
   const int tiles = packed_tiles(rows, false);
   const size_t qx_bytes = (size_t)n_tok * qact_row_bytes(cols);
   if (qx_bytes > kQxBytes)
@@ -123,9 +125,7 @@ extern "C" int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* pack
   a.partials = partials;
   a.counters = counters;
   a.err = err;
-  const long long items = (long long)a.tiles * a.chunks;
-  const long long cap = (long long)kCtasPerSm * ds->sms;
-  a.workers = (int)(items < cap ? items : cap);
+  a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * ds->sms);
   if ((e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, s, false)) != cudaSuccess)
     return fail(STAGE_E_CUDA, std::string("qgemv launch: ") + cudaGetErrorString(e));
   return 0;

@@ -51,23 +51,38 @@ struct PassArgs {
   int dn_units;        // Hv * 4
   int Hq, Hkv;
   unsigned* err;
+  // optional phase trace, [grid][n_phases][2] global-timer ns: when this CTA's
+  // consumers start the phase (past the barrier) and when they finish it
+  unsigned long long* trace;
+  int n_phases;
 };
 
-// Shared memory: ring + per-warp partials + rstd + mbarriers + flag + mixer
-// scratch, within ~113 KB so two CTAs share an SM.
+QHL_DEV unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Shared memory: the ring of item stages, then one scratch area shared by the
+// mixer units (attention / combine / DeltaNet / stage input, used by the
+// consumer warps during their phases) and the GEMV tile hand-off (reduction
+// buffers + final tile, used during projection phases), then rstd, mbarriers
+// and flags; within 113 KB so two CTAs share an SM.
 template <int QT, int NT>
 struct PassCfg {
   static constexpr int kIB = QLayout<QT>::kItemBytes;
   static constexpr int kSB = kIB + NT * kQChunkBytes;
-  static constexpr int kMix = 12 * 1024 + NT * 8 * 1024;              // attention / combine / DeltaNet / input scratch
-  static constexpr int kFixed = kConsumerWarps * NT * 64 * 4 + 16 * 4 + 32;
-  static constexpr int kRaw = (113 * 1024 - kFixed - kMix) / (kSB + 16);
-  static constexpr int kStages = kRaw > 12 ? 12 : kRaw;
-  static constexpr int kRedOff = kStages * kSB;
-  static constexpr int kBarOff = kRedOff + kConsumerWarps * NT * 64 * 4 + 16 * 4;
-  static constexpr int kFlagOff = kBarOff + 2 * kStages * 8;
-  static constexpr int kMixOff = (kFlagOff + 16 + 15) / 16 * 16;
-  static constexpr int kSmem = kMixOff + kMix;
+  static constexpr int kMixUnits = 12 * 1024 + NT * 8 * 1024;
+  static constexpr int kTileBytes = TileRing<NT>::kBytes + NT * 64 * 4;
+  static constexpr int kMix = kMixUnits > kTileBytes ? kMixUnits : kTileBytes;
+  static constexpr int kFixed = kMix + 16 * 4 + 2 * TileRing<NT>::kBufs * 8 + 16;
+  static constexpr int kRaw = (113 * 1024 - kFixed) / (kSB + 16);
+  static constexpr int kStages = kRaw > 16 ? 16 : kRaw;
+  static constexpr int kMixOff = kStages * kSB;                     // 16-byte aligned: kSB is a multiple of 16
+  static constexpr int kRstdOff = kMixOff + kMix;
+  static constexpr int kBarOff = kRstdOff + 16 * 4;
+  static constexpr int kFlagOff = kBarOff + (2 * kStages + 2 * TileRing<NT>::kBufs) * 8;
+  static constexpr int kSmem = kFlagOff + 16;
   // A deep enough ring and two CTAs per SM (Q8_0 at 4 tokens does not fit:
   // that pass runs as separate kernels).
   static constexpr bool kFits = kRaw >= 3 && kSmem <= 113 * 1024;
@@ -84,14 +99,16 @@ QHL_DEV unsigned ld_acquire(const unsigned* p) {
 // Order global data acquired through the generic proxy before later bulk
 // copies (async proxy) that read it.
 QHL_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-QHL_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
+// Wait (suspended, at most about `ns` nanoseconds) for the phase with the
+// given parity to complete; true once it has.
+QHL_DEV bool mbar_wait_for(uint32_t bar, uint32_t parity, uint32_t ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }
@@ -99,6 +116,12 @@ QHL_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
 // Spin bound of every grid-barrier and ring wait (seconds: far beyond any
 // legitimate wait, short of a hung GPU).
 constexpr uint32_t kSpinLimit = 1u << 24;
+
+// Grid-barrier arrival: add 1 with release semantics (the CTA's writes,
+// ordered before this thread by the preceding barrier, become visible with it).
+QHL_DEV void red_add_release(unsigned* p) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory");
+}
 
 QHL_DEV unsigned ld_relaxed(const unsigned* p) {
   unsigned v;
@@ -131,6 +154,7 @@ QHL_DEV bool grid_wait(const PassArgs& p, int ph, int* sflag, unsigned* ready) {
     const unsigned target = (unsigned)ph * (unsigned)p.grid;
     int ok = 1;
     for (uint32_t i = 0; ld_relaxed(p.bar) < target; ++i) {
+      __nanosleep(64);   // keep the polling of the counter's L2 line light
       if ((i & 63u) == 63u && ld_relaxed(p.err)) {
         ok = 0;
         break;
@@ -143,6 +167,7 @@ QHL_DEV bool grid_wait(const PassArgs& p, int ph, int* sflag, unsigned* ready) {
     }
     (void)ld_acquire(p.bar);
     if (ok) st_release_cta(ready, (unsigned)ph);
+    if (p.trace) p.trace[((size_t)blockIdx.x * p.n_phases + ph) * 2] = global_ns();
     *sflag = ok;
   }
   named_sync(1, 256);
@@ -152,12 +177,12 @@ QHL_DEV bool grid_wait(const PassArgs& p, int ph, int* sflag, unsigned* ready) {
 // Consumers: this CTA finished its share of the current phase.  Every thread
 // orders its global writes before later bulk copies (async proxy) that other
 // CTAs make of them; thread 0 then releases the arrival.
-QHL_DEV void grid_arrive(const PassArgs& p) {
+QHL_DEV void grid_arrive(const PassArgs& p, int ph) {
   fence_proxy_async_global();
   named_sync(1, 256);
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(p.bar, 1u);
+    if (p.trace) p.trace[((size_t)blockIdx.x * p.n_phases + ph) * 2 + 1] = global_ns();
+    red_add_release(p.bar);
   }
 }
 
@@ -205,17 +230,15 @@ QHL_DEV void pass_producer(const PassArgs& p, int cta, uint8_t* stages, uint64_t
     for (int gi = 0; gi < 4; ++gi) {
       const GemvArgs& a = L.g[gi];
       if (cta >= a.workers) continue;
-      const long long n_items = (long long)a.tiles * a.chunks;
-      const long long i0 = sk_begin(cta, n_items, a.workers);
-      const long long i1 = sk_begin(cta + 1, n_items, a.workers);
-      int c = (int)(i0 % a.chunks);
-      for (long long it = i0; it < i1; ++it, ++k) {
+      const StreamK sk(a.tiles * a.chunks, a.workers);
+      const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1);
+      int c = i0 % a.chunks;
+      for (int it = i0; it < i1; ++it, ++k) {
         if (round > 0) {
           const uint32_t empty = smem_u32(&bars[S + slot]);
           const uint32_t par = (round - 1) & 1u;
-          for (uint32_t spins = 0; !mbar_test(empty, par); ++spins) {
+          for (uint32_t spins = 0; !mbar_wait_for(empty, par, 256); ++spins) {
             service();
-            __nanosleep(20);
             if ((spins & 63u) == 63u && ld_relaxed(p.err)) {
               pass_drain();
               return;
@@ -229,7 +252,7 @@ QHL_DEV void pass_producer(const PassArgs& p, int cta, uint8_t* stages, uint64_t
         }
         const uint32_t full = smem_u32(&bars[slot]);
         mbar_arrive_expect_tx(full, SB);
-        bulk_g2s(smem_u32(stages + slot * SB), a.W + it * IB, IB, full, pol);
+        bulk_g2s(smem_u32(stages + slot * SB), a.W + (size_t)it * IB, IB, full, pol);
         int qt = qh + qn;
         if (qt >= S) qt -= S;
         q[qt] = XJob{a.qx + (size_t)c * kQChunkBytes, a.qx_stride, slot, phases[gi]};
@@ -245,7 +268,7 @@ QHL_DEV void pass_producer(const PassArgs& p, int cta, uint8_t* stages, uint64_t
   }
   for (uint32_t spins = 0; qn > 0; ++spins) {
     service();
-    __nanosleep(20);
+    __nanosleep(128);
     if ((spins & 63u) == 63u && ld_relaxed(p.err)) break;
     if (spins == kSpinLimit) {
       atomicOr(p.err, ERR_WAIT_TIMEOUT);
@@ -255,78 +278,138 @@ QHL_DEV void pass_producer(const PassArgs& p, int cta, uint8_t* stages, uint64_t
   if (qn > 0) pass_drain();
 }
 
+// The epilogue warp's arrival at the grid barrier after its share of a
+// projection phase: every lane orders its global writes before later bulk
+// copies that other CTAs make of them, lane 0 releases the arrival.
+QHL_DEV void epilogue_arrive(const PassArgs& p, int ph) {
+  fence_proxy_async_global();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    if (p.trace) p.trace[((size_t)blockIdx.x * p.n_phases + ph) * 2 + 1] = global_ns();
+    red_add_release(p.bar);
+  }
+}
+
+// Epilogue warp: wait until this CTA's consumers have seen phase `ph` open
+// (so the previous step's outputs, the RMS partials among them, are visible).
+// False if the pass is aborted.
+QHL_DEV bool epilogue_wait(const PassArgs& p, int ph, const unsigned* ready_sm) {
+  for (uint32_t i = 0; ld_acquire_cta(ready_sm) < (unsigned)ph; ++i) {
+    if ((i & 63u) == 63u && ld_relaxed(p.err)) return false;
+    if (i == kSpinLimit) {
+      atomicOr(p.err, ERR_WAIT_TIMEOUT);
+      return false;
+    }
+    __nanosleep(128);
+  }
+  return true;
+}
+
+// Epilogue warp over the whole pass: finishes every projection's tiles of this
+// CTA and arrives at the barrier that closes each projection phase.
+template <int NT>
+QHL_DEV void pass_epilogue(const PassArgs& p, int cta, const TileSync& ts, float* fin, float* rstd,
+                           const unsigned* ready_sm) {
+  uint32_t tc = 0;
+  bool timed_out = false;
+  for (int l = 0; l < p.n_layers; ++l) {
+    const PassLayer& L = p.layers[l];
+    const int ph_out = L.phase_in + (L.attn ? 3 : 2);
+    if (!epilogue_wait(p, L.phase_in, ready_sm)) break;
+    gemv_finish<EPI_STORE, NT>(L.g[0], cta, ts, fin, rstd, tc, timed_out);
+    epilogue_arrive(p, L.phase_in);
+    if (!epilogue_wait(p, ph_out, ready_sm)) break;
+    gemv_finish<EPI_RESID, NT>(L.g[1], cta, ts, fin, rstd, tc, timed_out);
+    epilogue_arrive(p, ph_out);
+    if (!epilogue_wait(p, ph_out + 1, ready_sm)) break;
+    gemv_finish<EPI_SWIGLU, NT>(L.g[2], cta, ts, fin, rstd, tc, timed_out);
+    epilogue_arrive(p, ph_out + 1);
+    if (!epilogue_wait(p, ph_out + 2, ready_sm)) break;
+    gemv_finish<EPI_RESID, NT>(L.g[3], cta, ts, fin, rstd, tc, timed_out);
+    epilogue_arrive(p, ph_out + 2);
+  }
+}
+
 template <int QT, int NT>
-__global__ void __launch_bounds__(kGemvThreads, 2) stage_pass_kernel(const PassArgs p) {
+__global__ void __launch_bounds__(kGemvCtaThreads, 2) stage_pass_kernel(const PassArgs p) {
   using C = PassCfg<QT, NT>;
   constexpr int S = C::kStages;
+  constexpr int RB = TileRing<NT>::kBufs;
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* stages = smem;
-  float* red = reinterpret_cast<float*>(smem + C::kRedOff);
-  float* rstd = red + kConsumerWarps * NT * 64;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint8_t* mix = smem + C::kMixOff;                                   // mixer scratch / tile hand-off
+  float* rstd = reinterpret_cast<float*>(smem + C::kRstdOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);   // full[S], empty[S], tile full[RB], tile free[RB]
+  const TileSync ts{reinterpret_cast<float*>(mix), bars + 2 * S, bars + 2 * S + RB};
+  float* fin = reinterpret_cast<float*>(mix + TileRing<NT>::kBytes);
   int* flag = reinterpret_cast<int*>(smem + C::kFlagOff);
-  uint8_t* mix = smem + C::kMixOff;
+  int* abort_flag = flag + 1;
+  unsigned* ready_sm = reinterpret_cast<unsigned*>(flag + 2);         // phases seen complete
 
   const int cta = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5;
-  unsigned* ready_sm = reinterpret_cast<unsigned*>(flag + 2);   // phases seen complete
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&bars[s]), 1);
       mbar_init(smem_u32(&bars[S + s]), kConsumerWarps);
     }
+    for (int b = 0; b < RB; ++b) {
+      mbar_init(smem_u32(&ts.full[b]), kConsumerWarps * 32);
+      mbar_init(smem_u32(&ts.free_[b]), 32);
+    }
     fence_mbar_init();
     *ready_sm = 0;
   }
   __syncthreads();
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     if ((tid & 31) == 0) pass_producer<QT, NT, S>(p, cta, stages, bars, ready_sm);
     return;
   }
+  if (warp == kEpilogueWarp) {
+    pass_epilogue<NT>(p, cta, ts, fin, rstd, ready_sm);
+    return;
+  }
 
+  // ---- consumers: items of every projection, and the mixer / input units ----
   int slot = 0;
-  uint32_t parity = 0;
+  uint32_t parity = 0, tc = 0;
   bool timed_out = false;
   int ph = 0;
-  int* abort_flag = flag + 1;
+  if (p.trace && tid == 0) p.trace[(size_t)cta * p.n_phases * 2] = global_ns();
   for (int u = cta; u < p.H / 64; u += p.grid)
     input_unit<NT>(p.h, p.H, p.gamma0, p.qz, p.qz_stride, p.ss, p.ss_stride, u, reinterpret_cast<float*>(mix));
-  grid_arrive(p);
+  grid_arrive(p, 0);
   ++ph;
-#define QHL_PASS_WAIT()                       \
-  if (!grid_wait(p, ph++, abort_flag, ready_sm)) { \
-    if (tid == 0) pass_drain();               \
-    return;                                   \
+#define QHL_PASS_WAIT()                                 \
+  if (!grid_wait(p, ph++, abort_flag, ready_sm)) {      \
+    if (tid == 0) pass_drain();                         \
+    return;                                             \
   }
   for (int l = 0; l < p.n_layers; ++l) {
     const PassLayer& L = p.layers[l];
     QHL_PASS_WAIT();
-    gemv_consume<QT, NT, EPI_STORE, S>(L.g[0], cta, stages, bars, red, rstd, flag, slot, parity, timed_out);
-    grid_arrive(p);
+    gemv_consume<QT, NT, S>(L.g[0], cta, stages, bars, ts, slot, parity, tc, timed_out);   // the epilogue warp arrives
     if (!L.attn) {
       QHL_PASS_WAIT();
       for (int u = cta; u < p.dn_units; u += p.grid) dn_unit<NT>(L.dn, u, reinterpret_cast<float(*)[32]>(mix));
-      grid_arrive(p);
+      grid_arrive(p, ph - 1);
     } else {
       QHL_PASS_WAIT();
       const int pos = *p.kv_len;
       const int units = (pos + NT + kAttChunk - 1) / kAttChunk * p.Hkv;
       for (int u = cta; u < units; u += p.grid) attn_unit<NT>(L.at, u / p.Hkv, u % p.Hkv, pos, mix);
-      grid_arrive(p);
+      grid_arrive(p, ph - 1);
       QHL_PASS_WAIT();
       for (int u = cta; u < NT * p.Hq; u += p.grid)
         combine_unit<NT>(L.at, u / p.Hq, u % p.Hq, pos, reinterpret_cast<float*>(mix));
-      grid_arrive(p);
+      grid_arrive(p, ph - 1);
     }
     QHL_PASS_WAIT();
-    gemv_consume<QT, NT, EPI_RESID, S>(L.g[1], cta, stages, bars, red, rstd, flag, slot, parity, timed_out);
-    grid_arrive(p);
+    gemv_consume<QT, NT, S>(L.g[1], cta, stages, bars, ts, slot, parity, tc, timed_out);
     QHL_PASS_WAIT();
-    gemv_consume<QT, NT, EPI_SWIGLU, S>(L.g[2], cta, stages, bars, red, rstd, flag, slot, parity, timed_out);
-    grid_arrive(p);
+    gemv_consume<QT, NT, S>(L.g[2], cta, stages, bars, ts, slot, parity, tc, timed_out);
     QHL_PASS_WAIT();
-    gemv_consume<QT, NT, EPI_RESID, S>(L.g[3], cta, stages, bars, red, rstd, flag, slot, parity, timed_out);
-    grid_arrive(p);
+    gemv_consume<QT, NT, S>(L.g[3], cta, stages, bars, ts, slot, parity, tc, timed_out);
   }
 #undef QHL_PASS_WAIT
   if (timed_out && tid == 0) pass_drain();
@@ -363,7 +446,7 @@ template <int QT, int NT>
 cudaError_t pass_occupancy_one(int* blocks) {
   *blocks = 0;
   if constexpr (PassCfg<QT, NT>::kFits)
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, stage_pass_kernel<QT, NT>, kGemvThreads,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, stage_pass_kernel<QT, NT>, kGemvCtaThreads,
                                                          PassCfg<QT, NT>::kSmem);
   else
     return cudaSuccess;
@@ -374,7 +457,7 @@ cudaError_t pass_launch_one(const PassArgs& p, cudaStream_t s) {
   if constexpr (PassCfg<QT, NT>::kFits) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(kGemvThreads);
+    cfg.blockDim = dim3(kGemvCtaThreads);
     cfg.dynamicSmemBytes = PassCfg<QT, NT>::kSmem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

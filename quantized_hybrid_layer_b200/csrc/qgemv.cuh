@@ -64,40 +64,27 @@ struct GemvArgs {
 };
 
 constexpr int kConsumerWarps = 8;
-constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;
 // Stream-K workers per SM: the grid is kCtasPerSm * SMs for every token count
 // (the split, and hence the summation order, must not depend on NT).
 constexpr int kCtasPerSm = 2;
 
-// A stage holds one item's packed weights followed by the item's x chunk for
-// every token ([NT][864] bytes).  Up to 2 tokens the ring is small enough for
-// two CTAs of this kernel plus one of the next (under programmatic dependent
-// launch) to share an SM; up to 4 tokens two CTAs fit; beyond that one CTA per
-// SM runs at a time.
-template <int QT, int NT>
-struct GemvCfg {
-  static constexpr int kStageBytes = QLayout<QT>::kItemBytes + NT * kQChunkBytes;
-  static constexpr int kBudget = NT <= 2 ? 72 * 1024 : (NT <= 4 ? 104 * 1024 : 196 * 1024);
-  static constexpr int kRaw = (kBudget - kConsumerWarps * NT * 64 * 4 - 512) / kStageBytes;
-  static constexpr int kStages = kRaw < 3 ? 3 : (kRaw > 12 ? 12 : kRaw);
-  static constexpr int kMinBlocks = NT <= 2 ? 3 : (NT <= 4 ? 2 : 1);
+// Balanced contiguous split of n items (n < 2^31) over p CTAs: CTA w owns
+// items [begin(w), begin(w + 1)) with begin(w) = floor(w n / p), evaluated in
+// 32-bit arithmetic as w q + floor(w r / p) (q = n / p, r = n % p).
+struct StreamK {
+  int n, p, q, r;
+  __host__ __device__ StreamK(int n_, int p_) : n(n_), p(p_), q(n_ / p_), r(n_ % p_) {}
+  __host__ __device__ int begin(int w) const { return w * q + (w * r) / p; }
+  // The CTA owning item i: the largest w with begin(w) <= i (a float estimate,
+  // then exact integer steps).
+  __host__ __device__ int owner(int i) const {
+    int w = (int)(((float)i + 0.5f) * (float)p / (float)n);
+    w = w < 0 ? 0 : (w >= p ? p - 1 : w);
+    while (w + 1 < p && begin(w + 1) <= i) ++w;
+    while (w > 0 && begin(w) > i) --w;
+    return w;
+  }
 };
-
-template <int QT, int NT>
-constexpr int gemv_smem_bytes() {
-  return GemvCfg<QT, NT>::kStages * GemvCfg<QT, NT>::kStageBytes   // stage ring
-         + kConsumerWarps * NT * 64 * 4                           // per-warp tile partials
-         + 16 * 4                                                 // rstd
-         + 2 * GemvCfg<QT, NT>::kStages * 8                       // full/empty mbarriers
-         + 16;                                                    // flags
-}
-
-// First item of CTA `w` in a balanced contiguous split of `n` items over `p` CTAs.
-__host__ __device__ inline long long sk_begin(long long w, long long n, long long p) { return (w * n) / p; }
-// CTA owning item i (the largest w with sk_begin(w) <= i).
-__host__ __device__ inline long long sk_owner(long long i, long long n, long long p) {
-  return ((i + 1) * p - 1) / n;
-}
 
 // The quants and scales one lane reads from a stage: its two rows of block `warp`.
 template <int QT> struct ItemRegs;
@@ -205,19 +192,72 @@ QHL_DEV void compute_item(const ItemRegs<QT>& r, const uint8_t* xs, int warp, fl
   }
 }
 
-// Epilogue for one finished tile; vals = [NT][64] final sums in shared memory.
-// Called by all 256 consumer threads.
+// ---------------------------------------------------------------------------
+// Warp roles of a GEMV CTA: warps 0..7 consume items, warp 8 produces (bulk
+// copies into the ring), warp 9 finishes tiles.  The consumers hand each
+// finished tile's per-warp sums to the epilogue warp through a small ring of
+// reduction buffers (mbarriers "tile full" / "tile free") and go straight on
+// with the next item; the epilogue warp sums the eight warps' partials, runs
+// the stream-K fix-up and the fused epilogue off the item loop's path.
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kEpilogueWarp = kConsumerWarps + 1;
+constexpr int kGemvCtaThreads = (kConsumerWarps + 2) * 32;
+
+// Reduction buffers between consumers and the epilogue warp.
+template <int NT>
+struct TileRing {
+  static constexpr int kBufs = NT <= 4 ? 2 : 1;
+  static constexpr int kBufFloats = kConsumerWarps * NT * 64;   // [8][NT][64]
+  static constexpr int kBytes = kBufs * kBufFloats * 4;
+};
+
+// Hand-off state shared by the consumers and the epilogue warp of one CTA.
+struct TileSync {
+  float* red;          // [kBufs][8][NT][64]
+  uint64_t* full;      // [kBufs], 256 arrivals (every consumer thread)
+  uint64_t* free_;     // [kBufs], 32 arrivals (every epilogue lane)
+};
+
+// Inputs of a tile's epilogue that do not depend on the tile's sums, loaded
+// before the sums are ready: the residual stream h (written by an earlier
+// step) and the next RMSNorm weight, for the lanes' elements.
+template <int NT>
+struct EpiInputs {
+  float h[NT * 2];     // element i * 32 + lane of [NT][64]
+  float gamma[2];      // rows lane and 32 + lane
+};
+
 template <int EPI, int NT>
-QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float* rstd, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
+QHL_DEV void gemv_prefetch(const GemvArgs& a, int tile, int lane, EpiInputs<NT>& in) {
+  if constexpr (EPI == EPI_RESID) {
+#pragma unroll
+    for (int i = 0; i < NT * 2; ++i) {
+      const int idx = i * 32 + lane, t = idx >> 6, gr = tile * 64 + (idx & 63);
+      in.h[i] = gr < a.out_valid ? ld_cg_once(a.y + (size_t)t * a.y_stride + gr) : 0.f;   // h: written by other CTAs
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int gr = tile * 64 + b * 32 + lane;
+      in.gamma[b] = a.qout && gr < a.out_valid ? __ldg(a.gamma_next + gr) : 0.f;
+    }
+  }
+}
+
+// Epilogue of one finished tile by the 32 lanes of the epilogue warp;
+// vals = [NT][64] final sums in shared memory, rstd = [NT].
+template <int EPI, int NT>
+QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float* rstd, int lane,
+                           const EpiInputs<NT>& in) {
   if constexpr (EPI == EPI_STORE) {
-    for (int idx = tid; idx < NT * 64; idx += 256) {
-      const int t = idx >> 6, row = idx & 63, gr = tile * 64 + row;
+#pragma unroll
+    for (int i = 0; i < NT * 2; ++i) {
+      const int idx = i * 32 + lane, t = idx >> 6, gr = tile * 64 + (idx & 63);
       if (gr < a.out_valid) a.y[(size_t)t * a.y_stride + gr] = __fmul_rn(vals[idx], rstd[t]);
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
     // tile rows 0..31 are gate rows of features tile*32.., rows 32..63 the matching up rows
-    for (int t = warp; t < NT; t += kConsumerWarps) {
+#pragma unroll 1
+    for (int t = 0; t < NT; ++t) {
       const int f = tile * 32 + lane;
       float u = 0.f;
       if (f < a.out_valid) {
@@ -228,59 +268,64 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float
       qact_store_block(u, a.qout + (size_t)t * a.qout_stride, tile, lane);
     }
   } else {
-    for (int idx = tid; idx < NT * 64; idx += 256) {
-      const int t = idx >> 6, row = idx & 63, gr = tile * 64 + row;
+#pragma unroll
+    for (int i = 0; i < NT * 2; ++i) {
+      const int idx = i * 32 + lane, t = idx >> 6, gr = tile * 64 + (idx & 63);
       float hn = 0.f;
       if (gr < a.out_valid) {
-        float* hp = a.y + (size_t)t * a.y_stride + gr;
-        hn = __fadd_rn(__ldcg(hp), vals[idx]);   // through L2: h may come from another CTA of the same kernel
-        *hp = hn;
+        hn = __fadd_rn(in.h[i], vals[idx]);
+        a.y[(size_t)t * a.y_stride + gr] = hn;
       }
       vals[idx] = hn;
     }
-    named_sync(1, 256);
+    __syncwarp();
     if (a.qout) {
-      for (int p = warp; p < NT * 2; p += kConsumerWarps) {
+#pragma unroll 1
+      for (int p = 0; p < NT * 2; ++p) {
         const int t = p >> 1, b = p & 1, gr = tile * 64 + b * 32 + lane;
-        const float z = gr < a.out_valid ? __fmul_rn(vals[t * 64 + b * 32 + lane], a.gamma_next[gr]) : 0.f;
+        const float z = gr < a.out_valid ? __fmul_rn(vals[t * 64 + b * 32 + lane], b ? in.gamma[1] : in.gamma[0]) : 0.f;
         qact_store_block(z, a.qout + (size_t)t * a.qout_stride, tile * 2 + b, lane);
       }
     }
-    if (a.ss_out && tid < NT) a.ss_out[(size_t)tid * a.ss_out_stride + tile] = sumsq64(vals + tid * 64);
+    if (a.ss_out && lane < NT) a.ss_out[(size_t)lane * a.ss_out_stride + tile] = sumsq64(vals + lane * 64);
+    __syncwarp();
   }
+}
+
+// Stream-K tile counter: add 1 with release (this CTA's partial, published
+// by every lane before the warp barrier, becomes visible with it) and acquire
+// (the last contributor then sees every other partial).
+QHL_DEV int counter_add_acq_rel(int* p) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
 }
 
 // Consumer side of one GEMV for CTA `cta` (the 256 threads of warps 0..7):
 // takes this CTA's stream-K items, in order, from the shared-memory ring
-// (`slot` / `phase` carry the ring position across calls), accumulates,
-// and finishes every tile it touches (directly or through the stream-K
-// partials).  `red` = [8][NT][64] f32, `rstd` = [16] f32, `flag` = one int.
-template <int QT, int NT, int EPI, int S>
-QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t* bars, float* red, float* rstd,
-                          int* flag, int& slot, uint32_t& phase, bool& timed_out) {
+// (`slot` / `phase` carry the ring position across calls) and hands every
+// tile's per-warp sums to the epilogue warp (`tc` counts hand-offs across
+// calls).
+template <int QT, int NT, int S>
+QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t* bars, const TileSync& ts, int& slot,
+                          uint32_t& phase, uint32_t& tc, bool& timed_out) {
   constexpr int IB = QLayout<QT>::kItemBytes;
   constexpr int SB = IB + NT * kQChunkBytes;
+  constexpr int RB = TileRing<NT>::kBufs;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long n_items = (long long)a.tiles * a.chunks;
-  const long long i0 = sk_begin(cta, n_items, a.workers);
-  const long long i1 = sk_begin(cta + 1, n_items, a.workers);
-  const int n_local = cta < a.workers ? (int)(i1 - i0) : 0;
-
+  if (cta >= a.workers) return;
+  const StreamK sk(a.tiles * a.chunks, a.workers);
+  const int i0 = sk.begin(cta), n_local = sk.begin(cta + 1) - i0;
   if (n_local == 0) return;
-  // the input's RMS scale, one warp per token; only the epilogue reads it,
-  // after the first flush's barriers
-  for (int t = warp; t < NT; t += kConsumerWarps) {
-    const float r = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
-    if (lane == 0) rstd[t] = r;
-  }
 
   float r0[NT], r1[NT];
 #pragma unroll
   for (int t = 0; t < NT; ++t) { r0[t] = 0.f; r1[t] = 0.f; }
-  int tile = (int)(i0 / a.chunks);
-  const int first_tile = tile;
-
-  auto flush = [&](int tl) {
+  auto handoff = [&]() {
+    const int buf = (int)(tc % RB);
+    const uint32_t use = tc / RB;
+    if (use > 0 && !timed_out && !mbar_wait(smem_u32(&ts.free_[buf]), (use - 1) & 1u, a.err)) timed_out = true;
+    float* red = ts.red + buf * TileRing<NT>::kBufFloats;
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       red[(warp * NT + t) * 64 + lane] = r0[t];
@@ -288,59 +333,14 @@ QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t*
       r0[t] = 0.f;
       r1[t] = 0.f;
     }
-    named_sync(1, 256);
-    for (int idx = tid; idx < NT * 64; idx += 256) {
-      float v = red[idx];
-#pragma unroll
-      for (int w = 1; w < kConsumerWarps; ++w) v = __fadd_rn(v, red[w * NT * 64 + idx]);
-      red[idx] = v;
-    }
-    named_sync(1, 256);
-    const long long t_lo = (long long)tl * a.chunks, t_hi = t_lo + a.chunks;
-    if (t_lo >= i0 && t_hi <= i1) {
-      gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
-    } else {
-      // stream-K: publish this CTA's partial; the last contributor finishes the tile
-      // (release: the barrier orders every thread's stores before thread 0's
-      // fence and counter increment; acquire: the last arriver's fence after
-      // its increment, then the barrier, orders the partial loads after it)
-      float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * 64;
-      for (int idx = tid; idx < NT * 64; idx += 256) mine[idx] = red[idx];
-      named_sync(1, 256);
-      const long long cf = sk_owner(t_lo, n_items, a.workers);
-      const long long cl = sk_owner(t_hi - 1, n_items, a.workers);
-      if (tid == 0) {
-        __threadfence();
-        const int old = atomicAdd(&a.counters[tl], 1);
-        const int last = (old == (int)(cl - cf)) ? 1 : 0;
-        if (last) __threadfence();
-        *flag = last;
-      }
-      named_sync(1, 256);
-      if (*flag) {
-        for (int idx = tid; idx < NT * 64; idx += 256) {
-          float v = 0.f;
-          for (long long c = cf; c <= cl; ++c) {
-            const int ft = (int)(sk_begin(c, n_items, a.workers) / a.chunks);
-            const float* pc = a.partials + (size_t)(2 * c + (tl == ft ? 0 : 1)) * NT * 64;
-            const float pv = __ldcg(pc + idx);
-            v = (c == cf) ? pv : __fadd_rn(v, pv);
-          }
-          red[idx] = v;
-        }
-        named_sync(1, 256);
-        gemv_epilogue<EPI, NT>(a, tl, red, rstd, tid);
-        if (tid == 0) a.counters[tl] = 0;
-      }
-    }
-    named_sync(1, 256);
+    mbar_arrive(smem_u32(&ts.full[buf]));
+    ++tc;
   };
 
-  int chunk = (int)(i0 - (long long)tile * a.chunks);
+  int chunk = i0 % a.chunks;
   for (int k = 0; k < n_local; ++k) {
     if (chunk == a.chunks) {
-      flush(tile);
-      ++tile;
+      handoff();
       chunk = 0;
     }
     // after one timed-out wait the rest of the call runs without waiting (the
@@ -358,40 +358,160 @@ QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t*
       phase ^= 1u;
     }
   }
-  flush(tile);
+  handoff();
+}
+
+// Epilogue-warp side of one GEMV: for every tile this CTA touches, in order,
+// sum the eight warps' partials (warps 0..7 in order), then either finish the
+// tile (all its chunks were this CTA's) or publish the partial and, if this
+// CTA is the last contributor to arrive, combine every contributor's partial
+// in CTA order and finish it.  `fin` = [NT][64], `rstd` = [NT] (computed
+// here, from the previous step's per-tile sums of squares).
+template <int EPI, int NT>
+QHL_DEV void gemv_finish(const GemvArgs& a, int cta, const TileSync& ts, float* fin, float* rstd, uint32_t& tc,
+                         bool& timed_out) {
+  constexpr int RB = TileRing<NT>::kBufs;
+  const int lane = threadIdx.x & 31;
+  if (cta >= a.workers) return;
+  const StreamK sk(a.tiles * a.chunks, a.workers);
+  const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1);
+  if (i1 == i0) return;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const float r = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
+    if (lane == 0) rstd[t] = r;
+  }
+  __syncwarp();
+  const int first_tile = i0 / a.chunks, last_tile = (i1 - 1) / a.chunks;
+  for (int tl = first_tile; tl <= last_tile; ++tl) {
+    EpiInputs<NT> in;
+    gemv_prefetch<EPI, NT>(a, tl, lane, in);
+    const int buf = (int)(tc % RB);
+    const uint32_t use = tc / RB;
+    if (!timed_out && !mbar_wait(smem_u32(&ts.full[buf]), use & 1u, a.err)) timed_out = true;
+    const float* red = ts.red + buf * TileRing<NT>::kBufFloats;
+#pragma unroll
+    for (int i = 0; i < NT * 2; ++i) {
+      const int idx = i * 32 + lane;
+      float v = red[idx];
+#pragma unroll
+      for (int w = 1; w < kConsumerWarps; ++w) v = __fadd_rn(v, red[w * NT * 64 + idx]);
+      fin[idx] = v;
+    }
+    __syncwarp();
+    mbar_arrive(smem_u32(&ts.free_[buf]));
+    ++tc;
+    const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
+    if (t_lo >= i0 && t_hi <= i1) {
+      gemv_epilogue<EPI, NT>(a, tl, fin, rstd, lane, in);
+      continue;
+    }
+    // stream-K: publish this CTA's partial; the last contributor to arrive
+    // combines every contributor's partial in CTA order and finishes the tile.
+    // Partials move as float2: lane owns elements 2q, 2q + 1, q = j * 32 + lane.
+    float2* mine = reinterpret_cast<float2*>(a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * 64);
+    const float2* fin2 = reinterpret_cast<const float2*>(fin);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) mine[j * 32 + lane] = fin2[j * 32 + lane];
+    __syncwarp();
+    const int cf = sk.owner(t_lo), cl = sk.owner(t_hi - 1);
+    int last = 0;
+    if (lane == 0) last = counter_add_acq_rel(&a.counters[tl]) == cl - cf ? 1 : 0;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) continue;
+    // Tile tl is the first tile of every contributor after cf, and of cf
+    // exactly when cf's range starts at the tile's first item.  Up to 4
+    // float2 loads per lane in flight.
+    constexpr int CB = NT >= 4 ? 1 : 4 / NT;
+    const int cf_slot = sk.begin(cf) == t_lo ? 0 : 1;
+    float2 acc[NT];
+    for (int c0 = cf; c0 <= cl; c0 += CB) {
+      float2 pv[CB][NT];
+#pragma unroll
+      for (int k = 0; k < CB; ++k) {
+        const int c = c0 + k;
+        if (c <= cl) {
+          const float2* pc =
+              reinterpret_cast<const float2*>(a.partials + (size_t)(2 * c + (c == cf ? cf_slot : 0)) * NT * 64);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) pv[k][j] = ld_cg_once(pc + j * 32 + lane);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < CB; ++k)
+        if (c0 + k <= cl) {
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+            acc[j] = (c0 + k == cf) ? pv[k][j]
+                                    : make_float2(__fadd_rn(acc[j].x, pv[k][j].x), __fadd_rn(acc[j].y, pv[k][j].y));
+        }
+    }
+    float2* fout = reinterpret_cast<float2*>(fin);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) fout[j * 32 + lane] = acc[j];
+    __syncwarp();
+    gemv_epilogue<EPI, NT>(a, tl, fin, rstd, lane, in);
+    if (lane == 0) a.counters[tl] = 0;
+  }
+}
+
+template <int QT, int NT>
+struct GemvCfg {
+  static constexpr int kStageBytes = QLayout<QT>::kItemBytes + NT * kQChunkBytes;
+  // two CTAs per SM up to 4 tokens, one beyond
+  static constexpr int kBudget = NT <= 4 ? 112 * 1024 : 200 * 1024;
+  static constexpr int kFixed = TileRing<NT>::kBytes + NT * 64 * 4 + 16 * 4 + 64;
+  static constexpr int kRaw = (kBudget - kFixed) / (kStageBytes + 16);
+  static constexpr int kStages = kRaw < 3 ? 3 : (kRaw > 16 ? 16 : kRaw);
+  static constexpr int kMinBlocks = NT <= 4 ? 2 : 1;
+  // shared-memory layout
+  static constexpr int kRedOff = kStages * kStageBytes;
+  static constexpr int kFinOff = kRedOff + TileRing<NT>::kBytes;
+  static constexpr int kRstdOff = kFinOff + NT * 64 * 4;
+  static constexpr int kBarOff = kRstdOff + 16 * 4;                        // 8-byte aligned
+  static constexpr int kSmem = kBarOff + (2 * kStages + 2 * TileRing<NT>::kBufs) * 8;
+};
+
+template <int QT, int NT>
+constexpr int gemv_smem_bytes() {
+  return GemvCfg<QT, NT>::kSmem;
 }
 
 template <int QT, int NT, int EPI>
-__global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
-  constexpr int S = GemvCfg<QT, NT>::kStages;
+__global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
+  using C = GemvCfg<QT, NT>;
+  constexpr int S = C::kStages;
   constexpr int IB = QLayout<QT>::kItemBytes;
-  constexpr int SB = GemvCfg<QT, NT>::kStageBytes;
+  constexpr int SB = C::kStageBytes;
+  constexpr int RB = TileRing<NT>::kBufs;
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* stages = smem;
-  float* red = reinterpret_cast<float*>(smem + S * SB);                 // [8][NT][64]
-  float* rstd = red + kConsumerWarps * NT * 64;                          // [16]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(rstd + 16);              // full[S], empty[S]
-  int* flag = reinterpret_cast<int*>(bars + 2 * S);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);   // full[S], empty[S], tile full[RB], tile free[RB]
+  const TileSync ts{reinterpret_cast<float*>(smem + C::kRedOff), bars + 2 * S, bars + 2 * S + RB};
+  float* fin = reinterpret_cast<float*>(smem + C::kFinOff);
+  float* rstd = reinterpret_cast<float*>(smem + C::kRstdOff);
 
   const int cta = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) pdl_launch();
   if (cta >= a.workers) return;
-  const long long n_items = (long long)a.tiles * a.chunks;
-  const long long i0 = sk_begin(cta, n_items, a.workers);
-  const long long i1 = sk_begin(cta + 1, n_items, a.workers);
-  const int n_local = (int)(i1 - i0);
+  const StreamK sk(a.tiles * a.chunks, a.workers);
+  const int i0 = sk.begin(cta), n_local = sk.begin(cta + 1) - i0;
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_u32(&bars[s]), 1);
       mbar_init(smem_u32(&bars[S + s]), kConsumerWarps);
     }
+    for (int b = 0; b < RB; ++b) {
+      mbar_init(smem_u32(&ts.full[b]), kConsumerWarps * 32);
+      mbar_init(smem_u32(&ts.free_[b]), 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
+  if (warp == kProducerWarp) {
     // ---------------- producer: stream this CTA's items into the ring ----------
     // Weights never depend on earlier kernels: the first S items' weights are
     // requested before griddepcontrol.wait.  Their x chunks (written by the
@@ -399,7 +519,7 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const int pre = n_local < S ? n_local : S;
-      const int c0 = (int)(i0 % a.chunks);
+      const int c0 = i0 % a.chunks;
       auto issue_x = [&](int k, int s) {
         int c = c0 + k;                    // chunk of local item k, without 64-bit division
         while (c >= a.chunks) c -= a.chunks;
@@ -411,29 +531,36 @@ __global__ void __launch_bounds__(kGemvThreads, GemvCfg<QT, NT>::kMinBlocks) qge
       for (int k = 0; k < pre; ++k) {
         const uint32_t full = smem_u32(&bars[k]);
         mbar_arrive_expect_tx(full, SB);
-        bulk_g2s(smem_u32(stages + k * SB), a.W + (i0 + k) * IB, IB, full, pol);
+        bulk_g2s(smem_u32(stages + k * SB), a.W + (size_t)(i0 + k) * IB, IB, full, pol);
       }
       pdl_wait();
       for (int k = 0; k < pre; ++k) issue_x(k, k);
       for (int k = pre; k < n_local; ++k) {
         const int s = k % S, round = k / S;
-        mbar_wait(smem_u32(&bars[S + s]), (round - 1) & 1, a.err);
+        if (!mbar_wait(smem_u32(&bars[S + s]), (round - 1) & 1, a.err)) {
+          drain_inflight_copies();   // error path
+          return;
+        }
         const uint32_t full = smem_u32(&bars[s]);
         mbar_arrive_expect_tx(full, SB);
-        bulk_g2s(smem_u32(stages + s * SB), a.W + (i0 + k) * IB, IB, full, pol);
+        bulk_g2s(smem_u32(stages + s * SB), a.W + (size_t)(i0 + k) * IB, IB, full, pol);
         issue_x(k, s);
       }
     }
     return;
   }
 
-  // ---------------- consumers ------------------------------------------------
   pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
-  int slot = 0;
-  uint32_t phase = 0;
+  uint32_t tc = 0;
   bool timed_out = false;
-  gemv_consume<QT, NT, EPI, S>(a, cta, stages, bars, red, rstd, flag, slot, phase, timed_out);
-  if (timed_out && tid == 0) drain_inflight_copies();   // error path
+  if (warp == kEpilogueWarp) {
+    gemv_finish<EPI, NT>(a, cta, ts, fin, rstd, tc, timed_out);
+  } else {
+    int slot = 0;
+    uint32_t phase = 0;
+    gemv_consume<QT, NT, S>(a, cta, stages, bars, ts, slot, phase, tc, timed_out);
+  }
+  if (timed_out && lane == 0) drain_inflight_copies();   // error path
 }
 
 }  // namespace qhl

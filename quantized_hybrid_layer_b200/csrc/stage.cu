@@ -95,6 +95,8 @@ struct stage {
   // persistent pass: per-layer step arguments on the device, grid-barrier counter
   PassLayer* pass_layers = nullptr;
   unsigned* bar = nullptr;
+  int n_phases = 0;
+  unsigned long long* trace = nullptr;   // [grid][n_phases][2], when tracing is on
   int pass_mode = STAGE_PASS_PERSISTENT;
   size_t weight_bytes = 0;
   std::string last_error;
@@ -173,10 +175,7 @@ GemvArgs gemv_base(const stage* st) {
   return a;
 }
 
-void set_workers(const stage* st, GemvArgs& a) {
-  const long long items = (long long)a.tiles * a.chunks;
-  a.workers = (int)std::min<long long>((long long)kCtasPerSm * st->sms, items);
-}
+void set_workers(const stage* st, GemvArgs& a) { a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * st->sms); }
 
 // Arguments of every step of layer i (shared by both execution paths, so they
 // run the same units with the same split).
@@ -354,6 +353,8 @@ cudaError_t record_persistent(stage* st, int n, cudaStream_t s) {
   p.Hq = c.att_q_heads;
   p.Hkv = c.att_kv_heads;
   p.err = st->err;
+  p.trace = st->trace;
+  p.n_phases = st->n_phases;
   return launch_pass(c.qtype, n, p, s);
 }
 
@@ -599,6 +600,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
       pl[i].phase_in = phase;
       phase += pl[i].attn ? 6 : 5;   // in-proj, mixer (attention: partials + combine), out, gate/up, down
     }
+    st->n_phases = phase;
     if ((s = dalloc_t(st, &st->pass_layers, pl.size() * sizeof(PassLayer))) != STAGE_OK ||
         (s = dalloc_t(st, &st->bar, 16)) != STAGE_OK)
       return bail(s);
@@ -773,6 +775,42 @@ stage_status stage_set_pass_mode(stage_t* st, int mode) {
       g = nullptr;
     }
   st->pass_mode = mode;
+  return STAGE_OK;
+}
+
+stage_status stage_set_trace(stage_t* st, int enable) {
+  if (!st) return STAGE_E_ARG;
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  if ((enable != 0) == (st->trace != nullptr)) return STAGE_OK;
+  CK(cudaStreamSynchronize(st->stream));
+  for (auto& g : st->exec)
+    if (g) {
+      CK(cudaGraphExecDestroy(g));
+      g = nullptr;
+    }
+  if (enable) {
+    const size_t bytes = (size_t)kCtasPerSm * st->sms * st->n_phases * 2 * sizeof(unsigned long long);
+    stage_status s = dalloc_t(st, &st->trace, bytes);
+    if (s != STAGE_OK) return s;
+    CK(cudaMemset(st->trace, 0, bytes));
+  } else {
+    cudaFree(st->trace);
+    st->allocs.erase(std::remove(st->allocs.begin(), st->allocs.end(), (void*)st->trace), st->allocs.end());
+    st->trace = nullptr;
+  }
+  return STAGE_OK;
+}
+
+stage_status stage_get_trace(stage_t* st, unsigned long long* host_dst, size_t count, int* grid, int* n_phases) {
+  if (!st) return STAGE_E_ARG;
+  if (!st->trace) return fail(st, STAGE_E_STATE, "tracing is off");
+  const size_t need = (size_t)kCtasPerSm * st->sms * st->n_phases * 2;
+  if (grid) *grid = kCtasPerSm * st->sms;
+  if (n_phases) *n_phases = st->n_phases;
+  if (!host_dst) return STAGE_OK;
+  if (count != need) return fail(st, STAGE_E_ARG, "count must be grid * n_phases * 2");
+  CK(cudaStreamSynchronize(st->stream));
+  CK(cudaMemcpy(host_dst, st->trace, need * sizeof(unsigned long long), cudaMemcpyDeviceToHost));
   return STAGE_OK;
 }
 

@@ -280,3 +280,28 @@ def test_persistent_pass_equals_kernel_chain(q, qtype, ns):
         assert e.value.code == -1
     finally:
         st.free()
+
+
+def test_persistent_pass_trace_shows_the_grid_barriers(q):
+    """With tracing on, every CTA records each phase; no CTA starts a phase
+    before every CTA has finished the previous one (the grid barrier)."""
+    st, _, _ = make_pair(FULL, Q4_0, 8, 0, 4, MAX_CTX, CTX, with_oracle=False)
+    try:
+        with pytest.raises(q.StageError):
+            st.get_trace()                                   # off by default
+        st.set_trace(True)
+        h = synth.hidden(FULL, 8, 0, 1)
+        run(st, h, CTX)
+        st.rollback()
+        tr = st.get_trace().astype(np.int64)
+        grid, n_phases, _ = tr.shape
+        assert n_phases == 1 + 3 * 5 + 6                      # input, 3 DeltaNet layers, 1 attention layer
+        assert (tr > 0).all()
+        assert (tr[:, :, 1] >= tr[:, :, 0]).all()
+        for ph in range(1, n_phases):
+            assert tr[:, ph, 0].min() >= tr[:, ph - 1, 1].max(), ph
+        st.set_trace(False)
+        run(st, h, CTX)                                       # still runs without the trace buffer
+        st.rollback()
+    finally:
+        st.free()
