@@ -148,7 +148,7 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
   a.counters = s->counters;
   a.err = s->err;
   a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * s->sms);
-  e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, static_cast<cudaStream_t>(stream), false);
+  e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, static_cast<cudaStream_t>(stream), true);
   return e == cudaSuccess ? 0 : cuda_err("qgemv launch", e);
 }
 

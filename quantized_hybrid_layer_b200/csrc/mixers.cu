@@ -35,8 +35,11 @@ __global__ void __launch_bounds__(256) stage_input_kernel(const float* h, int H,
   input_unit<NT>(h, H, gamma, qz, qz_stride, ss, ss_stride, blockIdx.x, sm);
 }
 
-// f32 rows -> block fixed point, one warp per (token, 32-column block).
+// f32 rows -> block fixed point, one warp per (token, 32-column block).  The
+// GEMV that follows is launched as a programmatic dependent: it may start
+// streaming weights at once and waits (griddepcontrol.wait) before reading qx.
 __global__ void quantize_rows_kernel(const float* x, int n, int cols, uint8_t* qx) {
+  if (threadIdx.x == 0) pdl_launch();
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31, nb = cols / 32;
   if (gw >= (long long)n * nb) return;

@@ -126,7 +126,7 @@ extern "C" int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* pack
   a.counters = counters;
   a.err = err;
   a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * ds->sms);
-  if ((e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, s, false)) != cudaSuccess)
+  if ((e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, s, true)) != cudaSuccess)
     return fail(STAGE_E_CUDA, std::string("qgemv launch: ") + cudaGetErrorString(e));
   return 0;
 }

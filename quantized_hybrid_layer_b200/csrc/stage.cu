@@ -36,11 +36,11 @@ namespace {
 
 constexpr int kMaxTok = 16;
 constexpr int kRing = kMaxTok + 1;
-// Programmatic dependent launch between the pass's kernels.  Measured on the
-// 8-layer decode pass it cost ~12% (801 vs 709 us), so the graph uses plain
-// stream order; the kernels still carry griddepcontrol.wait / launch_dependents
-// (no-ops without the launch attribute).
-constexpr bool kUsePdl = false;
+// Programmatic dependent launch between the pass's kernels: as the CTAs of a
+// projection finish, the next kernel's CTAs take their place and start
+// streaming weights while the last tiles are still being finished.  Measured
+// on the 64-layer decode pass: 4.19 ms with it, 4.73 ms in plain stream order.
+constexpr bool kUsePdl = true;
 
 struct Layer {
   int index = 0;
