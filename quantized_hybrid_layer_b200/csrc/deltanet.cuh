@@ -54,18 +54,24 @@ QHL_DEV float dot4(float4 a, float4 b) {
 // One unit: 32 rows of value head `unit / 4` (8 warps x 4 rows), all NT tokens.
 // ob: shared [NT][32] for the unit's outputs.  q, k, v, b, a are read through
 // L2 (they may have been written earlier in the same kernel by another CTA).
+// The unit's starting state rows (they never depend on the kernel before).
 template <int NT>
-QHL_DEV void dn_unit(const DnArgs& a, int unit, float (*ob)[32]) {
+QHL_DEV void dn_load(const DnArgs& a, int unit, float4 (&S)[4]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = unit >> 2, row0 = (unit & 3) * 32 + warp * 4;
+  const float* s_in = a.cur ? a.ring + (size_t)(*a.cur) * a.state_elems : a.s_in;
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+    S[r] = __ldg(reinterpret_cast<const float4*>(s_in + ((size_t)h * kDnDim + row0 + r) * kDnDim) + lane);
+}
+
+template <int NT>
+QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float (*ob)[32]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = unit >> 2;                       // 4 units of 32 rows per head
   const int row0 = (unit & 3) * 32 + warp * 4;
   const int g = h / (a.Hv / a.Hk);
   const int cur = a.cur ? *a.cur : 0;
-  const float* s_in = a.cur ? a.ring + (size_t)cur * a.state_elems : a.s_in;
-  float4 S[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-    S[r] = __ldg(reinterpret_cast<const float4*>(s_in + ((size_t)h * kDnDim + row0 + r) * kDnDim) + lane);
 
   const int off_k = a.Hk * kDnDim;
   const int off_v = 2 * a.Hk * kDnDim;
@@ -111,11 +117,20 @@ QHL_DEV void dn_unit(const DnArgs& a, int unit, float (*ob)[32]) {
 }
 
 template <int NT>
+QHL_DEV void dn_unit(const DnArgs& a, int unit, float (*ob)[32]) {
+  float4 S[4];
+  dn_load<NT>(a, unit, S);
+  dn_run<NT>(a, unit, S, ob);
+}
+
+template <int NT>
 __global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
   __shared__ float ob[NT][32];
   if (threadIdx.x == 0) pdl_launch();
-  pdl_wait();
-  dn_unit<NT>(a, blockIdx.x, ob);
+  float4 S[4];
+  dn_load<NT>(a, blockIdx.x, S);   // overlaps the in-projection's last tiles
+  pdl_wait();                      // q, k, v, b, a come from it
+  dn_run<NT>(a, blockIdx.x, S, ob);
 }
 
 }  // namespace qhl
