@@ -193,6 +193,123 @@ QHL_DEV void compute_item(const ItemRegs<QT>& r, const uint8_t* xs, int warp, fl
 }
 
 // ---------------------------------------------------------------------------
+// Integer tensor-core path (n_tok >= kMmaTok): the same exact int32 block sums
+// as the dp4a path, formed by mma.sync m16n8k32 (8-bit A = weights, B = one
+// activation byte plane, columns = tokens), so both paths give bit-identical
+// results and a 16-token verify still equals 16 single-token passes.  Warp w
+// still owns block w of each item; its 64 rows are 4 m-tiles of 16.  The
+// k order inside a block is GGUF's own: byte j of a Q4_0 row holds elements j
+// (low nibble) and j + 16 (high nibble), which is exactly the split of the
+// A fragment's k range into [4c, 4c + 4) and [16 + 4c, 16 + 4c + 4).
+constexpr int kMmaTok = 4;
+
+template <bool AS, bool BS>
+QHL_DEV void mma_i8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+#define QHL_MMA_I8(AT, BT)                                                                         \
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32." AT "." BT ".s32 {%0, %1, %2, %3}, "        \
+               "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"                                 \
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])                                    \
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0))
+  if constexpr (!AS && BS) QHL_MMA_I8("u8", "s8");
+  else if constexpr (!AS && !BS) QHL_MMA_I8("u8", "u8");
+  else if constexpr (AS && BS) QHL_MMA_I8("s8", "s8");
+  else QHL_MMA_I8("s8", "u8");
+#undef QHL_MMA_I8
+}
+
+// Tokens per thread in the C fragment (columns 2c, 2c + 1 of every n-tile).
+template <int NT>
+struct MmaShape {
+  static constexpr int kNTiles = (NT + 7) / 8;
+  static constexpr int kTok = 2 * kNTiles;
+};
+
+// Row of accumulator m (m-tile m / 2, half m % 2) for lane group g.
+QHL_DEV int mma_row(int m, int g) { return 16 * (m >> 1) + 8 * (m & 1) + g; }
+
+// One block (warp `warp`) of one item for all NT tokens; acc[m][j]: row
+// mma_row(m, g), token 8 * (j / 2) + 2c + (j % 2).
+template <int QT, int NT>
+QHL_DEV void compute_item_mma(const uint8_t* st, const uint8_t* xs, int warp, int lane,
+                              float (&acc)[8][MmaShape<NT>::kTok]) {
+  const int g = lane >> 2, c = lane & 3;
+  // A fragments of the 4 m-tiles: rows 16mt + g and 16mt + g + 8
+  uint32_t a[4][4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = 16 * mt + 8 * h + g;
+      if constexpr (QT == kQ4_0) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(st + ((warp * 2 + (r >> 5)) * 32 + (r & 31)) * 16 + 4 * c);
+        a[mt][h] = w & 0x0F0F0F0Fu;                // elements 4c .. 4c + 3
+        a[mt][2 + h] = (w >> 4) & 0x0F0F0F0Fu;     // elements 16 + 4c .. 16 + 4c + 3
+      } else {
+        const uint8_t* base = st + (warp * 4) * 32 * 16;
+        a[mt][h] = *reinterpret_cast<const uint32_t*>(base + ((0 * 2 + (r >> 5)) * 32 + (r & 31)) * 16 + 4 * c);
+        a[mt][2 + h] = *reinterpret_cast<const uint32_t*>(base + ((1 * 2 + (r >> 5)) * 32 + (r & 31)) * 16 + 4 * c);
+      }
+    }
+  }
+  // row scales: word (g + 8q) holds rows g + 8q (low half) and g + 8q + 32 (high half)
+  float dsc[8];
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int r = mma_row(m, g);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(st + QLayout<QT>::kQuantBytes + (warp * 32 + (r & 31)) * 4);
+    dsc[m] = __half2float(__ushort_as_half(static_cast<unsigned short>((r >> 5) ? (w >> 16) : (w & 0xFFFFu))));
+  }
+#pragma unroll
+  for (int nt = 0; nt < MmaShape<NT>::kNTiles; ++nt) {
+    // B fragments: column g = token 8nt + g, k = 4c .. 4c + 3 and 16 + 4c ..
+    const int tb = 8 * nt + g;
+    uint32_t b[3][2];
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+      if (tb < NT) {
+        const uint8_t* xp = xs + tb * kQChunkBytes + p * 256 + warp * 32;
+        b[p][0] = *reinterpret_cast<const uint32_t*>(xp + 4 * c);
+        b[p][1] = *reinterpret_cast<const uint32_t*>(xp + 16 + 4 * c);
+      } else {
+        b[p][0] = 0u;
+        b[p][1] = 0u;
+      }
+    }
+    // block scales of this thread's two C-fragment tokens
+    float s[2];
+    int shi[2], sml[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int t = 8 * nt + 2 * c + e;
+      const uint8_t* xt = xs + (t < NT ? t : 0) * kQChunkBytes;
+      s[e] = reinterpret_cast<const float*>(xt + 768)[warp];
+      shi[e] = reinterpret_cast<const int*>(xt + 800)[warp];
+      sml[e] = reinterpret_cast<const int*>(xt + 832)[warp];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      int dh[4], dm[4], dl[4];
+      mma_i8<QT == kQ8_0, true>(dh, a[mt], b[0][0], b[0][1]);    // hi plane: signed
+      mma_i8<QT == kQ8_0, false>(dm, a[mt], b[1][0], b[1][1]);   // mid plane: unsigned
+      mma_i8<QT == kQ8_0, false>(dl, a[mt], b[2][0], b[2][1]);   // lo plane: unsigned
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 8 * nt + 2 * c + e;
+          if (t < NT) {
+            const int m = 2 * mt + h, j = 2 * nt + e, q = 2 * h + e;
+            if constexpr (QT == kQ4_0)
+              acc[m][j] = block_update(dsc[m], s[e], dh[q] - 8 * shi[e], dm[q] * 256 + dl[q] - 8 * sml[e], acc[m][j]);
+            else
+              acc[m][j] = block_update(dsc[m], s[e], dh[q], dm[q] * 256 + dl[q], acc[m][j]);
+          }
+        }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Warp roles of a GEMV CTA: warps 0..7 consume items, warp 8 produces (bulk
 // copies into the ring), warp 9 finishes tiles.  The consumers hand each
 // finished tile's per-warp sums to the epilogue warp through a small ring of
@@ -318,20 +435,40 @@ QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t*
   const int i0 = sk.begin(cta), n_local = sk.begin(cta + 1) - i0;
   if (n_local == 0) return;
 
-  float r0[NT], r1[NT];
+  constexpr bool kMma = NT >= kMmaTok;
+  constexpr int kAccA = kMma ? 1 : NT;                        // dp4a: rows lane, lane + 32
+  constexpr int kAccT = kMma ? MmaShape<NT>::kTok : 1;        // mma: C-fragment rows and tokens
+  float r0[kAccA], r1[kAccA];
+  float acc[kMma ? 8 : 1][kAccT];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) { r0[t] = 0.f; r1[t] = 0.f; }
+  for (int t = 0; t < kAccA; ++t) { r0[t] = 0.f; r1[t] = 0.f; }
+#pragma unroll
+  for (int m = 0; m < (kMma ? 8 : 1); ++m)
+#pragma unroll
+    for (int j = 0; j < kAccT; ++j) acc[m][j] = 0.f;
   auto handoff = [&]() {
     const int buf = (int)(tc % RB);
     const uint32_t use = tc / RB;
     if (use > 0 && !timed_out && !mbar_wait(smem_u32(&ts.free_[buf]), (use - 1) & 1u, a.err)) timed_out = true;
     float* red = ts.red + buf * TileRing<NT>::kBufFloats;
+    if constexpr (kMma) {
+      const int g = lane >> 2, c = lane & 3;
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      red[(warp * NT + t) * 64 + lane] = r0[t];
-      red[(warp * NT + t) * 64 + 32 + lane] = r1[t];
-      r0[t] = 0.f;
-      r1[t] = 0.f;
+      for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int j = 0; j < kAccT; ++j) {
+          const int t = 8 * (j >> 1) + 2 * c + (j & 1);
+          if (t < NT) red[(warp * NT + t) * 64 + mma_row(m, g)] = acc[m][j];
+          acc[m][j] = 0.f;
+        }
+    } else {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        red[(warp * NT + t) * 64 + lane] = r0[t];
+        red[(warp * NT + t) * 64 + 32 + lane] = r1[t];
+        r0[t] = 0.f;
+        r1[t] = 0.f;
+      }
     }
     mbar_arrive(smem_u32(&ts.full[buf]));
     ++tc;
@@ -346,10 +483,14 @@ QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t*
     // after one timed-out wait the rest of the call runs without waiting (the
     // error is recorded; results are garbage, but the kernel ends promptly)
     if (!timed_out && !mbar_wait(smem_u32(&bars[slot]), phase, a.err)) timed_out = true;
-    ItemRegs<QT> regs;
     const uint8_t* st = stages + slot * SB;
-    load_item<QT>(st, warp, lane, regs);
-    compute_item<QT, NT>(regs, st + IB, warp, r0, r1);
+    if constexpr (kMma) {
+      compute_item_mma<QT, NT>(st, st + IB, warp, lane, acc);
+    } else {
+      ItemRegs<QT> regs;
+      load_item<QT>(st, warp, lane, regs);
+      compute_item<QT, NT>(regs, st + IB, warp, r0, r1);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&bars[S + slot]));   // stage free for the producer
     ++chunk;

@@ -61,7 +61,7 @@ def test_single_q4_0_gemv_1024(q):
 
 @pytest.mark.parametrize("qtype", [Q4_0, Q8_0])
 @pytest.mark.parametrize("rows,cols", [(1, 256), (63, 512), (65, 256), (1000, 1280), (77, 5120)])
-@pytest.mark.parametrize("n", [1, 3, 16])
+@pytest.mark.parametrize("n", [1, 3, 4, 16])
 def test_gemv_ragged_shapes(q, qtype, rows, cols, n):
     W, x = synth.gemv_problem(5 + rows + cols, rows, cols, n, qtype)
     P = packed_on_gpu(q, qtype, W)
@@ -75,7 +75,9 @@ def test_gemv_batched_is_bit_identical_to_single_tokens(q, qtype):
     rows, cols = 1500, 2304
     W, x = synth.gemv_problem(21, rows, cols, 16, qtype)
     P = packed_on_gpu(q, qtype, W)
-    for n in (16, 7, 2):
+    # n >= 4 runs the integer tensor-core path, n < 4 the dp4a path: both form
+    # the same exact block sums, so every n equals the single-token results
+    for n in (16, 9, 8, 7, 5, 4, 3, 2):
         yb = gemv_gpu(q, qtype, P, rows, cols, x[:n])
         for t in range(n):
             y1 = gemv_gpu(q, qtype, P, rows, cols, x[t:t + 1])
