@@ -24,6 +24,9 @@ namespace qhl {
 constexpr int kAttDim = 256;
 constexpr int kRopeDims = 64;
 constexpr int kAttChunk = 64;
+// Tokens one attention unit serves: a 16-token pass splits its tokens into
+// groups of 4, so its (chunk, KV head, group) units spread over 4x the CTAs.
+constexpr int kAttGroup = 4;
 
 struct AttnArgs {
   const float* y;          // [NT][y_stride] in-projection output: q | gate | k | v
@@ -55,7 +58,7 @@ __host__ __device__ constexpr int attn_smem_bytes(int nt, int rep) {
 }
 template <int NT>
 constexpr int attn_smem_bytes(int rep) {
-  return attn_smem_bytes(NT, rep);
+  return attn_smem_bytes(NT < kAttGroup ? NT : kAttGroup, rep);
 }
 
 // RMSNorm over one 256-wide head vector held as 8 values per lane (dims 8l..8l+7)
@@ -98,29 +101,31 @@ QHL_DEV void half8(uint4 w, float (&f)[8]) {
   }
 }
 
-// One attention unit: KV head g, context chunk c (rows 64c .. 64c+63), all NT
-// tokens and the group's query heads.  Writes per (token, head, chunk) the
-// max score, the sum of exp and the exp-weighted V sum.  The pass's own rows
-// are written first; then the chunk's K and V rows are loaded into registers
-// through L2.  All 256 threads of the CTA take part; `pos` is the
-// position of token 0.
+// One attention unit: KV head g, context chunk c (rows 64c .. 64c+63), tokens
+// t0 .. t0 + min(kAttGroup, NT - t0) - 1 and the group's query heads.  Writes
+// per (token, head, chunk) the max score, the sum of exp and the exp-weighted
+// V sum.  The unit's tokens' own rows in the chunk are written first; then the
+// chunk's K and V rows are loaded into registers through L2.  All 256 threads
+// of the CTA take part; `pos` is the position of token 0.  A token's results
+// depend only on the token and the chunk, whatever its group.
 template <int NT>
-QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) {
+QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t* smem) {
   const int rep = a.Hq / a.Hkv;
-  const int njobs = NT * rep;
+  const int ntk = min(kAttGroup, NT - t0);
+  const int njobs = ntk * rep;
   float* qs = reinterpret_cast<float*>(smem);                 // [njobs][256]
   float* sc = qs + njobs * kAttDim;                            // [njobs][64]
   float* vec_all = sc + njobs * kAttChunk;                     // [8][256]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int k0 = c * kAttChunk;
-  const int ctx_end = pos + NT;
+  const int ctx_end = pos + t0 + ntk;                          // rows the unit's tokens see
   const int nkeys = min(kAttChunk, ctx_end - k0);             // > 0 by the caller
   float* vec = vec_all + warp * kAttDim;
   const int q_off = 0, k_off = 2 * a.Hq * kAttDim, v_off = k_off + a.Hkv * kAttDim;
   const size_t head_base = (size_t)g * a.max_ctx;
 
   // this pass's own rows that fall in the chunk: QK-norm + RoPE k, round k and v to f16, store
-  const int p_lo = max(k0, pos), p_hi = min(k0 + kAttChunk, ctx_end);
+  const int p_lo = max(k0, pos + t0), p_hi = min(k0 + kAttChunk, ctx_end);
   for (int p = p_lo + warp; p < p_hi; p += 8) {
     const int t = p - pos;
     const float* yt = a.y + (size_t)t * a.y_stride;
@@ -143,7 +148,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
   }
   // queries of every token that sees this chunk
   for (int job = warp; job < njobs; job += 8) {
-    const int t = job / rep, j = job - t * rep;
+    const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
     if (pos + t < k0) continue;
     const float* yt = a.y + (size_t)t * a.y_stride;
     float x[8];
@@ -218,7 +223,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
 
   // chunk softmax statistics, one warp per query
   for (int job = warp; job < njobs; job += 8) {
-    const int t = job / rep, j = job - t * rep;
+    const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
     const int nk = min(kAttChunk, pos + t + 1 - k0);
     if (nk <= 0) continue;
     const bool v0 = lane < nk, v1 = lane + 32 < nk;
@@ -250,7 +255,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
     for (int jj = 0; jj < JB; ++jj) {
       o0[jj] = 0.f;
       o1[jj] = 0.f;
-      nk[jj] = j0 + jj < njobs ? min(kAttChunk, pos + (j0 + jj) / rep + 1 - k0) : 0;
+      nk[jj] = j0 + jj < njobs ? min(kAttChunk, pos + t0 + (j0 + jj) / rep + 1 - k0) : 0;
     }
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
@@ -277,7 +282,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, uint8_t* smem) 
       for (int jj = 0; jj < JB; ++jj) {
         const int job = j0 + jj;
         if (job < njobs && nk[jj] > 0) {
-          const int t = job / rep, j = job - t * rep;
+          const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
           const float2 h1 = reinterpret_cast<const float2*>(part + jj * kAttDim)[pair];
           float2* dst = reinterpret_cast<float2*>(a.po + (((size_t)t * a.Hq + g * rep + j) * a.nchunk + c) * kAttDim);
           dst[pair] = make_float2(__fadd_rn(o0[jj], h1.x), __fadd_rn(o1[jj], h1.y));
@@ -293,9 +298,10 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   if (threadIdx.x == 0) pdl_launch();
   const int pos = *a.kv_len;
-  if ((int)blockIdx.x * kAttChunk >= pos + NT) return;
+  const int t0 = blockIdx.z * kAttGroup, ntk = min(kAttGroup, NT - t0);
+  if ((int)blockIdx.x * kAttChunk >= pos + t0 + ntk) return;   // no token of the group sees the chunk
   pdl_wait();
-  attn_unit<NT>(a, blockIdx.x, blockIdx.y, pos, smem);
+  attn_unit<NT>(a, blockIdx.x, blockIdx.y, pos, t0, smem);
 }
 
 // Combine the chunk partials of one (token, query head) and apply the sigmoid

@@ -65,26 +65,53 @@ QHL_DEV void dn_load(const DnArgs& a, int unit, float4 (&S)[4]) {
     S[r] = __ldg(reinterpret_cast<const float4*>(s_in + ((size_t)h * kDnDim + row0 + r) * kDnDim) + lane);
 }
 
+// Shared memory of one unit (floats): outputs ob [NT][32], then the unit's
+// inputs staged once for all tokens: q, k [NT][128] each, v [NT][32], b, a [NT].
+constexpr int dn_smem_floats(int nt) { return nt * (32 + 2 * kDnDim + 32 + 2); }
+
 template <int NT>
-QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float (*ob)[32]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = unit >> 2;                       // 4 units of 32 rows per head
   const int row0 = (unit & 3) * 32 + warp * 4;
   const int g = h / (a.Hv / a.Hk);
   const int cur = a.cur ? *a.cur : 0;
+  float (*ob)[32] = reinterpret_cast<float (*)[32]>(sm);
+  float* sq = sm + NT * 32;                      // [NT][128]
+  float* sk = sq + NT * kDnDim;                  // [NT][128]
+  float* sv = sk + NT * kDnDim;                  // [NT][32]: value rows (unit & 3) * 32 ..
+  float* sb = sv + NT * 32;                      // [NT]
+  float* sa = sb + NT;                           // [NT]
 
   const int off_k = a.Hk * kDnDim;
   const int off_v = 2 * a.Hk * kDnDim;
   const int off_b = off_v + a.Hv * kDnDim;
   const int off_a = off_b + a.Hv;
-  for (int t = 0; t < NT; ++t) {
+  // every token's inputs in one round of loads (through L2: written by the
+  // in-projection, possibly earlier in the same kernel)
+  for (int i = tid; i < NT * 64; i += 256) {
+    const int t = i >> 6, q4 = i & 63;
     const float* yt = a.y + (size_t)t * a.y_stride;
-    float4 q = __ldcg(reinterpret_cast<const float4*>(yt + g * kDnDim) + lane);
-    float4 k = __ldcg(reinterpret_cast<const float4*>(yt + off_k + g * kDnDim) + lane);
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(yt + (q4 < 32 ? 0 : off_k) + g * kDnDim) + (q4 & 31));
+    reinterpret_cast<float4*>(q4 < 32 ? sq + t * kDnDim : sk + t * kDnDim)[q4 & 31] = v;
+  }
+  for (int i = tid; i < NT * 32; i += 256) {
+    const int t = i >> 5, r = i & 31;
+    sv[i] = __ldcg(a.y + (size_t)t * a.y_stride + off_v + h * kDnDim + (unit & 3) * 32 + r);
+  }
+  if (tid < NT) {
+    sb[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_b + h);
+    sa[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_a + h);
+  }
+  named_sync(1, 256);
+
+  for (int t = 0; t < NT; ++t) {
+    float4 q = reinterpret_cast<const float4*>(sq + t * kDnDim)[lane];
+    float4 k = reinterpret_cast<const float4*>(sk + t * kDnDim)[lane];
     float v[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) v[r] = __ldcg(yt + off_v + h * kDnDim + row0 + r);
-    const float bb = __ldcg(yt + off_b + h), aa = __ldcg(yt + off_a + h);
+    for (int r = 0; r < 4; ++r) v[r] = sv[t * 32 + warp * 4 + r];
+    const float bb = sb[t], aa = sa[t];
     const float rq = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(q, q)), 1e-6f)));
     const float rk = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(k, k)), 1e-6f)));
     q = make_float4(__fmul_rn(q.x, rq), __fmul_rn(q.y, rq), __fmul_rn(q.z, rq), __fmul_rn(q.w, rq));
@@ -113,24 +140,24 @@ QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float (*ob)[32]) 
   if (a.qo)
     for (int t = warp; t < NT; t += 8)
       qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (unit & 3), lane);
-  named_sync(1, 256);   // ob reusable by the caller
+  named_sync(1, 256);   // sm reusable by the caller
 }
 
 template <int NT>
-QHL_DEV void dn_unit(const DnArgs& a, int unit, float (*ob)[32]) {
+QHL_DEV void dn_unit(const DnArgs& a, int unit, float* sm) {
   float4 S[4];
   dn_load<NT>(a, unit, S);
-  dn_run<NT>(a, unit, S, ob);
+  dn_run<NT>(a, unit, S, sm);
 }
 
 template <int NT>
 __global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
-  __shared__ float ob[NT][32];
+  __shared__ __align__(16) float sm[dn_smem_floats(NT)];
   if (threadIdx.x == 0) pdl_launch();
   float4 S[4];
   dn_load<NT>(a, blockIdx.x, S);   // overlaps the in-projection's last tiles
   pdl_wait();                      // q, k, v, b, a come from it
-  dn_run<NT>(a, blockIdx.x, S, ob);
+  dn_run<NT>(a, blockIdx.x, S, sm);
 }
 
 }  // namespace qhl

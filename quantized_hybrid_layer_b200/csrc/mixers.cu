@@ -92,8 +92,8 @@ cudaError_t launch_attn_partial(int nt, const AttnArgs& a, int nchunk, int hkv, 
   switch (nt) {
 #define C(N)                                                                                               \
   case N:                                                                                                  \
-    return launch_ex(attn_partial_kernel<N>, dim3(nchunk, hkv), dim3(256), (size_t)attn_smem_bytes<N>(rep), s, \
-                     pdl, a);
+    return launch_ex(attn_partial_kernel<N>, dim3(nchunk, hkv, (N + kAttGroup - 1) / kAttGroup), dim3(256),    \
+                     (size_t)attn_smem_bytes<N>(rep), s, pdl, a);
     QHL_NT_CASES(C)
 #undef C
     default: return cudaErrorInvalidValue;

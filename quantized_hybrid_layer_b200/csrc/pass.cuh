@@ -391,13 +391,18 @@ __global__ void __launch_bounds__(kGemvCtaThreads, 2) stage_pass_kernel(const Pa
     gemv_consume<QT, NT, S>(L.g[0], cta, stages, bars, ts, slot, parity, tc, timed_out);   // the epilogue warp arrives
     if (!L.attn) {
       QHL_PASS_WAIT();
-      for (int u = cta; u < p.dn_units; u += p.grid) dn_unit<NT>(L.dn, u, reinterpret_cast<float(*)[32]>(mix));
+      for (int u = cta; u < p.dn_units; u += p.grid) dn_unit<NT>(L.dn, u, reinterpret_cast<float*>(mix));
       grid_arrive(p, ph - 1);
     } else {
       QHL_PASS_WAIT();
       const int pos = *p.kv_len;
-      const int units = (pos + NT + kAttChunk - 1) / kAttChunk * p.Hkv;
-      for (int u = cta; u < units; u += p.grid) attn_unit<NT>(L.at, u / p.Hkv, u % p.Hkv, pos, mix);
+      constexpr int kGroups = (NT + kAttGroup - 1) / kAttGroup;
+      const int units = (pos + NT + kAttChunk - 1) / kAttChunk * p.Hkv * kGroups;
+      for (int u = cta; u < units; u += p.grid) {
+        const int grp = u % kGroups, rest = u / kGroups, t0 = grp * kAttGroup;
+        const int c = rest / p.Hkv, g = rest % p.Hkv;
+        if (c * kAttChunk < pos + t0 + min(kAttGroup, NT - t0)) attn_unit<NT>(L.at, c, g, pos, t0, mix);
+      }
       grid_arrive(p, ph - 1);
       QHL_PASS_WAIT();
       for (int u = cta; u < NT * p.Hq; u += p.grid)

@@ -326,7 +326,7 @@ bool pass_eligible(const stage* st, int n) {
   }
   const int rep = st->cfg.att_q_heads / st->cfg.att_kv_heads;
   const int mix = pass_mix_bytes(qt, n);
-  const int need = std::max({n * 64 * 4, n * 32 * 4, st->nchunk * 3 * 4, st->nchunk ? attn_smem_bytes(n, rep) : 0});
+  const int need = std::max({n * 64 * 4, dn_smem_floats(n) * 4, st->nchunk * 3 * 4, st->nchunk ? attn_smem_bytes(std::min(n, kAttGroup), rep) : 0});
   return need <= mix;
 }
 
