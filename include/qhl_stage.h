@@ -167,14 +167,16 @@ stage_status stage_set_kv_len(stage_t* st, int kv_len);
 stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst);
 
 /* How a pass runs on the device.
- *   STAGE_PASS_PERSISTENT (default): one cooperative kernel runs the whole pass
+ *   STAGE_PASS_KERNELS (default): one kernel per step, all recorded in a CUDA
+ *     graph, each a programmatic dependent of the one before.
+ *   STAGE_PASS_PERSISTENT: one cooperative kernel runs the whole pass
  *     (stage input, then every layer's projections and mixer), its phases
  *     separated by grid-wide barriers, its CTAs streaming the next projection's
  *     weights across phase boundaries.  Used for n_tok 1..4 when two CTAs per
  *     SM are resident and the mixers' scratch fits (attention context of at
  *     most ~1700 chunks of 64 rows at n_tok 1); other passes fall back to
- *     kernels.
- *   STAGE_PASS_KERNELS: one kernel per step, all recorded in a CUDA graph.
+ *     kernels.  Slower than the kernels on B200 (per-step barriers and
+ *     fix-up tails on the critical path); kept as an option.
  * Both run the same units with the same split and reduction order, so they
  * give bit-identical results.  Refused while a pass is pending; waits for the
  * stage's stream and drops the recorded graphs. */

@@ -186,8 +186,8 @@ class Stage:
         return lib().stage_pending(self._h)
 
     def set_pass_mode(self, mode: int):
-        """PASS_PERSISTENT (one cooperative kernel per pass where eligible) or
-        PASS_KERNELS (one kernel per step)."""
+        """PASS_KERNELS (one kernel per step, the default) or PASS_PERSISTENT
+        (one cooperative kernel per pass where eligible)."""
         self._check(lib().stage_set_pass_mode(self._h, mode))
 
     def pass_persistent(self, n_tok: int) -> bool:

@@ -97,7 +97,7 @@ struct stage {
   unsigned* bar = nullptr;
   int n_phases = 0;
   unsigned long long* trace = nullptr;   // [grid][n_phases][2], when tracing is on
-  int pass_mode = STAGE_PASS_PERSISTENT;
+  int pass_mode = STAGE_PASS_KERNELS;
   size_t weight_bytes = 0;
   std::string last_error;
 };

@@ -244,6 +244,7 @@ def test_persistent_pass_equals_kernel_chain(q, qtype, ns):
     seed = 7
     st, _, _ = make_pair(FULL, qtype, seed, 0, 4, MAX_CTX, CTX, with_oracle=False)
     try:
+        assert not st.pass_persistent(1)                      # the chain of kernels by default
         assert not st.pass_persistent(16)
         S0 = _states(st, 0, 4)
         kv0 = {l: st.get_kv(l) for l in attn_layers(0, 4)}
@@ -289,6 +290,7 @@ def test_persistent_pass_trace_shows_the_grid_barriers(q):
     try:
         with pytest.raises(q.StageError):
             st.get_trace()                                   # off by default
+        st.set_pass_mode(q.PASS_PERSISTENT)
         st.set_trace(True)
         h = synth.hidden(FULL, 8, 0, 1)
         run(st, h, CTX)
