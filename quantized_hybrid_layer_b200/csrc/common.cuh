@@ -118,6 +118,11 @@ QHL_DEV void bulk_g2s_plain(uint32_t dst, const void* src, uint32_t bytes, uint3
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
+// Fetch `bytes` (multiple of 16, 16-byte aligned) from global memory into L2,
+// without a destination in shared memory.
+QHL_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (bulk copy) writes to the same memory.
 QHL_DEV void fence_proxy_async_smem() {

@@ -61,6 +61,10 @@ struct GemvArgs {
   int* counters;           // stream-K tile counters, zero between launches
   int workers;             // CTAs that own items (<= items, == grid size)
   unsigned* err;           // device error word
+  // The pass's next projection (null if none): this kernel's producers warm L2
+  // with the first items the next kernel's CTA of the same index will stream.
+  const uint8_t* next_W;
+  int next_items, next_workers;
 };
 
 constexpr int kConsumerWarps = 8;
@@ -686,6 +690,14 @@ __global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) 
         mbar_arrive_expect_tx(full, SB);
         bulk_g2s(smem_u32(stages + s * SB), a.W + (size_t)(i0 + k) * IB, IB, full, pol);
         issue_x(k, s);
+      }
+      // every own item is on its way: warm L2 with the next projection's first
+      // items of this CTA index while the consumers finish (the next kernel's
+      // copies of them then hit L2)
+      if (a.next_W && cta < a.next_workers) {
+        const StreamK skn(a.next_items, a.next_workers);
+        const int j0 = skn.begin(cta), nj = min(S, skn.begin(cta + 1) - j0);
+        for (int k = 0; k < nj; ++k) bulk_prefetch_l2(a.next_W + (size_t)(j0 + k) * IB, IB);
       }
     }
     return;

@@ -298,7 +298,17 @@ cudaError_t record_kernels(stage* st, int n, cudaStream_t s) {
                                      st->ss_stride, s);
   if (e != cudaSuccess) return e;
   for (size_t i = 0; i < st->layers.size(); ++i) {
-    const PassLayer P = layer_args(st, i);
+    PassLayer P = layer_args(st, i);
+    // each projection warms L2 with the next one's first items
+    auto chain = [](GemvArgs& a, const GemvArgs& next) {
+      a.next_W = next.W;
+      a.next_items = next.tiles * next.chunks;
+      a.next_workers = next.workers;
+    };
+    chain(P.g[0], P.g[1]);
+    chain(P.g[1], P.g[2]);
+    chain(P.g[2], P.g[3]);
+    if (i + 1 < st->layers.size()) chain(P.g[3], layer_args(st, i + 1).g[0]);
     if ((e = launch_gemv(qt, n, EPI_STORE, P.g[0], P.g[0].workers, s, kUsePdl)) != cudaSuccess) return e;
     if (!P.attn) {
       if ((e = launch_dn_step(n, P.dn, c.dn_v_heads * (kDnDim / 32), s, kUsePdl)) != cudaSuccess) return e;
