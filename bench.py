@@ -147,10 +147,16 @@ def measured_peaks() -> dict:
 
 
 def kernel_sources_sha() -> str:
+    """Hash of the GEMV's sources with comments and blank lines dropped (what
+    the compiler sees), to tell whether committed ncu counters still apply."""
+    import re
     h = hashlib.sha256()
     for f in ("qgemv.cuh", "qpack.cuh", "qact.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "quantized_hybrid_layer_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "quantized_hybrid_layer_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = re.sub(r"//.*", "", line).rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

@@ -20,8 +20,12 @@
 //    tile rows l and l + 32, so x is read as warp-uniform broadcasts and no
 //    cross-lane reduction is needed.  x arrives in block fixed-point form
 //    (qact.cuh): each block's sum_j q_j X_j is formed exactly in int32 with
-//    byte dot products (dp4a) against the 4-bit (or 8-bit) quants, and one FMA
-//    per block adds d * s * sum to the row's f32 accumulator.
+//    byte dot products (dp4a) against the 4-bit (or 8-bit) quants -- from 4
+//    tokens up by integer tensor-core mma instead, with the same exact sums --
+//    and one FMA per block adds d * s * sum to the row's f32 accumulator.
+//  * A tenth warp finishes tiles (sums the consumer warps' partials, stream-K
+//    fix-up, epilogue) while the consumers stream on; once its own items are
+//    issued the producer warms L2 with the pass's next projection.
 //  * Reduction order is fixed and independent of NT: per row, exact integer
 //    block sums, blocks in item order inside a warp, then warps 0..7, then CTAs
 //    in grid order (stream-K partials, combined by whichever CTA finishes a tile
