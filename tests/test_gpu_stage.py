@@ -307,3 +307,41 @@ def test_persistent_pass_trace_shows_the_grid_barriers(q):
         st.rollback()
     finally:
         st.free()
+
+
+def test_zero_weight_stage_is_the_identity(q):
+    """All quants at the Q4_0 zero point (nibble 8): every projection is 0, so
+    each layer adds exact zeros and the stage returns its input bit for bit
+    (a DeltaNet and an attention layer, a 3-token pass)."""
+    seed = 9
+    t = synth.stage_tensors(FULL, Q4_0, seed, 2, 4)
+    for name, v in t.items():
+        if v.dtype == np.uint8:                        # GGUF blocks: 2-byte scale + 16 bytes of nibbles
+            b = v.reshape(v.shape[0], -1, 18).copy()
+            b[:, :, 2:] = 0x88
+            t[name] = b.reshape(v.shape)
+    st, _, _ = make_pair(FULL, Q4_0, seed, 2, 4, MAX_CTX, CTX, with_oracle=False, tensors=t)
+    try:
+        h = synth.hidden(FULL, seed, 0, 3)
+        out = run(st, h, CTX)
+        assert np.array_equal(out, h.astype(np.float32))
+        st.commit(3)
+    finally:
+        st.free()
+
+
+@pytest.mark.parametrize("n", [1, 4])
+def test_long_context_attention_layer_matches_oracle(q, n):
+    """One attention layer at context 65536 (1025 chunks of 64 rows to split
+    and combine), against the oracle."""
+    seed = 10
+    ctx = 65536
+    st, orc, _ = make_pair(FULL, Q4_0, seed, 3, 4, ctx + 64, ctx)
+    try:
+        h = synth.hidden(FULL, seed, n, n)
+        got = run(st, h, ctx)
+        ref = orc.forward(h, ctx)
+        assert max(rel_err_rows(got, ref)) <= TOL
+        st.rollback()
+    finally:
+        st.free()
