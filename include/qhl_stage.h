@@ -4,18 +4,21 @@
  * A "stage" is a contiguous range of decoder layers of a hybrid Gated-DeltaNet +
  * attention model that a peer runs on the hidden state it is handed:
  *   - Unstable Legion: the peer-to-peer ChatGPT, "Splitting the workload": the
- *     model is cut into contiguous layer stages; each stage runs its own range
- *     of layers and keeps its own attention cache.  "The runtime": run an
- *     arbitrary range of layers with activations passed in and out.
+ *     model is cut into contiguous layer stages, and every stage holds the
+ *     attention cache of its layers only.  "The runtime": a peer is handed an
+ *     activation, pushes it through whatever layer range it was given, and
+ *     hands the result on.
  *   - Peer-to-peer LLM inference in browser tabs, Qwen 3.8 27B (SwarmLLM
  *     README): peers hold layers 0-21 / 22-42 / 43-63 of a 64-layer model with a
- *     5,120-float hidden state, GGUF Q4_0 weights ("4-bit blocks with f16
- *     scales"), prefill in 16-token batches, multi-token-prediction drafts
- *     verified "in a single batched pass with exact rollback of the recurrent
- *     state", and a speculative path equal to plain decoding.
- *   - ChatTorrent README, "What it can run": Gated DeltaNet layers mixed with
- *     full-attention layers that have partial RoPE, QK-norm and an output gate;
- *     RMSNorm and SwiGLU blocks; weights f32, f16 or q8.
+ *     5,120-float hidden state, GGUF Q4_0 weights (4-bit values, one f16
+ *     scale per block), prefill in 16-token batches, multi-token-prediction
+ *     drafts checked together in one batched pass whose rejected tail is
+ *     undone exactly in the recurrent state, and a speculative path that
+ *     produces what plain decoding produces.
+ *   - ChatTorrent README, "What it can run": the hybrid interleaves Gated
+ *     DeltaNet layers and full-attention layers; the latter rotate only part
+ *     of each head (partial RoPE), normalise q and k per head and gate their
+ *     output; blocks use RMSNorm and SwiGLU; weights may be f32, f16 or q8.
  *
  * Each layer: h += mixer(RMSNorm1(h)); h += W_down(silu(W_gate x) * (W_up x)),
  * x = RMSNorm2(h).  Layer i is full attention iff i % attn_every == attn_every-1,

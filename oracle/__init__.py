@@ -13,21 +13,23 @@ is stated at the function.
 
 Sources (page title, part of the page):
 
-* P1 "Unstable Legion: the peer-to-peer ChatGPT", "Splitting the workload" and
+* "Unstable Legion: the peer-to-peer ChatGPT", "Splitting the workload" and
   "The runtime": a stage runs a contiguous range of layers, activation in,
-  activation out; each stage keeps its own attention cache.
-* P2 "ChatTorrent" README, "What it can run": the hybrid mixes Gated DeltaNet
-  linear-attention layers with full-attention layers that have partial RoPE,
-  QK-norm and an attention output gate; blocks use RMSNorm and SwiGLU.
-* P3 "Peer-to-peer LLM inference in browser tabs, Qwen 3.8 27B" (SwarmLLM
+  activation out, and holds the attention cache of those layers only.
+* "ChatTorrent" README, "What it can run": the hybrid interleaves Gated
+  DeltaNet (linear attention) layers and full-attention layers; the latter
+  rotate part of each head (partial RoPE), normalise q and k per head and gate
+  their output; blocks use RMSNorm and SwiGLU.
+* "Peer-to-peer LLM inference in browser tabs, Qwen 3.8 27B" (SwarmLLM
   README): 27B hybrid Gated-DeltaNet + attention, GGUF Q4_0 with f16 block
-  scales, 5,120-wide hidden state, batched verify "with exact rollback of the
-  recurrent state", speculative path equal to plain decoding.
-* The update is the gated delta rule of the Gated DeltaNet paper, which P3
-  names among its prior work: ``S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T)
+  scales, 5,120-wide hidden state, drafts verified in one batched pass whose
+  rejected tail is undone exactly in the recurrent state, so the speculative
+  path gives what plain decoding gives.
+* The update is the gated delta rule of the Gated DeltaNet paper, which the
+  SwarmLLM README names among its prior work: ``S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T)
   + beta_t v_t k_t^T``, read out as ``o_t = S_t q_t``.
-* Shapes: hidden 5,120 (P3 diagram) and 64 layers (P3 peer split 0-21 / 22-42
-  / 43-63); FFN 17408, 16 key / 48 value heads of 128, 24 query / 4 KV heads
+* Shapes: hidden 5,120 (SwarmLLM README diagram) and 64 layers (its peer
+  split 0-21 / 22-42 / 43-63); FFN 17408, 16 key / 48 value heads of 128, 24 query / 4 KV heads
   of 256, RoPE on the first 64 dims with theta 1e7, eps 1e-6 and a 3:1
   DeltaNet:attention pattern are the defaults of ``synth.StageShape``.
 
@@ -131,7 +133,7 @@ def qgemv(qtype: int, blocks: np.ndarray, x: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 
 def rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
-    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * gamma (P2 "What it can run")."""
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * gamma (ChatTorrent README, "What it can run")."""
     x = np.asarray(x, dtype=np.float64)
     ms = np.mean(x * x, axis=-1, keepdims=True)
     return x / np.sqrt(ms + eps) * np.asarray(gamma, dtype=np.float64)
@@ -176,7 +178,7 @@ def rope(x: np.ndarray, pos: int, rope_dims: int, theta: float) -> np.ndarray:
 # ----------------------------------------------------------------------------
 
 def deltanet_token(S: np.ndarray, q_raw, k_raw, v, b, a, shape: StageShape):
-    """One gated-delta-rule step for every value head (Gated DeltaNet, P2 "What it can run").
+    """One gated-delta-rule step for every value head (Gated DeltaNet; ChatTorrent README, "What it can run").
 
     S is f64 [Hv, dv, dk].  Per value head h with key head g = h // (Hv/Hk):
     ``S <- alpha * S (I - beta k k^T) + beta v k^T`` and ``o = S q`` on the
@@ -224,7 +226,7 @@ def split_dn_in(y: np.ndarray, shape: StageShape):
 
 def attention_token(y: np.ndarray, pos: int, K: np.ndarray, V: np.ndarray,
                     gq: np.ndarray, gk: np.ndarray, shape: StageShape) -> np.ndarray:
-    """Full GQA attention for the token at absolute position ``pos`` (P2 "What it can run").
+    """Full GQA attention for the token at absolute position ``pos`` (ChatTorrent README, "What it can run").
 
     y is the token's in-projection output (rows q | gate | k | v).  The token's
     k, v are QK-normed (k) and RoPE'd (k), rounded to f16 and written to cache
@@ -265,8 +267,8 @@ class OracleStage:
     ``forward(h, pos)`` runs n tokens at positions pos .. pos+n-1 through every
     layer (layer by layer, tokens in order inside a layer) and leaves the pass
     pending; ``commit(j)`` keeps the first j tokens' effect on the DeltaNet
-    states and the KV length, ``rollback()`` keeps none (P3: verify "in a
-    single batched pass with exact rollback of the recurrent state").
+    states and the KV length, ``rollback()`` keeps none (SwarmLLM README:
+    a batched verify pass whose rejected drafts leave no trace in the state).
     """
 
     def __init__(self, shape: StageShape, qtype: int, tensors: dict, begin: int, end: int, max_ctx: int):

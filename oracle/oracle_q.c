@@ -7,17 +7,17 @@
  * or constant with the CUDA library.
  *
  * What it computes, and where the pages fix it:
- *  - Weights are GGUF Q4_0 blocks ("4-bit blocks with f16 scales", SwarmLLM
+ *  - Weights are GGUF Q4_0 blocks (4-bit values with an f16 scale, SwarmLLM
  *    README on "Peer-to-peer LLM inference in browser tabs, Qwen 3.8 27B",
  *    paragraph after the peer diagram; model table "GGUF Q4_0") or GGUF Q8_0
  *    blocks (same README, model table "GGUF Q8_0 / Q4_0"; ChatTorrent README,
- *    "What it can run": weights stored as f32, f16 or q8).
+ *    "What it can run": f32, f16 and q8 weights are supported).
  *  - Q4_0 block: binary16 scale d (little endian) then 16 bytes; element j
  *    (j < 16) is the low nibble of byte j, element j+16 its high nibble;
  *    weight = (nibble - 8) * d.  Q8_0 block: binary16 d then 32 signed bytes;
  *    weight = q * d.  Block b of a row covers input columns 32b .. 32b+31.
- *  - A projection is y = x W^T: "every token reads all of the weights once"
- *    (same README, paragraph after the peer diagram).
+ *  - A projection is y = x W^T, so one token streams the whole weight set a
+ *    single time (same README, paragraph after the peer diagram).
  *
  * Everything is done in double precision, in the plain order of the
  * definitions: each output is one sequential dot product over the input

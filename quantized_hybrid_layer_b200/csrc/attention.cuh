@@ -1,8 +1,7 @@
 // Split-K GQA decode attention with QK-norm, partial RoPE, f16 KV cache and a
-// sigmoid output gate (ChatTorrent README, "What it can run": full-attention
-// layers "that have partial RoPE, QK-norm and an attention output gate"; each
-// stage "keeps its own attention cache": Unstable Legion, "Splitting the
-// workload").
+// sigmoid output gate (ChatTorrent README, "What it can run", lists these three
+// features of the hybrid's full-attention layers; Unstable Legion, "Splitting
+// the workload": a stage holds the attention cache of its own layers only).
 //
 // Token t of a pass sits at absolute position pos + t and attends to cache rows
 // 0 .. pos + t.  The context is cut into fixed chunks of 64 rows at absolute

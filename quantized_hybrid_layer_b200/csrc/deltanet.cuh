@@ -13,8 +13,8 @@
 // holds columns 4l..4l+3) for all NT tokens (8 warps = 32 rows per CTA, so a
 // CTA owns whole 32-value output blocks), so the state is read from HBM once
 // and written once per token as the snapshot S_t used for exact rollback
-// (SwarmLLM README: batched verify "with exact rollback of the recurrent
-// state").  The state rows are loaded before griddepcontrol.wait, overlapping
+// (SwarmLLM README: drafts are verified in one batched pass and the rejected
+// tail is undone exactly in the recurrent state).  The state rows are loaded before griddepcontrol.wait, overlapping
 // the in-projection that produces q, k, v, b, a.  Reductions are xor
 // butterflies over fixed lane partials, so every token's arithmetic is the
 // same whatever NT is.

@@ -1,8 +1,9 @@
 // Fused dequant-GEMV / skinny GEMM over packed Q4_0 / Q8_0 weights.
 //
 // y[t][r] = sum_c x[t][c] * W[r][c] for n_tok = NT tokens (1..16), the
-// projection every layer of the stage streams: "every token reads all of the
-// weights once" (SwarmLLM README, paragraph after the peer diagram).  Decode is
+// projection every layer of the stage streams: one decoded token streams the
+// whole weight set a single time (SwarmLLM README, paragraph after the peer
+// diagram).  Decode is
 // memory-bound, so the kernel is built to keep HBM busy and the SM's integer
 // and FP pipes well below their limits:
 //

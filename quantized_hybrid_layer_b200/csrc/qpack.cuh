@@ -17,7 +17,7 @@
 //
 // A Q4_0 block keeps its GGUF meaning: element j (j < 16) is the low nibble of
 // byte j, element j + 16 the high nibble, weight = (nibble - 8) * d.  Q8_0:
-// weight = q * d.  (SwarmLLM README: "4-bit blocks with f16 scales"; model
+// weight = q * d.  (SwarmLLM README: 4-bit values with an f16 scale per block; model
 // table "GGUF Q4_0", "GGUF Q8_0 / Q4_0".)
 #pragma once
 

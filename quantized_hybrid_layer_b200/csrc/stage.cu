@@ -3,8 +3,8 @@
 // A stage owns, on one GPU: the packed weights of its layer range, a rollback
 // ring of DeltaNet state snapshots per DeltaNet layer, an f16 KV cache per
 // attention layer, activation buffers for up to 16 tokens, and one CUDA graph
-// per token count.  stage_forward launches that graph: "one command submit per
-// token" (SwarmLLM README, paragraph after the peer diagram).  Inside the graph
+// per token count.  stage_forward launches that graph, a single submission per
+// pass as on the pages (SwarmLLM README, paragraph after the peer diagram).  Inside the graph
 // every kernel after the first is launched with programmatic dependent launch,
 // so a projection's weights start streaming while the previous kernel drains.
 //
