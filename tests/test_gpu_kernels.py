@@ -12,7 +12,7 @@ import pytest
 import oracle
 import synth
 from synth import FULL, Q4_0, Q8_0
-from stage_helpers import TOL, rel_err_heads, rel_err_rows
+from stage_helpers import TOL, gemv_error_bound, rel_err_heads, rel_err_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +54,8 @@ def test_single_q4_0_gemv_1024(q):
     ref = oracle.qgemv(Q4_0, W, x)
     err = rel_err_rows(y, ref)
     assert max(err) <= TOL, err
-    # x enters as 16-bit block fixed point (step <= 2^-15 of the block max): the
+    assert np.all(np.abs(y - ref) <= gemv_error_bound(Q4_0, W, x))
+    # x enters as 24-bit block fixed point (step <= 2^-22 of the block max): the
     # error stays far inside the bound
     assert max(err) <= 2e-4
 
@@ -68,6 +69,7 @@ def test_gemv_ragged_shapes(q, qtype, rows, cols, n):
     y = gemv_gpu(q, qtype, P, rows, cols, x)
     ref = oracle.qgemv(qtype, W, x)
     assert max(rel_err_rows(y, ref)) <= TOL
+    assert np.all(np.abs(y - ref) <= gemv_error_bound(qtype, W, x))
 
 
 @pytest.mark.parametrize("qtype", [Q4_0, Q8_0])
@@ -96,6 +98,7 @@ def test_gemv_full_size_sampled_rows(q, rows, cols, n):
     idx = np.unique(np.concatenate([idx, [0, rows - 1]]))
     ref = oracle.qgemv(Q4_0, W[idx], x)             # the oracle computes just these rows
     assert max(rel_err_rows(y[:, idx], ref)) <= TOL
+    assert np.all(np.abs(y[:, idx] - ref) <= gemv_error_bound(Q4_0, W[idx], x))
 
 
 # ------------------------------------------------------------- dequant --
