@@ -122,6 +122,19 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
  * commit(1) each). */
 stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos);
 
+/* stage_forward with the hidden state in IEEE binary16, the form a peer sends
+ * on the wire (SwarmLLM README, paragraph under the benchmark table: one
+ * token's 5,120-value hidden state is 10 KB as f16; github-Nehanth-swarmllm
+ * summary, "How it works").  hidden_dev: caller-owned device binary16
+ * [n_tok, H], row-major, 2-byte aligned, read and overwritten in place.  The
+ * input is widened to f32 exactly, the pass is the one stage_forward runs, and
+ * the output is its f32 result rounded to nearest even (magnitudes beyond
+ * 65504 become +-inf, as IEEE rounding gives): for the same (f16) input
+ * values, out_f16 == round_f16(out_f32 of stage_forward), bit for bit.
+ * Same arguments, state rules and errors as stage_forward (STAGE_E_ARG also
+ * for a misaligned pointer, before any device work). */
+stage_status stage_forward_f16(stage_t* st, void* hidden_dev, int n_tok, int pos);
+
 /* Keep the first n_accepted tokens (0..n_tok) of the pending pass: each
  * DeltaNet state becomes the snapshot after token n_accepted (no copy: the
  * ring index moves) and the committed length becomes pos + n_accepted.  KV

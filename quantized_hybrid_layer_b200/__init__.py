@@ -30,7 +30,7 @@ STATUS = {
 
 #: every symbol include/qhl_stage.h declares
 EXPORTS = (
-    "stage_load", "stage_forward", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
+    "stage_load", "stage_forward", "stage_forward_f16", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
     "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_set_pass_mode", "stage_pass_persistent",
     "stage_set_trace", "stage_get_trace",
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "stage_load": (i, [ctypes.POINTER(StageConfig), ctypes.POINTER(StageTensor), i, i, i, vp,
                                ctypes.POINTER(vp)]),
             "stage_forward": (i, [vp, vp, i, i]),
+            "stage_forward_f16": (i, [vp, vp, i, i]),
             "stage_commit": (i, [vp, i]),
             "stage_rollback": (i, [vp]),
             "stage_reset": (i, [vp]),
@@ -154,6 +155,14 @@ class Stage:
         assert hidden.is_cuda and hidden.dtype.itemsize == 4 and hidden.is_contiguous()
         n = hidden.shape[0]
         self._check(lib().stage_forward(self._h, _ptr(hidden), n, pos))
+        return hidden
+
+    def forward_f16(self, hidden, pos: int):
+        """hidden: contiguous CUDA float16 tensor [n_tok, hidden] (the wire format),
+        updated in place with the pass's f32 result rounded to nearest even."""
+        assert hidden.is_cuda and hidden.dtype.itemsize == 2 and hidden.is_floating_point() and hidden.is_contiguous()
+        n = hidden.shape[0]
+        self._check(lib().stage_forward_f16(self._h, _ptr(hidden), n, pos))
         return hidden
 
     def forward_host(self, hidden_host, pos: int, dev_buf=None):
@@ -267,6 +276,10 @@ def stage_load(cfg: StageConfig, tensors: dict, layer_begin: int, layer_end: int
 
 def stage_forward(st: Stage, hidden, pos: int):
     return st.forward(hidden, pos)
+
+
+def stage_forward_f16(st: Stage, hidden, pos: int):
+    return st.forward_f16(hidden, pos)
 
 
 def stage_commit(st: Stage, n_accepted: int):

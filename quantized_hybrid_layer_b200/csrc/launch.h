@@ -46,6 +46,8 @@ cudaError_t launch_attn_combine(int nt, const AttnArgs& a, cudaStream_t s, bool 
 cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, uint8_t* qz, int qz_stride,
                                float* ss, int ss_stride, cudaStream_t s);
 cudaError_t launch_quantize_rows(const float* x, int n, int cols, uint8_t* qx, cudaStream_t s);
+cudaError_t launch_hidden_from_f16(const void* in, float* out, int n, cudaStream_t s);   // binary16 -> f32
+cudaError_t launch_hidden_to_f16(const float* in, void* out, int n, cudaStream_t s);     // f32 -> binary16 (RNE)
 
 cudaError_t launch_repack(int qt, const uint8_t* a, const uint8_t* b, int rows, int cols, uint8_t* out,
                           cudaStream_t s);

@@ -1,6 +1,8 @@
 // Mixer kernels' launch wrappers (DeltaNet step, attention), the stage input
 // kernel, weight repacking, dequantisation check, RoPE table and the tiny
 // control kernels used by commit / rollback.
+#include <algorithm>
+
 #include "launch.h"
 
 namespace qhl {
@@ -50,6 +52,30 @@ __global__ void quantize_rows_kernel(const float* x, int n, int cols, uint8_t* q
 cudaError_t launch_quantize_rows(const float* x, int n, int cols, uint8_t* qx, cudaStream_t s) {
   const long long warps = (long long)n * (cols / 32);
   quantize_rows_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(x, n, cols, qx);
+  return cudaGetLastError();
+}
+
+// Hidden state at the stage boundary in binary16 (the peers' wire format):
+// widened to f32 exactly on the way in, rounded to nearest even on the way out.
+__global__ void hidden_from_f16_kernel(const __half* in, float* out, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    out[i] = __half2float(in[i]);
+}
+
+__global__ void hidden_to_f16_kernel(const float* in, __half* out, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    out[i] = __float2half_rn(in[i]);
+}
+
+static unsigned elementwise_blocks(int n) { return (unsigned)std::min((n + 255) / 256, 148 * 8); }
+
+cudaError_t launch_hidden_from_f16(const void* in, float* out, int n, cudaStream_t s) {
+  hidden_from_f16_kernel<<<elementwise_blocks(n), 256, 0, s>>>(static_cast<const __half*>(in), out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hidden_to_f16(const float* in, void* out, int n, cudaStream_t s) {
+  hidden_to_f16_kernel<<<elementwise_blocks(n), 256, 0, s>>>(in, static_cast<__half*>(out), n);
   return cudaGetLastError();
 }
 

@@ -623,21 +623,38 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
   return STAGE_OK;
 }
 
-stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos) {
+// Checks shared by both forward entries; builds the n_tok graph on first use.
+static stage_status forward_begin(stage_t* st, const void* hidden_dev, int n_tok, int pos) {
   if (!st) return STAGE_E_ARG;
   if (!hidden_dev) return fail(st, STAGE_E_ARG, "hidden_dev is NULL");
   if (n_tok < 1 || n_tok > kMaxTok) return fail(st, STAGE_E_ARG, "n_tok must be in 1..16");
   if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending: commit or roll back first");
   if (pos != st->committed) return fail(st, STAGE_E_STATE, "pos must equal the committed length");
   if (pos + n_tok > st->cfg.max_ctx) return fail(st, STAGE_E_ARG, "pass would overflow max_ctx");
-  if (!st->exec[n_tok]) {
-    stage_status s = build_graph(st, n_tok);
-    if (s != STAGE_OK) return s;
-  }
+  if (!st->exec[n_tok]) return build_graph(st, n_tok);
+  return STAGE_OK;
+}
+
+stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos) {
+  stage_status s = forward_begin(st, hidden_dev, n_tok, pos);
+  if (s != STAGE_OK) return s;
   const size_t bytes = (size_t)n_tok * st->cfg.hidden * 4;
   CK(cudaMemcpyAsync(st->h, hidden_dev, bytes, cudaMemcpyDeviceToDevice, st->stream));
   CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
   CK(cudaMemcpyAsync(hidden_dev, st->h, bytes, cudaMemcpyDeviceToDevice, st->stream));
+  st->pending_n = n_tok;
+  st->pending_pos = pos;
+  return STAGE_OK;
+}
+
+stage_status stage_forward_f16(stage_t* st, void* hidden_dev, int n_tok, int pos) {
+  if (st && reinterpret_cast<uintptr_t>(hidden_dev) % 2) return fail(st, STAGE_E_ARG, "hidden_dev must be 2-byte aligned");
+  stage_status s = forward_begin(st, hidden_dev, n_tok, pos);
+  if (s != STAGE_OK) return s;
+  const int n = n_tok * st->cfg.hidden;
+  CK(launch_hidden_from_f16(hidden_dev, st->h, n, st->stream));
+  CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
+  CK(launch_hidden_to_f16(st->h, hidden_dev, n, st->stream));
   st->pending_n = n_tok;
   st->pending_pos = pos;
   return STAGE_OK;

@@ -75,6 +75,7 @@ def test_bad_arguments_are_rejected_before_any_device_work(qhl):
     assert lib.stage_load(ctypes.byref(bad), None, 0, 0, 1, None, ctypes.byref(out)) == -6
     assert out.value is None
     assert lib.stage_forward(None, None, 1, 0) == -1
+    assert lib.stage_forward_f16(None, None, 1, 0) == -1
     assert lib.stage_commit(None, 0) == -1
     assert lib.stage_rollback(None) == -1
     assert lib.stage_committed_len(None) == -1

@@ -345,3 +345,28 @@ def test_long_context_attention_layer_matches_oracle(q, n):
         st.rollback()
     finally:
         st.free()
+
+
+@pytest.mark.parametrize("n", [1, 5])
+def test_f16_boundary_equals_the_f32_pass_rounded(q, stage3, n):
+    """forward_f16 takes and returns the hidden state in binary16, the peers'
+    wire format (10 KB per token at hidden 5120): its output is, bit for bit,
+    the f32 pass on the same (f16-valued) input rounded to nearest even, and
+    it leaves the same pending pass (rolled back here)."""
+    import torch
+    st, _, _ = stage3
+    pos = st.committed_len
+    h16 = synth.hidden(FULL, 11, 0, n).astype(np.float16)
+    x16 = torch.from_numpy(h16.copy()).cuda()
+    st.forward_f16(x16, pos)
+    torch.cuda.synchronize()
+    st.sync()
+    got16 = x16.cpu().numpy()
+    assert st.pending == n
+    st.rollback()
+    out32 = run(st, h16.astype(np.float32), pos)
+    st.rollback()
+    with np.errstate(over="ignore"):      # outputs beyond 65504 round to +-inf, on both sides
+        want16 = out32.astype(np.float16)
+    assert np.array_equal(got16.view(np.uint16), want16.view(np.uint16))
+    assert st.committed_len == pos
