@@ -472,3 +472,100 @@ def test_stage_rejects_protocol_errors():
 def test_max_rel_err_definition():
     assert oracle.max_rel_err([1.0, 2.0], [1.0, 2.0]) == 0.0
     assert oracle.max_rel_err([1.0, 2.002], [1.0, 2.0]) == pytest.approx(1e-3)
+
+
+# ------------------------------------------------- layer wiring, closed form --
+# A constant hidden vector makes RMSNorm a closed form (c / sqrt(c^2 + eps) * gamma)
+# and one-hot Q4_0 rows make every projection pick one scaled input, so a whole
+# layer reduces to a few scalar formulas.  These pin the composition
+# h += mixer(RMSNorm_1(h)); h += W_down(silu(W_gate x) * W_up x), x = RMSNorm_2(h)
+# (ChatTorrent README, "What it can run"): a swapped norm weight, an FFN fed the
+# un-normed h, gate and up exchanged, or a missing residual fails them.
+
+def _onehot_q4(rows, cols, picks, scales):
+    """GGUF Q4_0 blocks of a [rows, cols] matrix whose row r is scales[r] at
+    column picks[r] and 0 elsewhere (nibble 9 = +1 unit there, 8 elsewhere)."""
+    scales = np.ascontiguousarray(np.broadcast_to(np.asarray(scales, dtype=np.float16), (rows,)))
+    W = np.empty((rows, cols // 32, 18), np.uint8)
+    W[:, :, 0:2] = scales.view(np.uint8).reshape(rows, 1, 2)
+    W[:, :, 2:] = 0x88
+    for r, c in enumerate(picks):
+        b, j = divmod(int(c), 32)
+        byte = 2 + j % 16
+        W[r, b, byte] = (W[r, b, byte] & 0xF0) | 0x09 if j < 16 else (W[r, b, byte] & 0x0F) | 0x90
+    return W
+
+
+def _zero_q4(W):
+    Z = W.copy()
+    Z[:, :, 2:] = 0x88
+    return Z
+
+
+def test_onehot_helper_dequantises_to_the_intended_matrix():
+    W = _onehot_q4(3, 64, [0, 17, 63], [0.5, -1.5, 2.0])
+    A = oracle.dequant(Q4_0, W)
+    want = np.zeros((3, 64))
+    want[0, 0], want[1, 17], want[2, 63] = 0.5, -1.5, 2.0
+    assert np.array_equal(A, want)
+
+
+def test_layer_wiring_ffn_reads_norm2_and_adds_to_h():
+    sh = TINY
+    H, F = sh.hidden, sh.ffn
+    t = synth.stage_tensors(sh, Q4_0, 7, 0, 1)                    # layer 0: gated DeltaNet
+    g1 = t["blk.0.norm1"].astype(np.float64)
+    g2 = t["blk.0.norm2"].astype(np.float64)
+    assert not np.allclose(g1, g2)
+    rng = np.random.default_rng(70)
+    cg, cu, cd = rng.integers(0, H, F), rng.integers(0, H, F), rng.integers(0, F, H)
+    t["blk.0.dn_out"] = _zero_q4(t["blk.0.dn_out"])              # the mixer adds exact zeros
+    t["blk.0.ffn_gate"] = _onehot_q4(F, H, cg, 0.75)
+    t["blk.0.ffn_up"] = _onehot_q4(F, H, cu, -1.5)
+    t["blk.0.ffn_down"] = _onehot_q4(H, F, cd, 0.5)
+    st = oracle.OracleStage(sh, Q4_0, t, 0, 1, 8)
+    st.set_dn_state(0, synth.dn_state(sh, 7, 0, 0.3))
+    consts = np.array([1.7, -0.4])
+    h = np.repeat(consts[:, None], H, axis=1)
+    out = st.forward(h, 0)
+    for i, c in enumerate(consts):
+        x2 = c / np.sqrt(c * c + sh.eps) * g2
+        g, u = 0.75 * x2[cg], -1.5 * x2[cu]
+        f = g / (1.0 + np.exp(-g)) * u
+        np.testing.assert_allclose(out[i], c + 0.5 * f[cd], rtol=1e-13, atol=1e-15)
+
+
+def test_layer_wiring_attention_reads_norm1_and_adds_gated_v_to_h():
+    """Attention layer at position 0: the softmax runs over one cached row (the
+    token's own), so o = v as stored in the f16 cache, then o * sigmoid(gate)."""
+    sh = TINY
+    H = sh.hidden
+    l = 3
+    assert sh.is_attention(l)
+    t = synth.stage_tensors(sh, Q4_0, 8, l, l + 1)
+    g1 = t[f"blk.{l}.norm1"].astype(np.float64)
+    Hq, Hkv, dh = sh.att_q_heads, sh.att_kv_heads, sh.att_dim
+    rep = Hq // Hkv
+    nq, nkv = Hq * dh, Hkv * dh
+    rows = 2 * nq + 2 * nkv                                       # q | gate | k | v
+    rng = np.random.default_rng(80)
+    picks = rng.integers(0, H, rows)
+    scales = np.full(rows, 0.5)
+    scales[nq:2 * nq] = -0.75                                     # gate rows
+    scales[2 * nq + nkv:] = 1.25                                  # v rows
+    t[f"blk.{l}.attn_in"] = _onehot_q4(rows, H, picks, scales)
+    co = rng.integers(0, nq, H)
+    t[f"blk.{l}.attn_out"] = _onehot_q4(H, nq, co, 0.25)
+    for tag in ("ffn_gate", "ffn_up", "ffn_down"):
+        t[f"blk.{l}.{tag}"] = _zero_q4(t[f"blk.{l}.{tag}"])      # the FFN adds exact zeros
+    st = oracle.OracleStage(sh, Q4_0, t, l, l + 1, 8)
+    c = 0.9
+    h = np.full((1, H), c)
+    out = st.forward(h, 0)
+    x1 = c / np.sqrt(c * c + sh.eps) * g1
+    gate = -0.75 * x1[picks[nq:2 * nq]]
+    v = 1.25 * x1[picks[2 * nq + nkv:]]                          # [Hkv * dh]
+    v16 = v.astype(np.float16).astype(np.float64)                # the cache holds f16
+    j = np.arange(nq)
+    o = v16[(j // dh) // rep * dh + j % dh] / (1.0 + np.exp(-gate))
+    np.testing.assert_allclose(out[0], c + 0.25 * o[co], rtol=1e-13, atol=1e-15)
