@@ -569,3 +569,50 @@ def test_layer_wiring_attention_reads_norm1_and_adds_gated_v_to_h():
     j = np.arange(nq)
     o = v16[(j // dh) // rep * dh + j % dh] / (1.0 + np.exp(-gate))
     np.testing.assert_allclose(out[0], c + 0.25 * o[co], rtol=1e-13, atol=1e-15)
+
+
+def test_layer_wiring_deltanet_rows_maps_heads_and_readout():
+    """One token through a gated-DeltaNet layer from a random state S0, with the
+    FFN zeroed and one-hot in/out projections: per value head h (key head
+    g = h // (Hv/Hk)), in the rank-one form of the update read out after it,
+        o_h = alpha_h (S0_h q - beta_h (S0_h k)(k.q)) + beta_h v_h (k.q),
+    q, k L2-normalised, beta = sigmoid(b), alpha = exp(-softplus(a)) = 1/(1+e^a),
+    in-projection rows q | k | v | b | a."""
+    sh = TINY
+    H = sh.hidden
+    Hk, Hv, d = sh.dn_k_heads, sh.dn_v_heads, sh.dn_dim
+    rep = Hv // Hk
+    t = synth.stage_tensors(sh, Q4_0, 9, 0, 1)
+    g1 = t["blk.0.norm1"].astype(np.float64)
+    rows = 2 * Hk * d + Hv * d + 2 * Hv
+    rng = np.random.default_rng(90)
+    picks = rng.integers(0, H, rows)
+    scales = np.empty(rows)
+    o_k, o_v, o_b = Hk * d, 2 * Hk * d, 2 * Hk * d + Hv * d
+    scales[:o_k], scales[o_k:o_v], scales[o_v:o_b] = 0.5, -0.75, 1.25
+    scales[o_b:o_b + Hv], scales[o_b + Hv:] = 0.5, -1.0
+    t["blk.0.dn_in"] = _onehot_q4(rows, H, picks, scales)
+    co = rng.integers(0, Hv * d, H)
+    t["blk.0.dn_out"] = _onehot_q4(H, Hv * d, co, 0.25)
+    for tag in ("ffn_gate", "ffn_up", "ffn_down"):
+        t[f"blk.0.{tag}"] = _zero_q4(t[f"blk.0.{tag}"])
+    S0 = synth.dn_state(sh, 9, 0, 0.3).astype(np.float64)        # [Hv, dv, dk]
+    st = oracle.OracleStage(sh, Q4_0, t, 0, 1, 8)
+    st.set_dn_state(0, S0.astype(np.float32))
+    c = 1.3
+    out = st.forward(np.full((1, H), c), 0)
+    y = scales * (c / np.sqrt(c * c + sh.eps) * g1)[picks]        # the in-projection, row by row
+    q = y[:o_k].reshape(Hk, d)
+    k = y[o_k:o_v].reshape(Hk, d)
+    v = y[o_v:o_b].reshape(Hv, d)
+    b, a = y[o_b:o_b + Hv], y[o_b + Hv:]
+    q = q / np.sqrt((q * q).sum(-1, keepdims=True) + 1e-6)
+    k = k / np.sqrt((k * k).sum(-1, keepdims=True) + 1e-6)
+    beta, alpha = 1.0 / (1.0 + np.exp(-b)), 1.0 / (1.0 + np.exp(a))
+    S0 = S0.astype(np.float32).astype(np.float64)
+    o = np.empty((Hv, d))
+    for h in range(Hv):
+        gq, gk = q[h // rep], k[h // rep]
+        kq = gk @ gq
+        o[h] = alpha[h] * (S0[h] @ gq - beta[h] * (S0[h] @ gk) * kq) + beta[h] * v[h] * kq
+    np.testing.assert_allclose(out[0], c + 0.25 * o.reshape(-1)[co], rtol=1e-12, atol=1e-14)
