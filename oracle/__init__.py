@@ -33,7 +33,7 @@ Sources (page title, part of the page):
   of 256, RoPE on the first 64 dims with theta 1e7, eps 1e-6 and a 3:1
   DeltaNet:attention pattern are the defaults of ``synth.StageShape``.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
 
 * RMSNorm is ``x / sqrt(mean(x^2) + eps) * gamma`` with gamma applied as given.
 * q, k of a DeltaNet key head are L2-normalised as ``x / sqrt(sum(x^2) + 1e-6)``.
