@@ -178,9 +178,11 @@ stage_status stage_set_kv_len(stage_t* st, int kv_len);
 
 /* Dequantise row `row` of weight tensor `tensor` (a name as in stage_tensor)
  * from the stage's packed device copy, with the same device code the GEMV
- * uses, into host_dst (f32 [cols]).  Synchronous.  Used to check that the
- * repacked weights dequantise bit-exactly. */
-stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst);
+ * uses, into host_dst (f32 [cols], the tensor's column count; dst_elems = the
+ * buffer's capacity in floats, STAGE_E_ARG if it is smaller, before any
+ * device work).  Synchronous.  Used to check that the repacked weights
+ * dequantise bit-exactly. */
+stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst, size_t dst_elems);
 
 /* How a pass runs on the device.
  *   STAGE_PASS_KERNELS (default): one kernel per step, all recorded in a CUDA

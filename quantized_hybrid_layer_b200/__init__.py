@@ -91,7 +91,7 @@ def lib() -> ctypes.CDLL:
             "stage_get_kv": (i, [vp, i, vp, vp, sz]),
             "stage_set_kv": (i, [vp, i, vp, vp, sz]),
             "stage_set_kv_len": (i, [vp, i]),
-            "stage_debug_dequant": (i, [vp, ctypes.c_char_p, i, vp]),
+            "stage_debug_dequant": (i, [vp, ctypes.c_char_p, i, vp, sz]),
             "stage_set_pass_mode": (i, [vp, i]),
             "stage_pass_persistent": (i, [vp, i]),
             "stage_set_trace": (i, [vp, i]),
@@ -126,6 +126,14 @@ def _ptr(t) -> int:
     return int(t.data_ptr())
 
 
+def _check_hidden(hidden, dtype: str, width: int):
+    """A forward's hidden buffer: contiguous CUDA tensor of `dtype`, [n_tok, width]."""
+    if not (hidden.is_cuda and str(hidden.dtype) == f"torch.{dtype}" and hidden.is_contiguous()
+            and hidden.dim() == 2 and hidden.shape[1] == width):
+        raise ValueError(f"hidden must be a contiguous CUDA {dtype} tensor [n_tok, {width}], got "
+                         f"{hidden.dtype} {tuple(hidden.shape)} on {hidden.device}")
+
+
 def _check_qhl(rc: int):
     if rc != 0:
         raise StageError(rc, lib().qhl_last_error().decode())
@@ -152,7 +160,7 @@ class Stage:
     # the pass -------------------------------------------------------------
     def forward(self, hidden, pos: int):
         """hidden: contiguous CUDA float32 tensor [n_tok, hidden], updated in place."""
-        assert hidden.is_cuda and hidden.dtype.itemsize == 4 and hidden.is_contiguous()
+        _check_hidden(hidden, "float32", self.cfg.hidden)
         n = hidden.shape[0]
         self._check(lib().stage_forward(self._h, _ptr(hidden), n, pos))
         return hidden
@@ -160,7 +168,7 @@ class Stage:
     def forward_f16(self, hidden, pos: int):
         """hidden: contiguous CUDA float16 tensor [n_tok, hidden] (the wire format),
         updated in place with the pass's f32 result rounded to nearest even."""
-        assert hidden.is_cuda and hidden.dtype.itemsize == 2 and hidden.is_floating_point() and hidden.is_contiguous()
+        _check_hidden(hidden, "float16", self.cfg.hidden)
         n = hidden.shape[0]
         self._check(lib().stage_forward_f16(self._h, _ptr(hidden), n, pos))
         return hidden
@@ -238,8 +246,12 @@ class Stage:
         return K, V
 
     def set_kv(self, layer: int, K: np.ndarray, V: np.ndarray):
+        c = self.cfg
         K = np.ascontiguousarray(K, dtype=np.float16)
         V = np.ascontiguousarray(V, dtype=np.float16)
+        want = (c.att_kv_heads, c.max_ctx, c.att_dim)
+        if K.shape != want or V.shape != want:
+            raise ValueError(f"K and V must both be f16 {want}, got {K.shape} and {V.shape}")
         self._check(lib().stage_set_kv(self._h, layer, K.ctypes.data, V.ctypes.data, K.nbytes))
 
     def set_kv_len(self, n: int):
@@ -247,7 +259,7 @@ class Stage:
 
     def debug_dequant(self, tensor: str, row: int, cols: int) -> np.ndarray:
         out = np.empty(cols, dtype=np.float32)
-        self._check(lib().stage_debug_dequant(self._h, tensor.encode(), row, out.ctypes.data))
+        self._check(lib().stage_debug_dequant(self._h, tensor.encode(), row, out.ctypes.data, out.size))
         return out
 
     def free(self):

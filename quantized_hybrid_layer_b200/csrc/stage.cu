@@ -756,7 +756,7 @@ stage_status stage_set_kv_len(stage_t* st, int kv_len) {
   return STAGE_OK;
 }
 
-stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst) {
+stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst, size_t dst_elems) {
   if (!st) return STAGE_E_ARG;
   int layer;
   std::string tag;
@@ -779,6 +779,9 @@ stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float
     return fail(st, STAGE_E_ARG, "not a quantised tensor of this layer");
   }
   if (row < 0 || row >= rows) return fail(st, STAGE_E_ARG, "row out of range");
+  if (dst_elems < (size_t)cols)
+    return fail(st, STAGE_E_ARG, "host_dst holds " + std::to_string(dst_elems) + " floats; the row has " +
+                                     std::to_string(cols));
   float* tmp = nullptr;
   cudaError_t e = cudaMalloc(&tmp, (size_t)cols * 4);
   if (e != cudaSuccess) return fail(st, STAGE_E_OOM, cuda_msg("cudaMalloc", e));

@@ -93,3 +93,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path, qhl):
     monkeypatch.setattr(qhl, "_lib", None)
     with pytest.raises(ImportError):
         qhl.lib()
+
+
+def test_binding_rejects_bad_buffers_before_calling_the_library(qhl):
+    """The binding checks dtype, device, layout and shape itself, so a wrong
+    buffer never reaches the C ABI (whose calls trust their sizes)."""
+    import numpy as np
+    import torch
+    cfg = qhl.StageConfig(5120, 17408, 16, 48, 128, 24, 4, 256, 64, 1e7, 1e-6, 4, 4352, 2)
+    st = qhl.Stage(0, cfg, 0, 4)                                # no handle: nothing is loaded
+    with pytest.raises(ValueError):
+        st.forward(torch.zeros(1, 5120), 0)                     # host tensor
+    with pytest.raises(ValueError):
+        st.forward_f16(torch.zeros(1, 5120, dtype=torch.float16), 0)
+    K = np.zeros((4, 4352, 256), np.float16)
+    with pytest.raises(ValueError):
+        st.set_kv(3, K, K[:, :100])                             # V shorter than K
+    with pytest.raises(ValueError):
+        st.set_kv(3, K[:, :100], K[:, :100])                    # neither the cache's shape
