@@ -1,9 +1,9 @@
 // The whole layer-stage pass in one persistent, cooperative kernel.
 //
 // The pages submit one command buffer per token (SwarmLLM README, paragraph
-// after the peer diagram); this takes that one step further on B200: instead of a chain of kernels (each
-// paying launch, ramp-up and tail), one grid of two CTAs per SM runs every
-// phase of the pass -- stage input, then per layer the mixer in-projection,
+// after the peer diagram); this takes that one step further on B200: instead
+// of a chain of kernels (each paying launch, ramp-up and tail), one grid of
+// two CTAs per SM runs every phase of the pass -- stage input, then per layer the mixer in-projection,
 // the DeltaNet step or the attention partials + combine, the out-projection,
 // gate/up and down -- separated by grid-wide barriers (a monotonic counter in
 // global memory; every wait is bounded).
