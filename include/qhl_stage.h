@@ -251,6 +251,7 @@ int qhl_repack(int qtype, int rows, int cols, const void* gguf_dev, const void* 
 
 /* Dequantise rows [row0, row0+nrows) of a packed matrix into out_dev (f32
  * [nrows, cols]) with the GEMV's own conversion code; bit-exact by design.
+ * packed_dev must be 16-byte aligned (STAGE_E_ARG otherwise).
  * paired != 0: rows 0..rows-1 address the first matrix of a pair, rows
  * rows..2*rows-1 the second. */
 int qhl_dequant(int qtype, int rows, int cols, const void* packed_dev, int paired, int row0, int nrows,
@@ -271,7 +272,9 @@ int qhl_qgemv(int qtype, int rows, int cols, const void* packed_dev, const float
  * q | k | v | b | a per token (q, k are L2-normalised here; beta = sigmoid(b),
  * alpha = exp(-softplus(a))).  s_in_dev: f32 [Hv, 128, 128] state before the
  * first token (not modified).  snaps_dev: f32 [n_tok, Hv, 128, 128] receives
- * the state after each token.  o_dev: f32 [n_tok, Hv*128] receives o_t = S_t q_t. */
+ * the state after each token.  o_dev: f32 [n_tok, Hv*128] receives o_t = S_t q_t.
+ * y_dev, s_in_dev and snaps_dev are read / written as 16-byte vectors and must
+ * be 16-byte aligned (STAGE_E_ARG otherwise, before any device work). */
 int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float* s_in_dev,
                       float* snaps_dev, float* o_dev, void* stream);
 

@@ -113,6 +113,7 @@ int qhl_dequant(int qtype, int rows, int cols, const void* packed_dev, int paire
   if (!valid_qt(qtype) || !packed_dev || !out_dev || rows <= 0 || cols <= 0 || cols % kChunkCols || row0 < 0 ||
       nrows < 0 || row0 + nrows > total)
     return err(STAGE_E_ARG, "qhl_dequant: bad argument");
+  if (reinterpret_cast<uintptr_t>(packed_dev) % 16) return err(STAGE_E_ARG, "qhl_dequant: packed_dev not 16-byte aligned");
   cudaError_t e = launch_dequant(qtype, static_cast<const uint8_t*>(packed_dev), rows, cols, paired ? 1 : 0, row0,
                                  nrows, out_dev, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? 0 : cuda_err("dequant", e);
@@ -156,6 +157,9 @@ int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float
                       float* o_dev, void* stream) {
   if (Hk <= 0 || Hv <= 0 || Hv % Hk || !y_dev || !s_in_dev || !snaps_dev || !o_dev || n_tok < 1 || n_tok > 16)
     return err(STAGE_E_ARG, "qhl_deltanet_step: bad argument");
+  if (reinterpret_cast<uintptr_t>(y_dev) % 16 || reinterpret_cast<uintptr_t>(s_in_dev) % 16 ||
+      reinterpret_cast<uintptr_t>(snaps_dev) % 16)
+    return err(STAGE_E_ARG, "qhl_deltanet_step: y_dev, s_in_dev and snaps_dev must be 16-byte aligned");
   DnArgs d = {};
   d.y = y_dev;
   d.y_stride = 2 * Hk * kDnDim + Hv * kDnDim + 2 * Hv;

@@ -84,6 +84,14 @@ def test_bad_arguments_are_rejected_before_any_device_work(qhl):
     assert lib.qhl_qgemv(2, 64, 256, 16, 16, 17, 16, None) == -1          # n_tok > 16
     assert lib.qhl_deltanet_step(16, 47, 16, 1, 16, 16, 16, None) == -1   # Hv % Hk
     assert lib.qhl_repack(2, 64, 300, 16, None, 16, None) == -1           # cols % 256
+    # pointers the kernels read as 16-byte vectors are checked before any device work
+    assert lib.qhl_qgemv(2, 64, 256, 16 + 4, 16, 1, 16, None) == -1       # packed_dev misaligned
+    assert b"aligned" in lib.qhl_last_error()
+    assert lib.qhl_dequant(2, 64, 256, 16 + 8, 0, 0, 1, 16, None) == -1    # packed_dev misaligned
+    assert b"aligned" in lib.qhl_last_error()
+    assert lib.qhl_deltanet_step(16, 48, 16 + 4, 1, 16, 16, 16, None) == -1  # y_dev misaligned
+    assert lib.qhl_deltanet_step(16, 48, 16, 1, 16, 16 + 8, 16, None) == -1  # snaps_dev misaligned
+    assert b"aligned" in lib.qhl_last_error()
     lib.stage_free(None)                                                  # no-op
 
 
