@@ -122,6 +122,17 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
  * commit(1) each). */
 stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos);
 
+/* stage_forward from and to host memory, the whole round trip in one call:
+ * hidden_in_host f32 [n_tok, H] is copied to the device, the pass runs, and
+ * the result is copied to hidden_out_host f32 [n_tok, H] (both caller-owned,
+ * row-major; they may be the same buffer).  All three steps are ordered on the
+ * stage's stream: with page-locked buffers the call returns at once and
+ * hidden_out_host is complete once that stream is synchronised (stage_sync);
+ * with pageable buffers the CUDA runtime copies synchronously.  Same state
+ * rules and errors as stage_forward; the output is bit-identical to it. */
+stage_status stage_forward_host(stage_t* st, const float* hidden_in_host, float* hidden_out_host, int n_tok,
+                                int pos);
+
 /* stage_forward with the hidden state in IEEE binary16, the form a peer sends
  * on the wire (SwarmLLM README, paragraph under the benchmark table: one
  * token's 5,120-value hidden state is 10 KB as f16; github-Nehanth-swarmllm

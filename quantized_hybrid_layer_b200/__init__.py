@@ -30,7 +30,7 @@ STATUS = {
 
 #: every symbol include/qhl_stage.h declares
 EXPORTS = (
-    "stage_load", "stage_forward", "stage_forward_f16", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
+    "stage_load", "stage_forward", "stage_forward_host", "stage_forward_f16", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
     "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_set_pass_mode", "stage_pass_persistent",
     "stage_set_trace", "stage_get_trace",
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
                                ctypes.POINTER(vp)]),
             "stage_forward": (i, [vp, vp, i, i]),
             "stage_forward_f16": (i, [vp, vp, i, i]),
+            "stage_forward_host": (i, [vp, vp, vp, i, i]),
             "stage_commit": (i, [vp, i]),
             "stage_rollback": (i, [vp]),
             "stage_reset": (i, [vp]),
@@ -134,6 +135,24 @@ def _check_hidden(hidden, dtype: str, width: int):
                          f"{hidden.dtype} {tuple(hidden.shape)} on {hidden.device}")
 
 
+def _host_ptr(x) -> int:
+    return int(x.data_ptr()) if hasattr(x, "data_ptr") else int(x.ctypes.data)
+
+
+def _check_host_hidden(x, width: int) -> int:
+    """A host f32 [n_tok, width] C-contiguous buffer (numpy array or CPU torch tensor); returns n_tok."""
+    if hasattr(x, "data_ptr"):
+        ok = (not x.is_cuda and str(x.dtype) == "torch.float32" and x.is_contiguous() and x.dim() == 2
+              and x.shape[1] == width)
+    else:
+        ok = (isinstance(x, np.ndarray) and x.dtype == np.float32 and x.flags.c_contiguous and x.ndim == 2
+              and x.shape[1] == width)
+    if not ok:
+        raise ValueError(f"expected a host C-contiguous float32 [n_tok, {width}] buffer, got "
+                         f"{type(x).__name__} {getattr(x, 'dtype', None)} {tuple(getattr(x, 'shape', ()))}")
+    return int(x.shape[0])
+
+
 def _check_qhl(rc: int):
     if rc != 0:
         raise StageError(rc, lib().qhl_last_error().decode())
@@ -172,6 +191,19 @@ class Stage:
         n = hidden.shape[0]
         self._check(lib().stage_forward_f16(self._h, _ptr(hidden), n, pos))
         return hidden
+
+    def forward_host_buffers(self, hidden_in, hidden_out, pos: int, sync: bool = True):
+        """One C call from host memory: copy in, pass, copy out (stage_forward_host).
+        hidden_in / hidden_out: host f32 [n_tok, hidden], C-contiguous numpy arrays or
+        CPU torch tensors (page-locked for asynchronous copies); they may be the same
+        buffer.  With sync=False the caller synchronises before reading hidden_out."""
+        n = _check_host_hidden(hidden_in, self.cfg.hidden)
+        if _check_host_hidden(hidden_out, self.cfg.hidden) != n:
+            raise ValueError("hidden_in and hidden_out must hold the same number of tokens")
+        self._check(lib().stage_forward_host(self._h, _host_ptr(hidden_in), _host_ptr(hidden_out), n, pos))
+        if sync:
+            self.sync()
+        return hidden_out
 
     def forward_host(self, hidden_host, pos: int, dev_buf=None):
         """End-to-end call from host memory: H2D copy, forward, D2H copy (on the stage stream)."""

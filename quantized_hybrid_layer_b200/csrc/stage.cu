@@ -626,7 +626,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
 // Checks shared by both forward entries; builds the n_tok graph on first use.
 static stage_status forward_begin(stage_t* st, const void* hidden_dev, int n_tok, int pos) {
   if (!st) return STAGE_E_ARG;
-  if (!hidden_dev) return fail(st, STAGE_E_ARG, "hidden_dev is NULL");
+  if (!hidden_dev) return fail(st, STAGE_E_ARG, "hidden buffer is NULL");
   if (n_tok < 1 || n_tok > kMaxTok) return fail(st, STAGE_E_ARG, "n_tok must be in 1..16");
   if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending: commit or roll back first");
   if (pos != st->committed) return fail(st, STAGE_E_STATE, "pos must equal the committed length");
@@ -642,6 +642,20 @@ stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos) {
   CK(cudaMemcpyAsync(st->h, hidden_dev, bytes, cudaMemcpyDeviceToDevice, st->stream));
   CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
   CK(cudaMemcpyAsync(hidden_dev, st->h, bytes, cudaMemcpyDeviceToDevice, st->stream));
+  st->pending_n = n_tok;
+  st->pending_pos = pos;
+  return STAGE_OK;
+}
+
+stage_status stage_forward_host(stage_t* st, const float* hidden_in_host, float* hidden_out_host, int n_tok,
+                                int pos) {
+  if (st && !hidden_out_host) return fail(st, STAGE_E_ARG, "hidden_out_host is NULL");
+  stage_status s = forward_begin(st, hidden_in_host, n_tok, pos);
+  if (s != STAGE_OK) return s;
+  const size_t bytes = (size_t)n_tok * st->cfg.hidden * 4;
+  CK(cudaMemcpyAsync(st->h, hidden_in_host, bytes, cudaMemcpyHostToDevice, st->stream));
+  CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
+  CK(cudaMemcpyAsync(hidden_out_host, st->h, bytes, cudaMemcpyDeviceToHost, st->stream));
   st->pending_n = n_tok;
   st->pending_pos = pos;
   return STAGE_OK;

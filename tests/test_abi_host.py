@@ -76,6 +76,7 @@ def test_bad_arguments_are_rejected_before_any_device_work(qhl):
     assert out.value is None
     assert lib.stage_forward(None, None, 1, 0) == -1
     assert lib.stage_forward_f16(None, None, 1, 0) == -1
+    assert lib.stage_forward_host(None, None, None, 1, 0) == -1
     assert lib.stage_commit(None, 0) == -1
     assert lib.stage_rollback(None) == -1
     assert lib.stage_committed_len(None) == -1
@@ -114,6 +115,12 @@ def test_binding_rejects_bad_buffers_before_calling_the_library(qhl):
         st.forward(torch.zeros(1, 5120), 0)                     # host tensor
     with pytest.raises(ValueError):
         st.forward_f16(torch.zeros(1, 5120, dtype=torch.float16), 0)
+    with pytest.raises(ValueError):
+        st.forward_host_buffers(np.zeros((1, 5120), np.float64), np.zeros((1, 5120), np.float32), 0)
+    with pytest.raises(ValueError):
+        st.forward_host_buffers(np.zeros((2, 5120), np.float32), np.zeros((1, 5120), np.float32), 0)
+    with pytest.raises(ValueError):
+        st.forward_host_buffers(np.zeros((1, 5120), np.float32), np.zeros((1, 10240), np.float32)[:, ::2], 0)
     K = np.zeros((4, 4352, 256), np.float16)
     with pytest.raises(ValueError):
         st.set_kv(3, K, K[:, :100])                             # V shorter than K

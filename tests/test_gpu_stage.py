@@ -370,3 +370,25 @@ def test_f16_boundary_equals_the_f32_pass_rounded(q, stage3, n):
         want16 = out32.astype(np.float16)
     assert np.array_equal(got16.view(np.uint16), want16.view(np.uint16))
     assert st.committed_len == pos
+
+
+def test_forward_from_host_buffers_equals_the_device_pass(q, stage3):
+    """stage_forward_host (copy in, pass, copy out in one C call) gives the
+    bits of stage_forward on a device buffer: pageable numpy buffers, and a
+    page-locked torch buffer used in place."""
+    import torch
+    st, _, _ = stage3
+    pos = st.committed_len
+    h = synth.hidden(FULL, 12, 0, 3)
+    out = np.empty_like(h)
+    st.forward_host_buffers(h, out, pos)
+    assert st.pending == 3
+    st.rollback()
+    ref = run(st, h, pos)
+    st.rollback()
+    assert np.array_equal(out, ref)
+    hp = torch.from_numpy(h.copy()).pin_memory()
+    st.forward_host_buffers(hp, hp, pos)
+    st.rollback()
+    assert np.array_equal(hp.numpy(), ref)
+    assert st.committed_len == pos
