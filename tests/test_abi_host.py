@@ -30,6 +30,24 @@ def declared_functions():
     return sorted(set(names))
 
 
+def declared_prototypes():
+    """{name: parameter count} of every function prototype in the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    protos = {}
+    for m in re.finditer(r"\b((?:stage|qhl)_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = " ".join(m.group(2).split())
+        protos[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return protos
+
+
+def test_binding_signatures_match_the_header(qhl):
+    protos = declared_prototypes()
+    assert set(protos) == set(declared_functions())
+    lib = qhl.lib()
+    for name, n in protos.items():
+        assert len(getattr(lib, name).argtypes) == n, name
+
+
 def test_header_declares_the_four_calls_of_the_stage():
     names = declared_functions()
     for n in ("stage_load", "stage_forward", "stage_commit", "stage_rollback"):
