@@ -4,9 +4,10 @@
 // ring of DeltaNet state snapshots per DeltaNet layer, an f16 KV cache per
 // attention layer, activation buffers for up to 16 tokens, and one CUDA graph
 // per token count.  stage_forward launches that graph, a single submission per
-// pass as on the pages (SwarmLLM README, paragraph after the peer diagram).  Inside the graph
-// every kernel after the first is launched with programmatic dependent launch,
-// so a projection's weights start streaming while the previous kernel drains.
+// pass as on the pages (SwarmLLM README, paragraph after the peer diagram).
+// Inside the graph every kernel after the first is launched with programmatic
+// dependent launch, so a projection's weights start streaming while the
+// previous kernel drains.
 //
 // The position of the pass and each DeltaNet layer's current ring slot live in
 // a small device control block (ctrl[0] = committed length, ctrl[1 + i] = ring
