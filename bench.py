@@ -127,11 +127,9 @@ def pass_bytes(shape, qtype, layers, ctx: int, n_tok: int = 1) -> dict:
     return {"weights": w, "kv": kv, "state": state, "total": w + kv + state}
 
 
-def launches_per_pass(shape, layers, persistent: bool) -> int:
-    """Kernels the stage launches per pass: one persistent kernel, or input +
-    per layer (in-proj, mixer kernel(s), out-proj, gate/up, down)."""
-    if persistent:
-        return 1
+def launches_per_pass(shape, layers) -> int:
+    """Kernels the stage launches per pass: input + per layer (in-proj, mixer
+    kernel(s), out-proj, gate/up, down)."""
     n = 1
     for l in layers:
         n += 6 if shape.is_attention(l) else 5
@@ -174,8 +172,12 @@ def committed_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while running."""
+    """SM clocks and clock-event (throttle) reasons sampled while the timed
+    region runs: NVML polled every 10 ms from a host thread (the timed regions
+    last tens of milliseconds), nvidia-smi at its 200 ms period as the fallback
+    where NVML is unavailable.  Only reads; changes no GPU setting."""
 
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -183,8 +185,48 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
+        self.thread = None
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
+
+    def _nvml_loop(self, stop):
+        import pynvml as nv
+        h = self._handle(nv)
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        while True:
+            mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.samples.append((mhz, {n for n, b in bits.items() if r & b}))
+            if stop.wait(0.01):
+                break
+
+    def _handle(self, nv):
+        """NVML handle of CUDA device self.idx, matched by UUID (CUDA and NVML
+        number the GPUs differently when CUDA_VISIBLE_DEVICES is set)."""
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.idx)
 
     def start(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self._handle(nv)
+            self.stop_ev = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(self.stop_ev,), daemon=True)
+            self.thread.start()
+            return
+        except Exception as e:   # no NVML: fall back to nvidia-smi
+            self.err = str(e)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -193,8 +235,15 @@ class ClockSampler:
             self.proc = None
 
     def stop(self) -> dict:
+        if self.thread is not None:
+            self.stop_ev.set()
+            self.thread.join(timeout=5)
+            sm = [m for m, _ in self.samples]
+            reasons = set().union(*[r for _, r in self.samples]) if self.samples else set()
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(reasons), "samples": len(sm), "source": "nvml, 10 ms"}
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
@@ -202,7 +251,6 @@ class ClockSampler:
             self.proc.kill()
             out, _ = self.proc.communicate()
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
@@ -212,11 +260,11 @@ class ClockSampler:
                 mx.append(float(f[2]))
             except ValueError:
                 continue
-            for name, v in zip(names, f[5:9]):
+            for name, v in zip(self.NAMES, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 200 ms"}
 
 
 def workload_config(args, shape) -> dict:
@@ -336,8 +384,6 @@ def run_ours(args, rank, world, local, pg):
     cfg = q.config_from_shape(shape, qtype, max_ctx)
     with torch.cuda.stream(stream):
         st = q.stage_load(cfg, tensors, 0, args.layers, stream=stream)
-        st.set_pass_mode(q.PASS_PERSISTENT if args.pass_mode == "persistent" else q.PASS_KERNELS)
-        persistent = st.pass_persistent(1)
         for l in layers:
             if shape.is_attention(l):
                 K, V = synth.kv_prefill(shape, SEED, l, CTX0, max_ctx)
@@ -375,31 +421,30 @@ def run_ours(args, rank, world, local, pg):
         tok_s = args.steps / dt
         value = tok_s * world
 
-        # ---- end to end: host buffers, copies inside the timed region ----
+        # ---- end to end through the C ABI's host-buffer call (stage_forward_host):
+        # every step copies its input from page-locked host memory, runs the
+        # pass and copies the result back, all inside the timed region ----
         e2e = None
         if not args.no_e2e:
             host_in = torch.from_numpy(synth.normal_f32(synth.rng_for(SEED, rank, 78), (n_steps, H))).pin_memory()
-            host_out = torch.empty((1, H), dtype=torch.float32).pin_memory()
-            dbuf = torch.empty((1, H), dtype=torch.float32, device=dev)
+            host_out = torch.empty((n_steps, H), dtype=torch.float32).pin_memory()
             for i in range(args.warmup):
-                host_out.copy_(host_in[i:i + 1])
-                st.forward_host(host_out, st.committed_len, dbuf)
+                st.forward_host_buffers(host_in[i:i + 1], host_out[i:i + 1], st.committed_len, sync=False)
                 st.commit(1)
             torch.cuda.synchronize()
             barrier(pg)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for i in range(args.warmup, n_steps):
-                dbuf.copy_(host_in[i:i + 1], non_blocking=True)
-                st.forward(dbuf, st.committed_len)
-                host_out.copy_(dbuf, non_blocking=True)
+                st.forward_host_buffers(host_in[i:i + 1], host_out[i:i + 1], st.committed_len, sync=False)
                 st.commit(1)
             e1.record(stream)
             torch.cuda.synchronize()
             barrier(pg)
+            st.sync()
             dte = max_over_ranks(e0.elapsed_time(e1) / 1e3, pg)
             e2e = {"value": args.steps / dte * world, "unit": "tok/s", "h2d_bytes_per_step": H * 4,
-                   "d2h_bytes_per_step": H * 4}
+                   "d2h_bytes_per_step": H * 4, "call": "stage_forward_host (page-locked host buffers)"}
 
         # ---- prefill: 16-token chunks over a 2048-token prompt from position 0 ----
         prefill = None
@@ -407,15 +452,14 @@ def run_ours(args, rank, world, local, pg):
             st.reset()
             n_chunks = PROMPT // CHUNK
             ph = torch.from_numpy(synth.normal_f32(synth.rng_for(SEED, rank, 79), (n_chunks, CHUNK, H))).to(dev)
-            st.forward(ph[0].clone(), 0)             # builds the 16-token graph
-            st.rollback()
+            st.prefill(ph[0].clone(), 0, chunked=True)      # builds the 16-token prefill graph
+            st.reset()
             torch.cuda.synchronize()
             barrier(pg)
             p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             p0.record(stream)
             for c in range(n_chunks):
-                st.forward(ph[c], c * CHUNK)
-                st.commit(CHUNK)
+                st.prefill(ph[c], c * CHUNK, chunked=True)
             p1.record(stream)
             torch.cuda.synchronize()
             barrier(pg)
@@ -423,7 +467,8 @@ def run_ours(args, rank, world, local, pg):
             dtp = max_over_ranks(p0.elapsed_time(p1) / 1e3, pg)
             pbp = pass_bytes(shape, qtype, layers, PROMPT // 2, CHUNK)
             prefill = {"tok_s": PROMPT / dtp * world, "ms_per_chunk": dtp / n_chunks * 1e3,
-                       "weight_gbs": pbp["weights"] * n_chunks / dtp / 1e9, "chunks": n_chunks}
+                       "weight_gbs": pbp["weights"] * n_chunks / dtp / 1e9, "chunks": n_chunks,
+                       "call": "stage_prefill, chunked DeltaNet form"}
 
         weight_bytes_packed = st.weight_bytes
         st.free()
@@ -459,8 +504,7 @@ def run_ours(args, rank, world, local, pg):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (launches_per_pass(shape, layers, persistent) + 1) * args.steps,
-        "pass_mode": "persistent" if persistent else "kernels",
+        "gpu_launches": (launches_per_pass(shape, layers) + 1) * args.steps,
         "clocks": clk,
     }
     return res
@@ -473,8 +517,8 @@ def gemv_roofline(q, torch, dev, stream, shape, qtype, hbm_peak, peak_src):
     rows, cols = 2 * shape.ffn, shape.hidden
     nbytes = q.qhl_packed_bytes(qtype, rows, cols)
     copies = max(8, int(np.ceil(2.0e9 / nbytes)))
-    item = 9216 if qtype == Q4_0 else 17408
-    qb = 8192 if qtype == Q4_0 else 16384
+    item = 18432 if qtype == Q4_0 else 34816     # packed item: 128 rows x 256 columns
+    qb = 16384 if qtype == Q4_0 else 32768       # quants first, then the block scales
     mats = []
     with torch.cuda.stream(stream):
         g = torch.Generator(device=dev)
@@ -518,8 +562,6 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-roofline", action="store_true")
-    ap.add_argument("--pass-mode", choices=("kernels", "persistent"), default="kernels",
-                    help="one kernel per step (CUDA graph) or the one-kernel persistent pass")
     ap.add_argument("--only-kernel-roofline", action="store_true",
                     help="time only the dominant kernel alone (the GEMV roofline leg) and print it")
     args = ap.parse_args(argv)

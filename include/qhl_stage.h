@@ -105,7 +105,11 @@ typedef struct {
 } stage_tensor;
 
 /* Create a stage for layers [layer_begin, layer_end) on the current CUDA
- * device.  Uploads and repacks the weights, allocates recurrent states (zero),
+ * device.  A peer holds and runs one contiguous range of the model's layers
+ * (Unstable Legion, "Splitting the workload"; SwarmLLM README, peer
+ * diagram: layers 0-21 / 22-42 / 43-63), and its weights are GGUF blocks of
+ * 4-bit values with an f16 scale (SwarmLLM README, paragraph after the peer
+ * diagram, and model table: "GGUF Q4_0", "GGUF Q8_0 / Q4_0").  Uploads and repacks the weights, allocates recurrent states (zero),
  * KV caches (zero), a rollback ring of 17 snapshots per DeltaNet layer and all
  * scratch.  cuda_stream (a cudaStream_t, may be NULL for the legacy default
  * stream) orders every later call of this stage.  Blocks until the upload is
@@ -114,7 +118,12 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
                         int layer_begin, int layer_end, void* cuda_stream, stage_t** out);
 
 /* Run n_tok tokens (1..16) at positions pos .. pos+n_tok-1 through every layer
- * of the stage (one CUDA-graph launch).  hidden_dev: caller-owned device f32
+ * of the stage (one CUDA-graph launch).  The stage is handed an activation and
+ * hands back the activation its layers produce (Unstable Legion, "The
+ * runtime"); a token's pass reads every weight once, in one submission
+ * (SwarmLLM README, paragraph after the peer diagram); prefill moves 16
+ * tokens per hop and drafts are checked in one batched pass (SwarmLLM README,
+ * feature list).  hidden_dev: caller-owned device f32
  * [n_tok, H], row-major, read and overwritten in place with the stage output.
  * pos must equal the committed length.  Leaves the pass pending: the next
  * forward is refused until stage_commit / stage_rollback.  Token t's output is
@@ -146,14 +155,42 @@ stage_status stage_forward_host(stage_t* st, const float* hidden_in_host, float*
  * for a misaligned pointer, before any device work). */
 stage_status stage_forward_f16(stage_t* st, void* hidden_dev, int n_tok, int pos);
 
-/* Keep the first n_accepted tokens (0..n_tok) of the pending pass: each
+/* Prefill: run n_tok prompt tokens (1..16) at positions pos .. pos+n_tok-1
+ * through every layer and commit them all in the same call (a prompt chunk is
+ * never rolled back, so no per-token state snapshots are written: each
+ * DeltaNet layer writes its final state only, 3.1 MB per layer instead of
+ * n_tok times that).  Prefill sends 16 tokens per hop (SwarmLLM README,
+ * feature list); the DeltaNet recurrence is what makes prefill serial and the
+ * known gap (SwarmLLM README, under the benchmark table; github-Nehanth-
+ * swarmllm summary, "How it works").  mode:
+ *   STAGE_PREFILL_EXACT    the token-by-token recurrence, as stage_forward:
+ *                          output and committed state bit-identical to
+ *                          stage_forward + stage_commit(n_tok);
+ *   STAGE_PREFILL_CHUNKED  the chunked closed form of the recurrence: per
+ *                          value head one unit lower-triangular solve over the
+ *                          chunk instead of n_tok dependent token steps, with
+ *                          every dot product against the starting state
+ *                          independent; within rounding of the exact mode, not
+ *                          bit-identical to it.
+ * hidden_dev as in stage_forward (read and overwritten in place); pos must
+ * equal the committed length; no pass may be pending; afterwards the committed
+ * length is pos + n_tok and nothing is pending. */
+typedef enum { STAGE_PREFILL_EXACT = 0, STAGE_PREFILL_CHUNKED = 1 } stage_prefill_mode;
+stage_status stage_prefill(stage_t* st, float* hidden_dev, int n_tok, int pos, int mode);
+
+/* Keep the first n_accepted tokens (0..n_tok) of the pending pass: the
+ * accepted prefix of a speculative batch, whose rejected tail is undone
+ * exactly in the recurrent state (SwarmLLM README, paragraph after the peer
+ * diagram; github-Nehanth-swarmllm summary, "How it works").  Each
  * DeltaNet state becomes the snapshot after token n_accepted (no copy: the
  * ring index moves) and the committed length becomes pos + n_accepted.  KV
  * rows beyond it stay in memory but are never read and are overwritten by the
  * next pass.  The result is bit-identical to having run only those tokens. */
 stage_status stage_commit(stage_t* st, int n_accepted);
 
-/* Discard the pending pass: identical to stage_commit(st, 0). */
+/* Discard the pending pass: identical to stage_commit(st, 0).  This is the
+ * exact rollback of the recurrent state and KV cache when no draft is
+ * accepted (SwarmLLM README, paragraph after the peer diagram). */
 stage_status stage_rollback(stage_t* st);
 
 /* Start a new sequence: zero every recurrent state, committed length 0.
@@ -195,39 +232,19 @@ stage_status stage_set_kv_len(stage_t* st, int kv_len);
  * dequantise bit-exactly. */
 stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst, size_t dst_elems);
 
-/* How a pass runs on the device.
- *   STAGE_PASS_KERNELS (default): one kernel per step, all recorded in a CUDA
- *     graph, each a programmatic dependent of the one before.
- *   STAGE_PASS_PERSISTENT: one cooperative kernel runs the whole pass
- *     (stage input, then every layer's projections and mixer), its phases
- *     separated by grid-wide barriers, its CTAs streaming the next projection's
- *     weights across phase boundaries.  Used for n_tok 1..4 when two CTAs per
- *     SM are resident and the mixers' scratch fits (attention context of at
- *     most ~1700 chunks of 64 rows at n_tok 1); other passes fall back to
- *     kernels.  Slower than the kernels on B200 (per-step barriers and
- *     fix-up tails on the critical path); kept as an option.
- * Both run the same units with the same split and reduction order, so they
- * give bit-identical results.  Refused while a pass is pending; waits for the
- * stage's stream and drops the recorded graphs. */
-typedef enum { STAGE_PASS_KERNELS = 0, STAGE_PASS_PERSISTENT = 1 } stage_pass_mode;
-stage_status stage_set_pass_mode(stage_t* st, int mode);
-
-/* 1 if an n_tok-token pass would run as the persistent kernel, 0 if as a chain
- * of kernels, -1 for a NULL stage or n_tok outside 1..16. */
-int stage_pass_persistent(stage_t* st, int n_tok);
-
-/* Phase trace of the persistent pass (a profiling aid; off by default).
- * stage_set_trace(st, 1) makes every later persistent pass record, per CTA and
- * phase, the global-timer time (ns) at which the CTA's consumers started the
- * phase (past the grid barrier) and finished it; phase 0 is the stage input,
- * then per layer in-projection, mixer (attention: partials, combine),
- * out-projection, gate/up, down.  Toggling waits for the stream and drops the
- * recorded graphs; refused while a pass is pending.
- * stage_get_trace copies the last pass's record, u64 [grid][n_phases][2], to
- * host_dst (count = grid * n_phases * 2; host_dst NULL only reports the sizes
- * through grid / n_phases); STAGE_E_STATE if tracing is off. */
-stage_status stage_set_trace(stage_t* st, int enable);
-stage_status stage_get_trace(stage_t* st, unsigned long long* host_dst, size_t count, int* grid, int* n_phases);
+/* Failure injection for tests of the device-side error path (no counterpart
+ * on the pages; the stage's kernels bound every wait, and this makes one run
+ * out without faulting anything).  fault_item >= 0: in the next recorded
+ * passes, CTA 0 of the first layer's in-projection never requests the quants
+ * of its local item fault_item, so the wait for them runs out; -1 turns that
+ * off.  wait_limit: iteration cap of every bounded wait of the stage's GEMV
+ * kernels (0 = the default, seconds; a test passes a few thousand so the
+ * injected stall ends in milliseconds).  The pass then finishes with garbage
+ * in its outputs and stage_sync() returns STAGE_E_DEVICE (clearing the error
+ * word and the stream-K tile counters); stage_rollback() keeps the committed
+ * state intact, so the next pass is correct once injection is off again.
+ * Drops the recorded graphs; refused while a pass is pending. */
+stage_status stage_debug_inject(stage_t* st, int fault_item, unsigned wait_limit);
 
 /* Bytes of weight storage the stage streams per pass (packed quants + scales). */
 size_t stage_weight_bytes(const stage_t* st);
@@ -246,9 +263,9 @@ void stage_free(stage_t* st);
  * ------------------------------------------------------------------------- */
 
 /* Bytes of the packed (repacked) form of a GGUF matrix [rows, cols]:
- * ceil(rows/64) * cols/256 items of 9216 (Q4_0) or 17408 (Q8_0) bytes.
+ * ceil(rows/128) * cols/256 items of 18432 (Q4_0) or 34816 (Q8_0) bytes.
  * For a gate/up pair (paired != 0) rows is the number of features of each
- * matrix and the result holds both: ceil(rows/32) items per 256 columns.
+ * matrix and the result holds both: ceil(rows/64) items per 256 columns.
  * Returns 0 for an unsupported shape (cols % 256 != 0, rows <= 0). */
 size_t qhl_packed_bytes(int qtype, int rows, int cols, int paired);
 
@@ -271,7 +288,7 @@ int qhl_dequant(int qtype, int rows, int cols, const void* packed_dev, int paire
 /* y = x W^T for n_tok tokens (1..16): x_dev f32 [n_tok, cols], y_dev f32
  * [n_tok, rows], W packed (not paired).  Reduction order is fixed and
  * independent of n_tok (a batched call equals n_tok single calls bit for bit).
- * At most 2^31 - 1 packed items (ceil(rows/64) * cols/256), else STAGE_E_ARG.
+ * At most 2^31 - 1 packed items (ceil(rows/128) * cols/256), else STAGE_E_ARG.
  * Uses library-owned scratch (stream-K partials and tile counters, allocated
  * on first use per device and grown on demand); concurrent calls on different
  * streams of the same device must not overlap. */
@@ -295,12 +312,12 @@ int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float
  * synchronise the device).  The pages have no counterpart of this call; it
  * exists for such callers only.  Same arguments and results as qhl_qgemv (same
  * kernels, so the outputs are identical), but every piece of scratch lives in
- * one static device array of about 3.6 MiB that each GPU loading this library
+ * one static device array of about 4.8 MiB that each GPU loading this library
  * holds until the process exits; the call itself allocates nothing.  Limits:
- * n_tok * (cols / 256) * 864 bytes must not exceed 1 MiB (for example cols up to
- * 19200 at 16 tokens, 310528 at 1 token), rows at most 1048576, and the device
- * at most 160 SMs; larger problems return STAGE_E_ARG (STAGE_E_UNSUPPORTED for
- * the SM count) before any device work.  The first call on a device looks up
+ * n_tok * (cols / 256) * 2048 bytes must not exceed 2.25 MiB (for example cols
+ * up to 18432 at 16 tokens, 294912 at 1 token), rows at most 2097152, and the
+ * device at most 160 SMs; larger problems return STAGE_E_ARG
+ * (STAGE_E_UNSUPPORTED for the SM count) before any device work.  The first call on a device looks up
  * the array's device address and sets kernel attributes; make that first call
  * before any stream capture.  All calls share the one array, which keeps the
  * last call's contents (the tile counters are cleared by every call): calls
@@ -308,6 +325,20 @@ int qhl_deltanet_step(int Hk, int Hv, const float* y_dev, int n_tok, const float
  * must be serialised by the caller. */
 int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* packed_dev, const float* x_dev, int n_tok,
                       float* y_dev, void* stream);
+
+/* Wait for `stream`, then report and clear the device-side error word of the
+ * qhl_qgemv / qhl_qgemv_noalloc kernels on the current device: STAGE_E_DEVICE
+ * if one of their bounded waits ran out since the last qhl_sync (their output
+ * is then garbage; the tile counters are cleared with the word so that later
+ * calls are correct), 0 otherwise.  Allocates nothing. */
+int qhl_sync(void* stream);
+
+/* Failure injection for tests of that error path (no counterpart on the
+ * pages): later qhl_qgemv calls make CTA 0 skip the quants of its local item
+ * fault_item (-1: off) and cap every bounded wait at wait_limit iterations
+ * (0: the default), so one wait runs out without faulting anything.
+ * Process-wide; qhl_qgemv_noalloc is not affected. */
+int qhl_debug_inject(int fault_item, unsigned wait_limit);
 
 /* Message of the last failed qhl_* call on this host thread ("" if none). */
 const char* qhl_last_error(void);

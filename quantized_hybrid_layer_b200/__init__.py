@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(HERE, "libqhl_stage.so")
 STAGE_Q4_0 = 2
 STAGE_Q8_0 = 8
 MAX_TOK = 16
+PREFILL_EXACT, PREFILL_CHUNKED = 0, 1
 
 STATUS = {
     0: "STAGE_OK", -1: "STAGE_E_ARG", -2: "STAGE_E_STATE", -3: "STAGE_E_OOM", -4: "STAGE_E_CUDA",
@@ -30,17 +31,13 @@ STATUS = {
 
 #: every symbol include/qhl_stage.h declares
 EXPORTS = (
-    "stage_load", "stage_forward", "stage_forward_host", "stage_forward_f16", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
+    "stage_load", "stage_forward", "stage_forward_host", "stage_forward_f16", "stage_prefill", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
-    "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_set_pass_mode", "stage_pass_persistent",
-    "stage_set_trace", "stage_get_trace",
+    "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_debug_inject",
     "stage_weight_bytes", "stage_last_error",
     "stage_free", "qhl_packed_bytes", "qhl_repack", "qhl_dequant", "qhl_qgemv", "qhl_deltanet_step",
-    "qhl_qgemv_noalloc", "qhl_last_error",
+    "qhl_qgemv_noalloc", "qhl_sync", "qhl_debug_inject", "qhl_last_error",
 )
-
-
-PASS_KERNELS, PASS_PERSISTENT = 0, 1
 
 
 class StageError(RuntimeError):
@@ -81,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "stage_forward": (i, [vp, vp, i, i]),
             "stage_forward_f16": (i, [vp, vp, i, i]),
             "stage_forward_host": (i, [vp, vp, vp, i, i]),
+            "stage_prefill": (i, [vp, vp, i, i, i]),
             "stage_commit": (i, [vp, i]),
             "stage_rollback": (i, [vp]),
             "stage_reset": (i, [vp]),
@@ -93,10 +91,7 @@ def lib() -> ctypes.CDLL:
             "stage_set_kv": (i, [vp, i, vp, vp, sz]),
             "stage_set_kv_len": (i, [vp, i]),
             "stage_debug_dequant": (i, [vp, ctypes.c_char_p, i, vp, sz]),
-            "stage_set_pass_mode": (i, [vp, i]),
-            "stage_pass_persistent": (i, [vp, i]),
-            "stage_set_trace": (i, [vp, i]),
-            "stage_get_trace": (i, [vp, vp, sz, ctypes.POINTER(i), ctypes.POINTER(i)]),
+            "stage_debug_inject": (i, [vp, i, ctypes.c_uint]),
             "stage_weight_bytes": (sz, [vp]),
             "stage_last_error": (ctypes.c_char_p, [vp]),
             "stage_free": (None, [vp]),
@@ -106,6 +101,8 @@ def lib() -> ctypes.CDLL:
             "qhl_qgemv": (i, [i, i, i, vp, vp, i, vp, vp]),
             "qhl_deltanet_step": (i, [i, i, vp, i, vp, vp, vp, vp]),
             "qhl_qgemv_noalloc": (i, [i, i, i, vp, vp, i, vp, vp]),
+            "qhl_sync": (i, [vp]),
+            "qhl_debug_inject": (i, [i, ctypes.c_uint]),
             "qhl_last_error": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -205,14 +202,12 @@ class Stage:
             self.sync()
         return hidden_out
 
-    def forward_host(self, hidden_host, pos: int, dev_buf=None):
-        """End-to-end call from host memory: H2D copy, forward, D2H copy (on the stage stream)."""
-        import torch
-        buf = dev_buf if dev_buf is not None else torch.empty(hidden_host.shape, dtype=torch.float32, device="cuda")
-        buf.copy_(hidden_host, non_blocking=True)
-        self.forward(buf, pos)
-        hidden_host.copy_(buf, non_blocking=True)
-        return hidden_host
+    def prefill(self, hidden, pos: int, chunked: bool = False):
+        """Prompt chunk, committed in the same call (stage_prefill): the exact
+        token-by-token recurrence, or its chunked closed form."""
+        _check_hidden(hidden, "float32", self.cfg.hidden)
+        mode = PREFILL_CHUNKED if chunked else PREFILL_EXACT
+        self._check(lib().stage_prefill(self._h, _ptr(hidden), hidden.shape[0], pos, mode))
 
     def commit(self, n_accepted: int):
         self._check(lib().stage_commit(self._h, n_accepted))
@@ -234,26 +229,9 @@ class Stage:
     def pending(self) -> int:
         return lib().stage_pending(self._h)
 
-    def set_pass_mode(self, mode: int):
-        """PASS_KERNELS (one kernel per step, the default) or PASS_PERSISTENT
-        (one cooperative kernel per pass where eligible)."""
-        self._check(lib().stage_set_pass_mode(self._h, mode))
-
-    def pass_persistent(self, n_tok: int) -> bool:
-        """Whether an n_tok pass runs as the persistent kernel."""
-        return lib().stage_pass_persistent(self._h, n_tok) == 1
-
-    def set_trace(self, enable: bool):
-        """Record per-CTA phase times of later persistent passes."""
-        self._check(lib().stage_set_trace(self._h, 1 if enable else 0))
-
-    def get_trace(self) -> np.ndarray:
-        """The last persistent pass's record: u64 ns [grid, n_phases, 2] (start, end)."""
-        g, n = ctypes.c_int(0), ctypes.c_int(0)
-        self._check(lib().stage_get_trace(self._h, None, 0, ctypes.byref(g), ctypes.byref(n)))
-        out = np.zeros((g.value, n.value, 2), dtype=np.uint64)
-        self._check(lib().stage_get_trace(self._h, out.ctypes.data, out.size, ctypes.byref(g), ctypes.byref(n)))
-        return out
+    def debug_inject(self, fault_item: int = -1, wait_limit: int = 0):
+        """Failure injection for tests of the bounded waits (stage_debug_inject)."""
+        self._check(lib().stage_debug_inject(self._h, fault_item, wait_limit))
 
     @property
     def weight_bytes(self) -> int:
@@ -371,3 +349,14 @@ def qhl_qgemv_noalloc(qtype: int, rows: int, cols: int, packed, x, y, stream=Non
 def qhl_deltanet_step(Hk: int, Hv: int, y, s_in, snaps, o, stream=None):
     n = y.shape[0]
     _check_qhl(lib().qhl_deltanet_step(Hk, Hv, _ptr(y), n, _ptr(s_in), _ptr(snaps), _ptr(o), _stream(stream)))
+
+
+def qhl_sync(stream=None):
+    """Wait for the stream; raise StageError(STAGE_E_DEVICE) if a qhl_qgemv /
+    qhl_qgemv_noalloc kernel's bounded wait ran out since the last qhl_sync."""
+    _check_qhl(lib().qhl_sync(_stream(stream)))
+
+
+def qhl_debug_inject(fault_item: int = -1, wait_limit: int = 0):
+    """Failure injection for tests of the qhl_qgemv error path (qhl_debug_inject)."""
+    _check_qhl(lib().qhl_debug_inject(fault_item, wait_limit))

@@ -56,10 +56,15 @@ QHL_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The iteration cap of a wait: `limit`, or kWaitLimit when it is 0 (tests of
+// the error path pass a small cap so that an injected stall ends quickly).
+QHL_DEV uint32_t wait_limit(uint32_t limit) { return limit ? limit : kWaitLimit; }
+
 // Wait for the phase with the given parity to complete; false (and an error
-// bit) if it did not within kWaitLimit tries.
-QHL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
+// bit) if it did not within wait_limit(limit) tries.
+QHL_DEV bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err, uint32_t limit = 0) {
+  const uint32_t n = wait_limit(limit);
+  for (uint32_t i = 0; i < n; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   if (err) atomicOr(err, ERR_WAIT_TIMEOUT);
   return false;
@@ -140,6 +145,20 @@ QHL_DEV void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" :::
 QHL_DEV void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Named barrier that also ANDs a predicate over the participating threads:
+// every thread gets the same answer.
+QHL_DEV bool bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 
 // ---- warp reductions: xor butterflies give every lane the same bits --------
 QHL_DEV float warp_sum(float v) {
@@ -151,16 +170,6 @@ QHL_DEV float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
-}
-
-// Sum of squares of 64 values in row order; the one definition used for the
-// per-tile RMSNorm partials everywhere, so a stage's result never depends on
-// which kernel produced its input.
-QHL_DEV float sumsq64(const float* v) {
-  float s = 0.f;
-#pragma unroll 8
-  for (int r = 0; r < 64; ++r) s = __fmaf_rn(v[r], v[r], s);
-  return s;
 }
 
 // 1 / sqrt(mean + eps) from per-tile partial sums, computed by one warp: lane

@@ -42,7 +42,19 @@ struct DnArgs {
   int o_stride;
   uint8_t* qo;             // optional output in block fixed point (the out-projection's input)
   int qo_stride;
+  int mode;                // DN_SNAPSHOTS, DN_FINAL or DN_CHUNKED
 };
+
+// What a pass keeps of the recurrent state:
+//   DN_SNAPSHOTS  the state after every token (a verify pass: any prefix can
+//                 be committed),
+//   DN_FINAL      the state after the last token only, the same sequential
+//                 arithmetic (a prefill chunk, committed whole: bit-identical
+//                 to DN_SNAPSHOTS followed by commit of every token),
+//   DN_CHUNKED    the state after the last token by the chunked closed form of
+//                 the recurrence (a prefill chunk; not bit-identical to the
+//                 token-by-token steps, within rounding of them).
+enum DnMode : int { DN_SNAPSHOTS = 0, DN_FINAL = 1, DN_CHUNKED = 2 };
 
 QHL_DEV float dot4(float4 a, float4 b) {
   float s = __fmul_rn(a.x, b.x);
@@ -66,8 +78,10 @@ QHL_DEV void dn_load(const DnArgs& a, int unit, float4 (&S)[4]) {
 }
 
 // Shared memory of one unit (floats): outputs ob [NT][32], then the unit's
-// inputs staged once for all tokens: q, k [NT][128] each, v [NT][32], b, a [NT].
-constexpr int dn_smem_floats(int nt) { return nt * (32 + 2 * kDnDim + 32 + 2); }
+// inputs staged once for all tokens: q, k [NT][128] each, v [NT][32], b, a
+// [NT]; then, for the chunked form, c, e^c, e^(c_n - c) [NT] and two [NT][NT]
+// coefficient matrices.
+constexpr int dn_smem_floats(int nt) { return nt * (32 + 2 * kDnDim + 32 + 2) + 3 * nt + 2 * nt * nt; }
 
 template <int NT>
 QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
@@ -120,6 +134,7 @@ QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
     const float alpha = sigmoidf_(-aa);    // exp(-softplus(a)) = sigmoid(-a)
     float* dst = a.cur ? a.ring + (size_t)((cur + 1 + t) % a.ring_size) * a.state_elems
                        : a.ring + (size_t)t * a.state_elems;
+    const bool keep = a.mode == DN_SNAPSHOTS || t == NT - 1;   // DN_FINAL: the last state only
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const float kS = warp_sum(dot4(S[r], k));
@@ -133,7 +148,7 @@ QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
         ob[t][warp * 4 + r] = o;
         if (a.o) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
       }
-      reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = S[r];
+      if (keep) reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = S[r];
     }
   }
   named_sync(1, 256);
@@ -141,6 +156,141 @@ QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
     for (int t = warp; t < NT; t += 8)
       qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (unit & 3), lane);
   named_sync(1, 256);   // sm reusable by the caller
+}
+
+// Chunked form of the same recurrence for a prefill chunk whose tokens are
+// committed together (only the final state is kept).  With c_t = sum over
+// m <= t of log alpha_m and u_t = beta_t (v_t - alpha_t S_{t-1} k_t), the state
+// after token t is
+//     S_t = e^{c_t} S_0 + sum_{j <= t} e^{c_t - c_j} u_j k_j^T,
+// so each value row i needs only dot products against the starting state:
+//     u_t[i] = beta_t (v_t[i] - e^{c_t} (S_0 k_t)[i] - sum_{j < t} e^{c_t - c_j} (k_j . k_t) u_j[i])
+//     o_t[i] = e^{c_t} (S_0 q_t)[i] + sum_{j <= t} e^{c_t - c_j} (q_t . k_j) u_j[i]
+//     S_n[i] = e^{c_n} S_0[i] + sum_j e^{c_n - c_j} u_j[i] k_j
+// (a unit lower-triangular solve per row).  The 2 NT dot products against S_0
+// are independent of one another -- no chain of token steps -- and the state is
+// read once and written once.  Ratios of the decays are formed as exp of
+// differences of c, which is never above 0, so nothing overflows.
+template <int NT>
+QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = unit >> 2;
+  const int row0 = (unit & 3) * 32 + warp * 4;
+  const int g = h / (a.Hv / a.Hk);
+  const int cur = a.cur ? *a.cur : 0;
+  float (*ob)[32] = reinterpret_cast<float (*)[32]>(sm);
+  float* sq = sm + NT * 32;
+  float* sk = sq + NT * kDnDim;
+  float* sv = sk + NT * kDnDim;
+  float* sb = sv + NT * 32;
+  float* sa = sb + NT;
+  float* cl = sa + NT;            // c_t
+  float* eg = cl + NT;            // e^{c_t}
+  float* ef = eg + NT;            // e^{c_{n-1} - c_t}
+  float* Lm = ef + NT;            // [t][j]: e^{c_t - c_j} k_j . k_t, j < t
+  float* Pm = Lm + NT * NT;       // [t][j]: e^{c_t - c_j} q_t . k_j, j <= t
+
+  const int off_k = a.Hk * kDnDim;
+  const int off_v = 2 * a.Hk * kDnDim;
+  const int off_b = off_v + a.Hv * kDnDim;
+  const int off_a = off_b + a.Hv;
+  for (int i = tid; i < NT * 64; i += 256) {
+    const int t = i >> 6, q4 = i & 63;
+    const float* yt = a.y + (size_t)t * a.y_stride;
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(yt + (q4 < 32 ? 0 : off_k) + g * kDnDim) + (q4 & 31));
+    reinterpret_cast<float4*>(q4 < 32 ? sq + t * kDnDim : sk + t * kDnDim)[q4 & 31] = v;
+  }
+  for (int i = tid; i < NT * 32; i += 256) {
+    const int t = i >> 5, r = i & 31;
+    sv[i] = __ldcg(a.y + (size_t)t * a.y_stride + off_v + h * kDnDim + (unit & 3) * 32 + r);
+  }
+  if (tid < NT) {
+    sb[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_b + h);
+    sa[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_a + h);
+  }
+  named_sync(1, 256);
+  // q, k normalised in place (warp w: tokens w, w + 8); decays by thread 0
+  for (int t = warp; t < NT; t += 8) {
+    float4 q = reinterpret_cast<const float4*>(sq + t * kDnDim)[lane];
+    float4 k = reinterpret_cast<const float4*>(sk + t * kDnDim)[lane];
+    const float rq = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(q, q)), 1e-6f)));
+    const float rk = __frcp_rn(__fsqrt_rn(__fadd_rn(warp_sum(dot4(k, k)), 1e-6f)));
+    reinterpret_cast<float4*>(sq + t * kDnDim)[lane] =
+        make_float4(__fmul_rn(q.x, rq), __fmul_rn(q.y, rq), __fmul_rn(q.z, rq), __fmul_rn(q.w, rq));
+    reinterpret_cast<float4*>(sk + t * kDnDim)[lane] =
+        make_float4(__fmul_rn(k.x, rk), __fmul_rn(k.y, rk), __fmul_rn(k.z, rk), __fmul_rn(k.w, rk));
+  }
+  if (tid == 0) {
+    float c = 0.f;
+    for (int t = 0; t < NT; ++t) {
+      const float x = sa[t];   // log alpha = -softplus(a), computed without overflow
+      const float sp = x > 0.f ? __fadd_rn(x, log1pf(expf(-x))) : log1pf(expf(x));
+      c = __fsub_rn(c, sp);
+      cl[t] = c;
+      eg[t] = expf(c);
+      sb[t] = sigmoidf_(sb[t]);   // beta
+    }
+    for (int t = 0; t < NT; ++t) ef[t] = expf(__fsub_rn(cl[NT - 1], cl[t]));
+  }
+  named_sync(1, 256);
+  for (int p = warp; p < NT * NT; p += 8) {
+    const int t = p / NT, j = p % NT;
+    const float4 kj = reinterpret_cast<const float4*>(sk + j * kDnDim)[lane];
+    const float kk = warp_sum(dot4(kj, reinterpret_cast<const float4*>(sk + t * kDnDim)[lane]));
+    const float qk = warp_sum(dot4(kj, reinterpret_cast<const float4*>(sq + t * kDnDim)[lane]));
+    if (lane == 0) {
+      const float e = j <= t ? expf(__fsub_rn(cl[t], cl[j])) : 0.f;
+      Lm[p] = j < t ? __fmul_rn(e, kk) : 0.f;
+      Pm[p] = __fmul_rn(e, qk);
+    }
+  }
+  named_sync(1, 256);
+
+  float* dst = a.cur ? a.ring + (size_t)((cur + NT) % a.ring_size) * a.state_elems
+                     : a.ring + (size_t)(NT - 1) * a.state_elems;
+#pragma unroll 1
+  for (int r = 0; r < 4; ++r) {
+    float A[NT], B[NT], u[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      A[t] = warp_sum(dot4(S[r], reinterpret_cast<const float4*>(sk + t * kDnDim)[lane]));
+      B[t] = warp_sum(dot4(S[r], reinterpret_cast<const float4*>(sq + t * kDnDim)[lane]));
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float x = __fsub_rn(sv[t * 32 + warp * 4 + r], __fmul_rn(eg[t], A[t]));
+#pragma unroll
+      for (int j = 0; j < t; ++j) x = __fsub_rn(x, __fmul_rn(Lm[t * NT + j], u[j]));
+      u[t] = __fmul_rn(sb[t], x);
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float o = __fmul_rn(eg[t], B[t]);
+#pragma unroll
+      for (int j = 0; j <= t; ++j) o = __fmaf_rn(Pm[t * NT + j], u[j], o);
+      if (lane == 0) {
+        ob[t][warp * 4 + r] = o;
+        if (a.o) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
+      }
+    }
+    const float e = eg[NT - 1];
+    float4 sn = make_float4(__fmul_rn(e, S[r].x), __fmul_rn(e, S[r].y), __fmul_rn(e, S[r].z), __fmul_rn(e, S[r].w));
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const float w = __fmul_rn(ef[j], u[j]);
+      const float4 kj = reinterpret_cast<const float4*>(sk + j * kDnDim)[lane];
+      sn.x = __fmaf_rn(w, kj.x, sn.x);
+      sn.y = __fmaf_rn(w, kj.y, sn.y);
+      sn.z = __fmaf_rn(w, kj.z, sn.z);
+      sn.w = __fmaf_rn(w, kj.w, sn.w);
+    }
+    reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = sn;
+  }
+  named_sync(1, 256);
+  if (a.qo)
+    for (int t = warp; t < NT; t += 8)
+      qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (unit & 3), lane);
+  named_sync(1, 256);
 }
 
 template <int NT>
@@ -157,7 +307,10 @@ __global__ void __launch_bounds__(256) dn_step_kernel(const DnArgs a) {
   float4 S[4];
   dn_load<NT>(a, blockIdx.x, S);   // overlaps the in-projection's last tiles
   pdl_wait();                      // q, k, v, b, a come from it
-  dn_run<NT>(a, blockIdx.x, S, sm);
+  if (a.mode == DN_CHUNKED)
+    dn_run_chunked<NT>(a, blockIdx.x, S, sm);
+  else
+    dn_run<NT>(a, blockIdx.x, S, sm);
 }
 
 }  // namespace qhl

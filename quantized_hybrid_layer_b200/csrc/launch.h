@@ -10,7 +10,6 @@
 #include "attention.cuh"
 #include "deltanet.cuh"
 #include "input.cuh"
-#include "pass.cuh"
 #include "qgemv.cuh"
 
 namespace qhl {
@@ -57,24 +56,10 @@ cudaError_t launch_rope_table(float2* tab, int max_ctx, int rope_dims, double th
 cudaError_t launch_commit(int* ctrl, int n_accepted, int n_dn, int ring, cudaStream_t s);
 cudaError_t launch_set_int(int* p, int v, cudaStream_t s);
 
-// Persistent pass (pass.cuh), instantiated in pass_q4.cu / pass_q8.cu.
-extern template struct PassOps<kQ4_0>;
-extern template struct PassOps<kQ8_0>;
-inline cudaError_t pass_prepare(int qt) { return qt == kQ4_0 ? PassOps<kQ4_0>::prepare() : PassOps<kQ8_0>::prepare(); }
-inline cudaError_t pass_occupancy(int qt, int nt, int* blocks) {
-  return qt == kQ4_0 ? PassOps<kQ4_0>::occupancy(nt, blocks) : PassOps<kQ8_0>::occupancy(nt, blocks);
-}
-inline int pass_mix_bytes(int qt, int nt) {
-  return qt == kQ4_0 ? PassOps<kQ4_0>::mix_bytes(nt) : PassOps<kQ8_0>::mix_bytes(nt);
-}
-inline cudaError_t launch_pass(int qt, int nt, const PassArgs& p, cudaStream_t s) {
-  return qt == kQ4_0 ? PassOps<kQ4_0>::launch(nt, p, s) : PassOps<kQ8_0>::launch(nt, p, s);
-}
-
-// CTAs that own items of a tiles x chunks GEMV on `cap` co-resident CTAs.
+// CTAs that own items of a tiles x chunks GEMV on `cap` CTAs (one per SM).
 // When the CTAs can own whole tiles -- a divisor of `tiles` no smaller than
 // 85% of `cap` -- no tile is split and no stream-K fix-up runs (the gate/up
-// projection of the 27B shape: 544 tiles on 272 of 296 CTAs); otherwise a
+// projection of the 27B shape: 272 tiles on 136 of 148 CTAs); otherwise a
 // balanced stream-K split over min(cap, items) CTAs.  Depends on the shape
 // and `cap` only, never on the token count.
 inline int gemv_workers(int tiles, int chunks, int cap) {
@@ -86,7 +71,7 @@ inline int gemv_workers(int tiles, int chunks, int cap) {
 }
 
 // packed-layout geometry
-inline int packed_tiles(int rows, bool paired) { return paired ? (rows + 31) / 32 : (rows + 63) / 64; }
+inline int packed_tiles(int rows, bool paired) { return paired ? (rows + 63) / 64 : (rows + kTileRows - 1) / kTileRows; }
 inline size_t packed_bytes(int qt, int rows, int cols, bool paired) {
   if (rows <= 0 || cols <= 0 || cols % kChunkCols || (qt != kQ4_0 && qt != kQ8_0)) return 0;
   return (size_t)packed_tiles(rows, paired) * (cols / kChunkCols) * item_bytes(qt);

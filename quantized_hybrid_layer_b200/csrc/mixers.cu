@@ -7,34 +7,18 @@
 
 namespace qhl {
 
-cudaError_t gemv_prepare_4();
-cudaError_t gemv_prepare_8();
-cudaError_t launch_gemv_4(int nt, int epi, const GemvArgs& a, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_gemv_8(int nt, int epi, const GemvArgs& a, int grid, cudaStream_t s, bool pdl);
-int gemv_smem_4(int nt);
-int gemv_smem_8(int nt);
-
-cudaError_t gemv_prepare(int qt) { return qt == kQ4_0 ? gemv_prepare_4() : gemv_prepare_8(); }
-cudaError_t launch_gemv(int qt, int nt, int epi, const GemvArgs& a, int grid, cudaStream_t s, bool pdl) {
-  if (qt == kQ4_0) return launch_gemv_4(nt, epi, a, grid, s, pdl);
-  if (qt == kQ8_0) return launch_gemv_8(nt, epi, a, grid, s, pdl);
-  return cudaErrorInvalidValue;
-}
-int gemv_smem(int qt, int nt) { return qt == kQ4_0 ? gemv_smem_4(nt) : gemv_smem_8(nt); }
-
 #define QHL_NT_CASES(X) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
 
 // ---------------------------------------------------------------------------
 // stage input: z = h * gamma (the first layer's RMSNorm weight) in block fixed
 // point and per-tile sums of squares of h, exactly as the residual epilogue of
-// the GEMV writes them, so a stage that starts at layer L gives the same bits
-// as the same layers inside a longer stage.
+// the GEMV writes them (input.cuh), one 128-row tile per CTA of 128 threads.
 template <int NT>
-__global__ void __launch_bounds__(256) stage_input_kernel(const float* h, int H, const float* gamma, uint8_t* qz,
+__global__ void __launch_bounds__(128) stage_input_kernel(const float* h, int H, const float* gamma, uint8_t* qz,
                                                           int qz_stride, float* ss, int ss_stride) {
-  __shared__ float sm[NT * 64];
+  __shared__ float red[4];
   if (threadIdx.x == 0) pdl_launch();
-  input_unit<NT>(h, H, gamma, qz, qz_stride, ss, ss_stride, blockIdx.x, sm);
+  input_unit<NT>(h, H, gamma, qz, qz_stride, ss, ss_stride, blockIdx.x, red, 1);
 }
 
 // f32 rows -> block fixed point, one warp per (token, 32-column block).  The
@@ -138,7 +122,7 @@ cudaError_t launch_attn_combine(int nt, const AttnArgs& a, cudaStream_t s, bool 
 cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma, uint8_t* qz, int qz_stride,
                                float* ss, int ss_stride, cudaStream_t s) {
   switch (nt) {
-#define C(N) case N: return launch_ex(stage_input_kernel<N>, dim3(H / 64), dim3(256), 0, s, false, h, H, gamma, qz, qz_stride, ss, ss_stride);
+#define C(N) case N: return launch_ex(stage_input_kernel<N>, dim3(H / kTileRows), dim3(128), 0, s, false, h, H, gamma, qz, qz_stride, ss, ss_stride);
     QHL_NT_CASES(C)
 #undef C
     default: return cudaErrorInvalidValue;
@@ -147,24 +131,24 @@ cudaError_t launch_stage_input(int nt, const float* h, int H, const float* gamma
 
 // ---------------------------------------------------------------------------
 // GGUF array-of-structs blocks -> packed items (layout in qpack.cuh).
-// One thread per (item, block, tile row).  Rows past the matrix are filled
-// with zero weights.  paired: tile rows 0..31 come from a (features t*32..),
-// rows 32..63 from b (the same features), for the SwiGLU epilogue.
+// One thread per (item, block, tile row).  Rows past the matrix get zero
+// weights (Q4_0 nibbles 8, Q8_0 bytes 0, scale 0).  paired: tile rows 0..63
+// come from a (features 64 t ..), rows 64..127 from b (the same features), for
+// the SwiGLU epilogue.
 __global__ void repack_kernel(int qt, const uint8_t* a, const uint8_t* b, int rows, int paired, int tiles,
                               int chunks, uint8_t* out) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)tiles * chunks * 512) return;
-  const long long item = idx / 512;
-  const int rem = (int)(idx % 512), blk = rem / 64, r = rem % 64;
+  if (idx >= (long long)tiles * chunks * (kChunkBlocks * kTileRows)) return;
+  const long long item = idx / (kChunkBlocks * kTileRows);
+  const int rem = (int)(idx % (kChunkBlocks * kTileRows)), blk = rem / kTileRows, r = rem % kTileRows;
   const int t = (int)(item / chunks), c = (int)(item % chunks);
-  const int h = r / 32, lane = r % 32;
   const uint8_t* src = a;
   int srow;
   if (paired) {
-    srow = t * 32 + lane;
-    src = h ? b : a;
+    srow = t * 64 + (r & 63);
+    src = r >= 64 ? b : a;
   } else {
-    srow = t * 64 + r;
+    srow = t * kTileRows + r;
   }
   const bool valid = srow < rows;
   const int bb = gguf_block_bytes(qt);
@@ -172,87 +156,65 @@ __global__ void repack_kernel(int qt, const uint8_t* a, const uint8_t* b, int ro
   const uint8_t* sp = src + (valid ? ((long long)srow * nb + (long long)c * kChunkBlocks + blk) * bb : 0);
   uint8_t* base = out + item * item_bytes(qt);
   if (qt == kQ4_0) {
-    uint8_t* q = base + ((blk * 2 + h) * 32 + lane) * 16;
+    uint8_t* q = base + q4_off(blk, r);
     for (int i = 0; i < 16; ++i) q[i] = valid ? sp[2 + i] : 0x88;
-    uint8_t* s = base + 8192 + (blk * 32 + lane) * 4 + h * 2;
-    s[0] = valid ? sp[0] : 0;
-    s[1] = valid ? sp[1] : 0;
   } else {
-    for (int half = 0; half < 2; ++half) {
-      uint8_t* q = base + (((blk * 2 + half) * 2 + h) * 32 + lane) * 16;
-      for (int i = 0; i < 16; ++i) q[i] = valid ? sp[2 + 16 * half + i] : 0;
+    for (int h = 0; h < 2; ++h) {
+      uint8_t* q = base + q8_off(blk, h, r);
+      for (int i = 0; i < 16; ++i) q[i] = valid ? sp[2 + 16 * h + i] : 0;
     }
-    uint8_t* s = base + 16384 + (blk * 32 + lane) * 4 + h * 2;
-    s[0] = valid ? sp[0] : 0;
-    s[1] = valid ? sp[1] : 0;
   }
+  uint8_t* sc = base + scale_off(qt, blk, r);
+  sc[0] = valid ? sp[0] : 0;
+  sc[1] = valid ? sp[1] : 0;
 }
 
 cudaError_t launch_repack(int qt, const uint8_t* a, const uint8_t* b, int rows, int cols, uint8_t* out,
                           cudaStream_t s) {
   const bool paired = b != nullptr;
   const int tiles = packed_tiles(rows, paired), chunks = cols / kChunkCols;
-  const long long n = (long long)tiles * chunks * 512;
+  const long long n = (long long)tiles * chunks * (kChunkBlocks * kTileRows);
   repack_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(qt, a, b, rows, paired ? 1 : 0, tiles, chunks, out);
   return cudaGetLastError();
 }
 
-// Dequantise rows of a packed matrix with the GEMV's conversion (q4_word /
-// q8_word) times the f16 scale: one thread per (row, block).
+// Dequantise rows of a packed matrix: the GEMV's own operand preparation (the
+// 8-bit A bytes q4_unpack / the Q8_0 bytes give the MMA) times the f16 scale,
+// one thread per (row, block).
 __global__ void dequant_kernel(int qt, const uint8_t* P, int rows, int cols, int paired, int row0, int nrows,
                                float* out) {
   const int nb = cols / 32;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)nrows * nb) return;
   const int r = row0 + (int)(idx / nb), kb = (int)(idx % nb);
-  int tile, h, lane;
+  int tile, tr;
   if (paired) {
     const int f = r % rows;
-    h = r / rows;
-    tile = f / 32;
-    lane = f % 32;
+    tile = f / 64;
+    tr = (r / rows) * 64 + f % 64;
   } else {
-    tile = r / 64;
-    h = (r % 64) / 32;
-    lane = r % 32;
+    tile = r / kTileRows;
+    tr = r % kTileRows;
   }
   const int chunks = cols / kChunkCols, c = kb / kChunkBlocks, blk = kb % kChunkBlocks;
   const uint8_t* base = P + ((size_t)tile * chunks + c) * item_bytes(qt);
-  const int qb = qt == kQ4_0 ? 8192 : 16384;
-  const uint16_t sbits = *reinterpret_cast<const uint16_t*>(base + qb + (blk * 32 + lane) * 4 + h * 2);
+  const uint16_t sbits = *reinterpret_cast<const uint16_t*>(base + scale_off(qt, blk, tr));
   const float d = __half2float(__ushort_as_half(sbits));
-  float w[32];
+  uint32_t av[8];
   if (qt == kQ4_0) {
-    const uint4 wv = *reinterpret_cast<const uint4*>(base + ((blk * 2 + h) * 32 + lane) * 16);
-    const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
-    for (int i = 0; i < 4; ++i) {
-      float2 p[4];
-      q4_word(ws[i], p);
-      w[4 * i] = p[0].x;
-      w[4 * i + 1] = p[0].y;
-      w[4 * i + 2] = p[1].x;
-      w[4 * i + 3] = p[1].y;
-      w[16 + 4 * i] = p[2].x;
-      w[17 + 4 * i] = p[2].y;
-      w[18 + 4 * i] = p[3].x;
-      w[19 + 4 * i] = p[3].y;
-    }
+    q4_unpack(*reinterpret_cast<const uint4*>(base + q4_off(blk, tr)), av);
   } else {
-    for (int half = 0; half < 2; ++half) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(base + (((blk * 2 + half) * 2 + h) * 32 + lane) * 16);
-      const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
-      for (int i = 0; i < 4; ++i) {
-        float2 p[2];
-        q8_word(ws[i], p);
-        w[16 * half + 4 * i] = p[0].x;
-        w[16 * half + 4 * i + 1] = p[0].y;
-        w[16 * half + 4 * i + 2] = p[1].x;
-        w[16 * half + 4 * i + 3] = p[1].y;
-      }
-    }
+    const uint4 w0 = *reinterpret_cast<const uint4*>(base + q8_off(blk, 0, tr));
+    const uint4 w1 = *reinterpret_cast<const uint4*>(base + q8_off(blk, 1, tr));
+    av[0] = w0.x; av[1] = w0.y; av[2] = w0.z; av[3] = w0.w;
+    av[4] = w1.x; av[5] = w1.y; av[6] = w1.z; av[7] = w1.w;
   }
   float* o = out + (size_t)(r - row0) * cols + kb * 32;
-  for (int e = 0; e < 32; ++e) o[e] = __fmul_rn(w[e], d);
+  for (int e = 0; e < 32; ++e) {
+    const uint32_t byte = (av[e >> 2] >> (8 * (e & 3))) & 0xFFu;
+    const int q = qt == kQ4_0 ? (int)byte - 8 : (int)(int8_t)byte;
+    o[e] = __fmul_rn((float)q, d);
+  }
 }
 
 cudaError_t launch_dequant(int qt, const uint8_t* packed, int rows, int cols, int paired, int row0, int nrows,

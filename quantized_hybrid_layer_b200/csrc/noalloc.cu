@@ -14,6 +14,7 @@
 // qhl_stage.h); larger ones are rejected before any device work.
 #include <cuda_runtime.h>
 
+#include <deque>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -30,9 +31,9 @@ void set_last_error(const std::string& s);   // kernel_abi.cu
 namespace {
 
 // Regions of the scratch array (bytes).
-constexpr size_t kPartialBytes = (size_t)5 << 19;   // 2.5 MiB: 2 * kCtasPerSm * SMs * 16 tokens * 64 rows f32
-constexpr size_t kCounterBytes = (size_t)64 << 10;  // 64 KiB: one int per 64-row tile (16384 tiles)
-constexpr size_t kQxBytes = (size_t)1 << 20;        // 1 MiB: the input in block fixed point
+constexpr size_t kPartialBytes = (size_t)5 << 19;     // 2.5 MiB: 2 * SMs * 16 tokens * 128 rows f32, SMs <= 160
+constexpr size_t kCounterBytes = (size_t)64 << 10;    // 64 KiB: one int per 128-row tile (16384 tiles)
+constexpr size_t kQxBytes = (size_t)9 << 18;          // 2.25 MiB: the input in block fixed point
 constexpr size_t kErrBytes = 256;
 constexpr size_t kScratchBytes = kPartialBytes + kCounterBytes + kQxBytes + kErrBytes;
 
@@ -45,8 +46,10 @@ struct DeviceScratch {
   bool prepared[9] = {};
 };
 
+// Entries live in a deque: references to one stay valid while another host
+// thread adds a device.  Callers still copy what they need under the lock.
 std::mutex g_mu;
-std::vector<DeviceScratch> g_dev;
+std::deque<DeviceScratch> g_dev;
 
 int fail(int code, const std::string& msg) {
   set_last_error("qhl_qgemv_noalloc: " + msg);
@@ -67,44 +70,47 @@ extern "C" int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* pack
   const int tiles = packed_tiles(rows, false);
   const size_t qx_bytes = (size_t)n_tok * qact_row_bytes(cols);
   if (qx_bytes > kQxBytes)
-    return fail(STAGE_E_ARG, "n_tok * cols/256 * 864 = " + std::to_string(qx_bytes) + " bytes exceeds the " +
+    return fail(STAGE_E_ARG, "n_tok * cols/256 * 2048 = " + std::to_string(qx_bytes) + " bytes exceeds the " +
                                  std::to_string(kQxBytes) + "-byte input region of the static scratch");
   if ((size_t)tiles * sizeof(int) > kCounterBytes)
     return fail(STAGE_E_ARG, "rows exceed the static scratch's tile counters (at most " +
-                                 std::to_string(kCounterBytes / sizeof(int) * 64) + " rows)");
+                                 std::to_string(kCounterBytes / sizeof(int) * kTileRows) + " rows)");
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(STAGE_E_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-  DeviceScratch* ds = nullptr;
+  unsigned char* base = nullptr;
+  int sms = 0;
   {
     // once per device, with that device current: the scratch array's device
     // address (a host-side use of g_scratch would be a host stand-in, not it)
     std::lock_guard<std::mutex> lk(g_mu);
     if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
-    ds = &g_dev[dev];
-    if (!ds->ready) {
+    DeviceScratch& ds = g_dev[dev];
+    if (!ds.ready) {
       void* p = nullptr;
       if ((e = cudaGetSymbolAddress(&p, g_scratch)) != cudaSuccess)
         return fail(STAGE_E_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-      if ((e = cudaDeviceGetAttribute(&ds->sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      if ((e = cudaDeviceGetAttribute(&ds.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return fail(STAGE_E_CUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
-      ds->base = static_cast<unsigned char*>(p);
-      ds->ready = true;
+      ds.base = static_cast<unsigned char*>(p);
+      ds.ready = true;
     }
-    if (!ds->prepared[qtype]) {
+    if (!ds.prepared[qtype]) {
       if ((e = gemv_prepare(qtype)) != cudaSuccess)
         return fail(STAGE_E_CUDA, std::string("gemv_prepare: ") + cudaGetErrorString(e));
-      ds->prepared[qtype] = true;
+      ds.prepared[qtype] = true;
     }
+    base = ds.base;
+    sms = ds.sms;
   }
-  if ((size_t)2 * kCtasPerSm * ds->sms * 16 * 64 * sizeof(float) > kPartialBytes)
+  if ((size_t)2 * sms * 16 * kTileRows * sizeof(float) > kPartialBytes)
     return fail(STAGE_E_UNSUPPORTED, "this device has more SMs than the static stream-K region holds");
 
-  float* partials = reinterpret_cast<float*>(ds->base);
-  int* counters = reinterpret_cast<int*>(ds->base + kPartialBytes);
-  uint8_t* qx = ds->base + kPartialBytes + kCounterBytes;
-  unsigned* err = reinterpret_cast<unsigned*>(ds->base + kPartialBytes + kCounterBytes + kQxBytes);
+  float* partials = reinterpret_cast<float*>(base);
+  int* counters = reinterpret_cast<int*>(base + kPartialBytes);
+  uint8_t* qx = base + kPartialBytes + kCounterBytes;
+  unsigned* err = reinterpret_cast<unsigned*>(base + kPartialBytes + kCounterBytes + kQxBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   // the array keeps the previous call's contents: the tile counters must start at zero
@@ -125,8 +131,30 @@ extern "C" int qhl_qgemv_noalloc(int qtype, int rows, int cols, const void* pack
   a.partials = partials;
   a.counters = counters;
   a.err = err;
-  a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * ds->sms);
+  a.workers = gemv_workers(a.tiles, a.chunks, sms);
+  a.fault_item = -1;
   if ((e = launch_gemv(qtype, n_tok, EPI_STORE, a, a.workers, s, true)) != cudaSuccess)
     return fail(STAGE_E_CUDA, std::string("qgemv launch: ") + cudaGetErrorString(e));
   return 0;
 }
+
+namespace qhl {
+// The static scratch's error word on device `dev` (current), read and cleared
+// with the tile counters; 0 if the array was never used there.  For qhl_sync.
+unsigned noalloc_take_error(int dev) {
+  unsigned char* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((int)g_dev.size() > dev && g_dev[dev].ready) base = g_dev[dev].base;
+  }
+  if (!base) return 0;
+  unsigned* err = reinterpret_cast<unsigned*>(base + kPartialBytes + kCounterBytes + kQxBytes);
+  unsigned w = 0;
+  if (cudaMemcpy(&w, err, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return 0;
+  if (w) {
+    cudaMemset(err, 0, sizeof(w));
+    cudaMemset(base + kPartialBytes, 0, kCounterBytes);
+  }
+  return w;
+}
+}  // namespace qhl

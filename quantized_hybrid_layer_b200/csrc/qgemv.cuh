@@ -1,46 +1,46 @@
-// Fused dequant-GEMV / skinny GEMM over packed Q4_0 / Q8_0 weights.
+// Fused dequant-GEMV / skinny GEMM over packed Q4_0 / Q8_0 weights on the
+// fifth-generation tensor cores.
 //
 // y[t][r] = sum_c x[t][c] * W[r][c] for n_tok = NT tokens (1..16), the
 // projection every layer of the stage streams: one decoded token streams the
 // whole weight set a single time (SwarmLLM README, paragraph after the peer
-// diagram).  Decode is
-// memory-bound, so the kernel is built to keep HBM busy and the SM's integer
-// and FP pipes well below their limits:
+// diagram).  Decode is memory-bound, so the kernel is built to keep HBM busy
+// with as little SM work per weight byte as possible:
 //
-//  * Persistent stream-K grid, two CTAs per SM.  The (tile, chunk) items of the
-//    packed matrix are split into contiguous equal ranges, one per CTA, so every
-//    SM streams the same number of bytes whatever the matrix shape.
-//  * One producer warp per CTA moves items (64 rows x 256 columns, one
-//    contiguous record) and the matching x columns into a ring of shared-memory
-//    stages with bulk async copies (cp.async.bulk + mbarrier, L2 evict-first for
-//    weights).  The weights never depend on the previous kernel, so the first
-//    stages are requested before griddepcontrol.wait: under programmatic
-//    dependent launch a projection's weights stream in while the previous
-//    kernel drains.
-//  * Eight consumer warps; warp w handles block w of each item.  Lane l owns
-//    tile rows l and l + 32, so x is read as warp-uniform broadcasts and no
-//    cross-lane reduction is needed.  x arrives in block fixed-point form
-//    (qact.cuh): each block's sum_j q_j X_j is formed exactly in int32 with
-//    byte dot products (dp4a) against the 4-bit (or 8-bit) quants -- from 4
-//    tokens up by integer tensor-core mma instead, with the same exact sums --
-//    and one FMA per block adds d * s * sum to the row's f32 accumulator.
-//  * A tenth warp finishes tiles (sums the consumer warps' partials, stream-K
-//    fix-up, epilogue) while the consumers stream on; once its own items are
-//    issued the producer warms L2 with the pass's next projection.
+//  * Persistent stream-K grid of one CTA per SM.  The (tile, chunk) items of
+//    the packed matrix (128 rows x 256 columns, qpack.cuh) are split into
+//    contiguous equal ranges, one per CTA.  A CTA needs under half an SM's
+//    shared and tensor memory at one or two tokens, so the next projection's
+//    CTA (a programmatic dependent launch) is resident beside it and streams
+//    its own weights while this one drains.
+//  * Warp roles.  Warp 0 (one thread) streams items into two shared-memory
+//    rings with bulk async copies: the quants into the weight ring, the block
+//    scales and the item's x columns (qact.cuh) into the x ring.  Warps 2..5
+//    ("unpack", thread = row) turn a row's quants into the MMA's 8-bit A
+//    operand and store it in tensor memory.  Warp 1 (one thread) issues, per
+//    block of 32 columns, one tcgen05.mma kind::i8 of M = 128 rows,
+//    N = 8 rows per token (the hi / mid / lo digit planes of x and five
+//    unused rows), K = 32: exact int32 sums H, M, L per (row, token) in
+//    tensor memory.  Warps 6..9 ("update", thread = row) read them back and
+//    add d * s * (65536 H + 256 M + L) to the row's f32 accumulator, then
+//    finish tiles (stream-K fix-up and the fused epilogue).
 //  * Reduction order is fixed and independent of NT: per row, exact integer
-//    block sums, blocks in item order inside a warp, then warps 0..7, then CTAs
-//    in grid order (stream-K partials, combined by whichever CTA finishes a tile
-//    last).  Each token's result is produced by the same operations whatever NT
-//    is, so a 16-token pass is bit-identical to 16 single-token passes.
+//    block sums, one f32 update per block in item order, then CTAs in grid
+//    order (stream-K partials, combined by whichever CTA finishes a tile
+//    last).  Each token's result is produced by the same operations whatever
+//    NT is, so a 16-token pass is bit-identical to 16 single-token passes.
 //  * Fused epilogues: input RMS scale (RMSNorm folded as rstd * sum(z W) with
 //    z = h * gamma written by the producer of h), SwiGLU on paired gate/up rows
 //    writing the down projection's input in block fixed-point form, and the
 //    residual add writing h, the next RMSNorm's z (block fixed point) and its
 //    per-tile sums of squares.
+//  * Every wait is bounded (common.cuh); after a timeout each role stops, the
+//    MMA thread waits for its issued MMAs, and the CTA frees its tensor memory.
 #pragma once
 
 #include "qact.cuh"
 #include "qpack.cuh"
+#include "tc5.cuh"
 
 namespace qhl {
 
@@ -62,20 +62,21 @@ struct GemvArgs {
   const float* gamma_next; // RESID: next RMSNorm weight
   float* ss_out;           // RESID: per-tile sum of squares of h_new, [NT][ss_out_stride], or null
   int ss_out_stride;
-  float* partials;         // stream-K scratch: [2 * workers][NT][64]
+  float* partials;         // stream-K scratch: [2 * workers][NT][128]
   int* counters;           // stream-K tile counters, zero between launches
   int workers;             // CTAs that own items (<= items, == grid size)
   unsigned* err;           // device error word
-  // The pass's next projection (null if none): this kernel's producers warm L2
+  // The pass's next projection (null if none): this kernel's producer warms L2
   // with the first items the next kernel's CTA of the same index will stream.
   const uint8_t* next_W;
   int next_items, next_workers;
+  // Failure injection for tests of the bounded waits (0 / -1 in normal use):
+  // iteration cap of every wait (0 = kWaitLimit), and a local item index whose
+  // quants CTA 0's producer never requests, so that its unpack warps' wait on
+  // them runs out.
+  uint32_t wait_limit;
+  int fault_item;
 };
-
-constexpr int kConsumerWarps = 8;
-// Stream-K workers per SM: the grid is kCtasPerSm * SMs for every token count
-// (the split, and hence the summation order, must not depend on NT).
-constexpr int kCtasPerSm = 2;
 
 // Balanced contiguous split of n items (n < 2^31) over p CTAs: CTA w owns
 // items [begin(w), begin(w + 1)) with begin(w) = floor(w n / p), evaluated in
@@ -95,531 +96,50 @@ struct StreamK {
   }
 };
 
-// The quants and scales one lane reads from a stage: its two rows of block `warp`.
-template <int QT> struct ItemRegs;
-template <> struct ItemRegs<kQ4_0> { uint32_t a[4], b[4]; uint32_t sc; };
-template <> struct ItemRegs<kQ8_0> { uint32_t a[8], b[8]; uint32_t sc; };
+// Warp roles.
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kUnpackWarp0 = 2;   // warps 2..5
+constexpr int kUpdateWarp0 = 6;   // warps 6..9
+constexpr int kGemvCtaThreads = 320;
+// Named barriers: 1 = the four update warps, 2 = every warp that touches tensor memory.
+constexpr int kBarUpdate = 1;
+constexpr int kBarTmem = 2;
 
-template <int QT>
-QHL_DEV void load_item(const uint8_t* st, int warp, int lane, ItemRegs<QT>& r) {
-  if constexpr (QT == kQ4_0) {
-    const uint4 wa = *reinterpret_cast<const uint4*>(st + ((warp * 2 + 0) * 32 + lane) * 16);
-    const uint4 wb = *reinterpret_cast<const uint4*>(st + ((warp * 2 + 1) * 32 + lane) * 16);
-    r.a[0] = wa.x; r.a[1] = wa.y; r.a[2] = wa.z; r.a[3] = wa.w;
-    r.b[0] = wb.x; r.b[1] = wb.y; r.b[2] = wb.z; r.b[3] = wb.w;
-  } else {
-    const uint8_t* base = st + (warp * 4) * 32 * 16;   // [half][h][lane][16]
-    const uint4 wa0 = *reinterpret_cast<const uint4*>(base + ((0 * 2 + 0) * 32 + lane) * 16);
-    const uint4 wa1 = *reinterpret_cast<const uint4*>(base + ((1 * 2 + 0) * 32 + lane) * 16);
-    const uint4 wb0 = *reinterpret_cast<const uint4*>(base + ((0 * 2 + 1) * 32 + lane) * 16);
-    const uint4 wb1 = *reinterpret_cast<const uint4*>(base + ((1 * 2 + 1) * 32 + lane) * 16);
-    r.a[0] = wa0.x; r.a[1] = wa0.y; r.a[2] = wa0.z; r.a[3] = wa0.w;
-    r.a[4] = wa1.x; r.a[5] = wa1.y; r.a[6] = wa1.z; r.a[7] = wa1.w;
-    r.b[0] = wb0.x; r.b[1] = wb0.y; r.b[2] = wb0.z; r.b[3] = wb0.w;
-    r.b[4] = wb1.x; r.b[5] = wb1.y; r.b[6] = wb1.z; r.b[7] = wb1.w;
-  }
-  r.sc = *reinterpret_cast<const uint32_t*>(st + QLayout<QT>::kQuantBytes + (warp * 32 + lane) * 4);
-}
-
-// x words of one block: 8 words per byte plane (word k = elements 4k..4k+3).
-struct XBlock { uint32_t hi[8], mid[8], lo[8]; float s; int s_hi, s_ml; };
-
-QHL_DEV void load_xblock(const uint8_t* xt, int warp, XBlock& x) {
-  const uint4* ph = reinterpret_cast<const uint4*>(xt + warp * 32);
-  const uint4* pm = reinterpret_cast<const uint4*>(xt + 256 + warp * 32);
-  const uint4* pl = reinterpret_cast<const uint4*>(xt + 512 + warp * 32);
-  const uint4 h0 = ph[0], h1 = ph[1], m0 = pm[0], m1 = pm[1], l0 = pl[0], l1 = pl[1];
-  x.hi[0] = h0.x; x.hi[1] = h0.y; x.hi[2] = h0.z; x.hi[3] = h0.w;
-  x.hi[4] = h1.x; x.hi[5] = h1.y; x.hi[6] = h1.z; x.hi[7] = h1.w;
-  x.mid[0] = m0.x; x.mid[1] = m0.y; x.mid[2] = m0.z; x.mid[3] = m0.w;
-  x.mid[4] = m1.x; x.mid[5] = m1.y; x.mid[6] = m1.z; x.mid[7] = m1.w;
-  x.lo[0] = l0.x; x.lo[1] = l0.y; x.lo[2] = l0.z; x.lo[3] = l0.w;
-  x.lo[4] = l1.x; x.lo[5] = l1.y; x.lo[6] = l1.z; x.lo[7] = l1.w;
-  x.s = reinterpret_cast<const float*>(xt + 768)[warp];
-  x.s_hi = reinterpret_cast<const int*>(xt + 800)[warp];
-  x.s_ml = reinterpret_cast<const int*>(xt + 832)[warp];
-}
-
-// acc = fma(d * s, 65536 * H + ML, acc): the block's exact integer partial sums
-// turned into one f32 update by a fixed sequence of operations.
-QHL_DEV float block_update(float d, float s, int H, int ML, float acc) {
-  const float v = __fmaf_rn(__int2float_rn(H), 65536.f, __int2float_rn(ML));
-  return __fmaf_rn(__fmul_rn(d, s), v, acc);
-}
-
-// One block for both rows and all NT tokens.
-template <int QT, int NT>
-QHL_DEV void compute_item(const ItemRegs<QT>& r, const uint8_t* xs, int warp, float (&r0)[NT], float (&r1)[NT]) {
-  const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(r.sc & 0xFFFFu)));
-  const float d1 = __half2float(__ushort_as_half(static_cast<unsigned short>(r.sc >> 16)));
-  if constexpr (QT == kQ4_0) {
-    // low nibbles of word i are elements 4i..4i+3, high nibbles 16+4i..16+4i+3
-    uint32_t qa[8], qb[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      qa[i] = r.a[i] & 0x0F0F0F0Fu;
-      qa[4 + i] = (r.a[i] >> 4) & 0x0F0F0F0Fu;
-      qb[i] = r.b[i] & 0x0F0F0F0Fu;
-      qb[4 + i] = (r.b[i] >> 4) & 0x0F0F0F0Fu;
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      XBlock x;
-      load_xblock(xs + t * kQChunkBytes, warp, x);
-      int H0 = 0, M0 = 0, L0 = 0, H1 = 0, M1 = 0, L1 = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {        // q in 0..15: signed x signed is exact for hi
-        H0 = dp4a_ss(qa[k], x.hi[k], H0);
-        M0 = dp4a_uu(qa[k], x.mid[k], M0);
-        L0 = dp4a_uu(qa[k], x.lo[k], L0);
-        H1 = dp4a_ss(qb[k], x.hi[k], H1);
-        M1 = dp4a_uu(qb[k], x.mid[k], M1);
-        L1 = dp4a_uu(qb[k], x.lo[k], L1);
-      }
-      // sum_j (q_j - 8) X_j = 65536 (H - 8 sum hi) + (256 M + L - 8 sum ml)
-      r0[t] = block_update(d0, x.s, H0 - 8 * x.s_hi, M0 * 256 + L0 - 8 * x.s_ml, r0[t]);
-      r1[t] = block_update(d1, x.s, H1 - 8 * x.s_hi, M1 * 256 + L1 - 8 * x.s_ml, r1[t]);
-    }
-  } else {
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      XBlock x;
-      load_xblock(xs + t * kQChunkBytes, warp, x);
-      int H0 = 0, M0 = 0, L0 = 0, H1 = 0, M1 = 0, L1 = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {        // word k holds signed quants 4k..4k+3
-        H0 = dp4a_ss(r.a[k], x.hi[k], H0);
-        M0 = dp4a_su(r.a[k], x.mid[k], M0);
-        L0 = dp4a_su(r.a[k], x.lo[k], L0);
-        H1 = dp4a_ss(r.b[k], x.hi[k], H1);
-        M1 = dp4a_su(r.b[k], x.mid[k], M1);
-        L1 = dp4a_su(r.b[k], x.lo[k], L1);
-      }
-      r0[t] = block_update(d0, x.s, H0, M0 * 256 + L0, r0[t]);
-      r1[t] = block_update(d1, x.s, H1, M1 * 256 + L1, r1[t]);
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Integer tensor-core path (n_tok >= kMmaTok): the same exact int32 block sums
-// as the dp4a path, formed by mma.sync m16n8k32 (8-bit A = weights, B = one
-// activation byte plane, columns = tokens), so both paths give bit-identical
-// results and a 16-token verify still equals 16 single-token passes.  Warp w
-// still owns block w of each item; its 64 rows are 4 m-tiles of 16.  The
-// k order inside a block is GGUF's own: byte j of a Q4_0 row holds elements j
-// (low nibble) and j + 16 (high nibble), which is exactly the split of the
-// A fragment's k range into [4c, 4c + 4) and [16 + 4c, 16 + 4c + 4).
-constexpr int kMmaTok = 4;
-
-template <bool AS, bool BS>
-QHL_DEV void mma_i8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-#define QHL_MMA_I8(AT, BT)                                                                         \
-  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32." AT "." BT ".s32 {%0, %1, %2, %3}, "        \
-               "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"                                 \
-               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])                                    \
-               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0))
-  if constexpr (!AS && BS) QHL_MMA_I8("u8", "s8");
-  else if constexpr (!AS && !BS) QHL_MMA_I8("u8", "u8");
-  else if constexpr (AS && BS) QHL_MMA_I8("s8", "s8");
-  else QHL_MMA_I8("s8", "u8");
-#undef QHL_MMA_I8
-}
-
-// Tokens per thread in the C fragment (columns 2c, 2c + 1 of every n-tile).
-template <int NT>
-struct MmaShape {
-  static constexpr int kNTiles = (NT + 7) / 8;
-  static constexpr int kTok = 2 * kNTiles;
-};
-
-// Row of accumulator m (m-tile m / 2, half m % 2) for lane group g.
-QHL_DEV int mma_row(int m, int g) { return 16 * (m >> 1) + 8 * (m & 1) + g; }
-
-// One block (warp `warp`) of one item for all NT tokens; acc[m][j]: row
-// mma_row(m, g), token 8 * (j / 2) + 2c + (j % 2).
-template <int QT, int NT>
-QHL_DEV void compute_item_mma(const uint8_t* st, const uint8_t* xs, int warp, int lane,
-                              float (&acc)[8][MmaShape<NT>::kTok]) {
-  const int g = lane >> 2, c = lane & 3;
-  // A fragments of the 4 m-tiles: rows 16mt + g and 16mt + g + 8
-  uint32_t a[4][4];
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = 16 * mt + 8 * h + g;
-      if constexpr (QT == kQ4_0) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(st + ((warp * 2 + (r >> 5)) * 32 + (r & 31)) * 16 + 4 * c);
-        a[mt][h] = w & 0x0F0F0F0Fu;                // elements 4c .. 4c + 3
-        a[mt][2 + h] = (w >> 4) & 0x0F0F0F0Fu;     // elements 16 + 4c .. 16 + 4c + 3
-      } else {
-        const uint8_t* base = st + (warp * 4) * 32 * 16;
-        a[mt][h] = *reinterpret_cast<const uint32_t*>(base + ((0 * 2 + (r >> 5)) * 32 + (r & 31)) * 16 + 4 * c);
-        a[mt][2 + h] = *reinterpret_cast<const uint32_t*>(base + ((1 * 2 + (r >> 5)) * 32 + (r & 31)) * 16 + 4 * c);
-      }
-    }
-  }
-  // row scales: word (g + 8q) holds rows g + 8q (low half) and g + 8q + 32 (high half)
-  float dsc[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int r = mma_row(m, g);
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(st + QLayout<QT>::kQuantBytes + (warp * 32 + (r & 31)) * 4);
-    dsc[m] = __half2float(__ushort_as_half(static_cast<unsigned short>((r >> 5) ? (w >> 16) : (w & 0xFFFFu))));
-  }
-#pragma unroll
-  for (int nt = 0; nt < MmaShape<NT>::kNTiles; ++nt) {
-    // B fragments: column g = token 8nt + g, k = 4c .. 4c + 3 and 16 + 4c ..
-    const int tb = 8 * nt + g;
-    uint32_t b[3][2];
-#pragma unroll
-    for (int p = 0; p < 3; ++p) {
-      if (tb < NT) {
-        const uint8_t* xp = xs + tb * kQChunkBytes + p * 256 + warp * 32;
-        b[p][0] = *reinterpret_cast<const uint32_t*>(xp + 4 * c);
-        b[p][1] = *reinterpret_cast<const uint32_t*>(xp + 16 + 4 * c);
-      } else {
-        b[p][0] = 0u;
-        b[p][1] = 0u;
-      }
-    }
-    // block scales of this thread's two C-fragment tokens
-    float s[2];
-    int shi[2], sml[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int t = 8 * nt + 2 * c + e;
-      const uint8_t* xt = xs + (t < NT ? t : 0) * kQChunkBytes;
-      s[e] = reinterpret_cast<const float*>(xt + 768)[warp];
-      shi[e] = reinterpret_cast<const int*>(xt + 800)[warp];
-      sml[e] = reinterpret_cast<const int*>(xt + 832)[warp];
-    }
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-      int dh[4], dm[4], dl[4];
-      mma_i8<QT == kQ8_0, true>(dh, a[mt], b[0][0], b[0][1]);    // hi plane: signed
-      mma_i8<QT == kQ8_0, false>(dm, a[mt], b[1][0], b[1][1]);   // mid plane: unsigned
-      mma_i8<QT == kQ8_0, false>(dl, a[mt], b[2][0], b[2][1]);   // lo plane: unsigned
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 8 * nt + 2 * c + e;
-          if (t < NT) {
-            const int m = 2 * mt + h, j = 2 * nt + e, q = 2 * h + e;
-            if constexpr (QT == kQ4_0)
-              acc[m][j] = block_update(dsc[m], s[e], dh[q] - 8 * shi[e], dm[q] * 256 + dl[q] - 8 * sml[e], acc[m][j]);
-            else
-              acc[m][j] = block_update(dsc[m], s[e], dh[q], dm[q] * 256 + dl[q], acc[m][j]);
-          }
-        }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Warp roles of a GEMV CTA: warps 0..7 consume items, warp 8 produces (bulk
-// copies into the ring), warp 9 finishes tiles.  The consumers hand each
-// finished tile's per-warp sums to the epilogue warp through a small ring of
-// reduction buffers (mbarriers "tile full" / "tile free") and go straight on
-// with the next item; the epilogue warp sums the eight warps' partials, runs
-// the stream-K fix-up and the fused epilogue off the item loop's path.
-constexpr int kProducerWarp = kConsumerWarps;
-constexpr int kEpilogueWarp = kConsumerWarps + 1;
-constexpr int kGemvCtaThreads = (kConsumerWarps + 2) * 32;
-
-// Reduction buffers between consumers and the epilogue warp.
-template <int NT>
-struct TileRing {
-  static constexpr int kBufs = NT <= 4 ? 2 : 1;
-  static constexpr int kBufFloats = kConsumerWarps * NT * 64;   // [8][NT][64]
-  static constexpr int kBytes = kBufs * kBufFloats * 4;
-};
-
-// Hand-off state shared by the consumers and the epilogue warp of one CTA.
-struct TileSync {
-  float* red;          // [kBufs][8][NT][64]
-  uint64_t* full;      // [kBufs], 256 arrivals (every consumer thread)
-  uint64_t* free_;     // [kBufs], 32 arrivals (every epilogue lane)
-};
-
-// Inputs of a tile's epilogue that do not depend on the tile's sums, loaded
-// before the sums are ready: the residual stream h (written by an earlier
-// step) and the next RMSNorm weight, for the lanes' elements.
-template <int NT>
-struct EpiInputs {
-  float h[NT * 2];     // element i * 32 + lane of [NT][64]
-  float gamma[2];      // rows lane and 32 + lane
-};
-
-template <int EPI, int NT>
-QHL_DEV void gemv_prefetch(const GemvArgs& a, int tile, int lane, EpiInputs<NT>& in) {
-  if constexpr (EPI == EPI_RESID) {
-#pragma unroll
-    for (int i = 0; i < NT * 2; ++i) {
-      const int idx = i * 32 + lane, t = idx >> 6, gr = tile * 64 + (idx & 63);
-      in.h[i] = gr < a.out_valid ? ld_cg_once(a.y + (size_t)t * a.y_stride + gr) : 0.f;   // h: written by other CTAs
-    }
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const int gr = tile * 64 + b * 32 + lane;
-      in.gamma[b] = a.qout && gr < a.out_valid ? __ldg(a.gamma_next + gr) : 0.f;
-    }
-  }
-}
-
-// Epilogue of one finished tile by the 32 lanes of the epilogue warp;
-// vals = [NT][64] final sums in shared memory, rstd = [NT].
-template <int EPI, int NT>
-QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, float* vals, const float* rstd, int lane,
-                           const EpiInputs<NT>& in) {
-  if constexpr (EPI == EPI_STORE) {
-#pragma unroll
-    for (int i = 0; i < NT * 2; ++i) {
-      const int idx = i * 32 + lane, t = idx >> 6, gr = tile * 64 + (idx & 63);
-      if (gr < a.out_valid) a.y[(size_t)t * a.y_stride + gr] = __fmul_rn(vals[idx], rstd[t]);
-    }
-  } else if constexpr (EPI == EPI_SWIGLU) {
-    // tile rows 0..31 are gate rows of features tile*32.., rows 32..63 the matching up rows
-#pragma unroll 1
-    for (int t = 0; t < NT; ++t) {
-      const int f = tile * 32 + lane;
-      float u = 0.f;
-      if (f < a.out_valid) {
-        const float g = __fmul_rn(vals[t * 64 + lane], rstd[t]);
-        const float up = __fmul_rn(vals[t * 64 + 32 + lane], rstd[t]);
-        u = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), up);   // silu(g) * up
-      }
-      qact_store_block(u, a.qout + (size_t)t * a.qout_stride, tile, lane);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < NT * 2; ++i) {
-      const int idx = i * 32 + lane, t = idx >> 6, gr = tile * 64 + (idx & 63);
-      float hn = 0.f;
-      if (gr < a.out_valid) {
-        hn = __fadd_rn(in.h[i], vals[idx]);
-        a.y[(size_t)t * a.y_stride + gr] = hn;
-      }
-      vals[idx] = hn;
-    }
-    __syncwarp();
-    if (a.qout) {
-#pragma unroll 1
-      for (int p = 0; p < NT * 2; ++p) {
-        const int t = p >> 1, b = p & 1, gr = tile * 64 + b * 32 + lane;
-        const float z = gr < a.out_valid ? __fmul_rn(vals[t * 64 + b * 32 + lane], b ? in.gamma[1] : in.gamma[0]) : 0.f;
-        qact_store_block(z, a.qout + (size_t)t * a.qout_stride, tile * 2 + b, lane);
-      }
-    }
-    if (a.ss_out && lane < NT) a.ss_out[(size_t)lane * a.ss_out_stride + tile] = sumsq64(vals + lane * 64);
-    __syncwarp();
-  }
-}
-
-// Stream-K tile counter: add 1 with release (this CTA's partial, published
-// by every lane before the warp barrier, becomes visible with it) and acquire
-// (the last contributor then sees every other partial).
-QHL_DEV int counter_add_acq_rel(int* p) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
-  return old;
-}
-
-// Consumer side of one GEMV for CTA `cta` (the 256 threads of warps 0..7):
-// takes this CTA's stream-K items, in order, from the shared-memory ring
-// (`slot` / `phase` carry the ring position across calls) and hands every
-// tile's per-warp sums to the epilogue warp (`tc` counts hand-offs across
-// calls).
-template <int QT, int NT, int S>
-QHL_DEV void gemv_consume(const GemvArgs& a, int cta, uint8_t* stages, uint64_t* bars, const TileSync& ts, int& slot,
-                          uint32_t& phase, uint32_t& tc, bool& timed_out) {
-  constexpr int IB = QLayout<QT>::kItemBytes;
-  constexpr int SB = IB + NT * kQChunkBytes;
-  constexpr int RB = TileRing<NT>::kBufs;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (cta >= a.workers) return;
-  const StreamK sk(a.tiles * a.chunks, a.workers);
-  const int i0 = sk.begin(cta), n_local = sk.begin(cta + 1) - i0;
-  if (n_local == 0) return;
-
-  constexpr bool kMma = NT >= kMmaTok;
-  constexpr int kAccA = kMma ? 1 : NT;                        // dp4a: rows lane, lane + 32
-  constexpr int kAccT = kMma ? MmaShape<NT>::kTok : 1;        // mma: C-fragment rows and tokens
-  float r0[kAccA], r1[kAccA];
-  float acc[kMma ? 8 : 1][kAccT];
-#pragma unroll
-  for (int t = 0; t < kAccA; ++t) { r0[t] = 0.f; r1[t] = 0.f; }
-#pragma unroll
-  for (int m = 0; m < (kMma ? 8 : 1); ++m)
-#pragma unroll
-    for (int j = 0; j < kAccT; ++j) acc[m][j] = 0.f;
-  auto handoff = [&]() {
-    const int buf = (int)(tc % RB);
-    const uint32_t use = tc / RB;
-    if (use > 0 && !timed_out && !mbar_wait(smem_u32(&ts.free_[buf]), (use - 1) & 1u, a.err)) timed_out = true;
-    float* red = ts.red + buf * TileRing<NT>::kBufFloats;
-    if constexpr (kMma) {
-      const int g = lane >> 2, c = lane & 3;
-#pragma unroll
-      for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int j = 0; j < kAccT; ++j) {
-          const int t = 8 * (j >> 1) + 2 * c + (j & 1);
-          if (t < NT) red[(warp * NT + t) * 64 + mma_row(m, g)] = acc[m][j];
-          acc[m][j] = 0.f;
-        }
-    } else {
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        red[(warp * NT + t) * 64 + lane] = r0[t];
-        red[(warp * NT + t) * 64 + 32 + lane] = r1[t];
-        r0[t] = 0.f;
-        r1[t] = 0.f;
-      }
-    }
-    mbar_arrive(smem_u32(&ts.full[buf]));
-    ++tc;
-  };
-
-  int chunk = i0 % a.chunks;
-  for (int k = 0; k < n_local; ++k) {
-    if (chunk == a.chunks) {
-      handoff();
-      chunk = 0;
-    }
-    // after one timed-out wait the rest of the call runs without waiting (the
-    // error is recorded; results are garbage, but the kernel ends promptly)
-    if (!timed_out && !mbar_wait(smem_u32(&bars[slot]), phase, a.err)) timed_out = true;
-    const uint8_t* st = stages + slot * SB;
-    if constexpr (kMma) {
-      compute_item_mma<QT, NT>(st, st + IB, warp, lane, acc);
-    } else {
-      ItemRegs<QT> regs;
-      load_item<QT>(st, warp, lane, regs);
-      compute_item<QT, NT>(regs, st + IB, warp, r0, r1);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&bars[S + slot]));   // stage free for the producer
-    ++chunk;
-    if (++slot == S) {
-      slot = 0;
-      phase ^= 1u;
-    }
-  }
-  handoff();
-}
-
-// Epilogue-warp side of one GEMV: for every tile this CTA touches, in order,
-// sum the eight warps' partials (warps 0..7 in order), then either finish the
-// tile (all its chunks were this CTA's) or publish the partial and, if this
-// CTA is the last contributor to arrive, combine every contributor's partial
-// in CTA order and finish it.  `fin` = [NT][64], `rstd` = [NT] (computed
-// here, from the previous step's per-tile sums of squares).
-template <int EPI, int NT>
-QHL_DEV void gemv_finish(const GemvArgs& a, int cta, const TileSync& ts, float* fin, float* rstd, uint32_t& tc,
-                         bool& timed_out) {
-  constexpr int RB = TileRing<NT>::kBufs;
-  const int lane = threadIdx.x & 31;
-  if (cta >= a.workers) return;
-  const StreamK sk(a.tiles * a.chunks, a.workers);
-  const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1);
-  if (i1 == i0) return;
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const float r = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
-    if (lane == 0) rstd[t] = r;
-  }
-  __syncwarp();
-  const int first_tile = i0 / a.chunks, last_tile = (i1 - 1) / a.chunks;
-  for (int tl = first_tile; tl <= last_tile; ++tl) {
-    EpiInputs<NT> in;
-    gemv_prefetch<EPI, NT>(a, tl, lane, in);
-    const int buf = (int)(tc % RB);
-    const uint32_t use = tc / RB;
-    if (!timed_out && !mbar_wait(smem_u32(&ts.full[buf]), use & 1u, a.err)) timed_out = true;
-    const float* red = ts.red + buf * TileRing<NT>::kBufFloats;
-#pragma unroll
-    for (int i = 0; i < NT * 2; ++i) {
-      const int idx = i * 32 + lane;
-      float v = red[idx];
-#pragma unroll
-      for (int w = 1; w < kConsumerWarps; ++w) v = __fadd_rn(v, red[w * NT * 64 + idx]);
-      fin[idx] = v;
-    }
-    __syncwarp();
-    mbar_arrive(smem_u32(&ts.free_[buf]));
-    ++tc;
-    const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
-    if (t_lo >= i0 && t_hi <= i1) {
-      gemv_epilogue<EPI, NT>(a, tl, fin, rstd, lane, in);
-      continue;
-    }
-    // stream-K: publish this CTA's partial; the last contributor to arrive
-    // combines every contributor's partial in CTA order and finishes the tile.
-    // Partials move as float2: lane owns elements 2q, 2q + 1, q = j * 32 + lane.
-    float2* mine = reinterpret_cast<float2*>(a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * 64);
-    const float2* fin2 = reinterpret_cast<const float2*>(fin);
-#pragma unroll
-    for (int j = 0; j < NT; ++j) mine[j * 32 + lane] = fin2[j * 32 + lane];
-    __syncwarp();
-    const int cf = sk.owner(t_lo), cl = sk.owner(t_hi - 1);
-    int last = 0;
-    if (lane == 0) last = counter_add_acq_rel(&a.counters[tl]) == cl - cf ? 1 : 0;
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) continue;
-    // Tile tl is the first tile of every contributor after cf, and of cf
-    // exactly when cf's range starts at the tile's first item.  Up to 4
-    // float2 loads per lane in flight.
-    constexpr int CB = NT >= 4 ? 1 : 4 / NT;
-    const int cf_slot = sk.begin(cf) == t_lo ? 0 : 1;
-    float2 acc[NT];
-    for (int c0 = cf; c0 <= cl; c0 += CB) {
-      float2 pv[CB][NT];
-#pragma unroll
-      for (int k = 0; k < CB; ++k) {
-        const int c = c0 + k;
-        if (c <= cl) {
-          const float2* pc =
-              reinterpret_cast<const float2*>(a.partials + (size_t)(2 * c + (c == cf ? cf_slot : 0)) * NT * 64);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) pv[k][j] = ld_cg_once(pc + j * 32 + lane);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < CB; ++k)
-        if (c0 + k <= cl) {
-#pragma unroll
-          for (int j = 0; j < NT; ++j)
-            acc[j] = (c0 + k == cf) ? pv[k][j]
-                                    : make_float2(__fadd_rn(acc[j].x, pv[k][j].x), __fadd_rn(acc[j].y, pv[k][j].y));
-        }
-    }
-    float2* fout = reinterpret_cast<float2*>(fin);
-#pragma unroll
-    for (int j = 0; j < NT; ++j) fout[j * 32 + lane] = acc[j];
-    __syncwarp();
-    gemv_epilogue<EPI, NT>(a, tl, fin, rstd, lane, in);
-    if (lane == 0) a.counters[tl] = 0;
-  }
-}
-
+// Geometry and shared-memory layout of one (weight type, token count).
 template <int QT, int NT>
 struct GemvCfg {
-  static constexpr int kStageBytes = QLayout<QT>::kItemBytes + NT * kQChunkBytes;
-  // two CTAs per SM up to 4 tokens, one beyond
-  static constexpr int kBudget = NT <= 4 ? 112 * 1024 : 200 * 1024;
-  static constexpr int kFixed = TileRing<NT>::kBytes + NT * 64 * 4 + 16 * 4 + 64;
-  static constexpr int kRaw = (kBudget - kFixed) / (kStageBytes + 16);
-  static constexpr int kStages = kRaw < 3 ? 3 : (kRaw > 16 ? 16 : kRaw);
-  static constexpr int kMinBlocks = NT <= 4 ? 2 : 1;
-  // shared-memory layout
-  static constexpr int kRedOff = kStages * kStageBytes;
-  static constexpr int kFinOff = kRedOff + TileRing<NT>::kBytes;
-  static constexpr int kRstdOff = kFinOff + NT * 64 * 4;
-  static constexpr int kBarOff = kRstdOff + 16 * 4;                        // 8-byte aligned
-  static constexpr int kSmem = kBarOff + (2 * kStages + 2 * TileRing<NT>::kBufs) * 8;
+  static constexpr int kN = NT == 1 ? 8 : 16 * ((NT + 1) / 2);   // MMA N: 8 rows per token, padded
+  static constexpr int kNTP = kN / 8;                              // token regions in an x slot
+  static constexpr int kGB = (64 / kN) >= 8 ? 8 : ((64 / kN) >= 1 ? 64 / kN : 1);   // blocks per D group
+  static constexpr int kNG = 8 / kGB;                              // D groups per item
+  static constexpr int kDCols = kGB * kN;                          // tensor-memory columns of a D buffer
+  static constexpr int kACols = 64;                                // 8 blocks x 32 bytes / 4
+  static constexpr int kDOff = 2 * kACols;
+  static constexpr int kTmemCols = kDOff + 2 * kDCols <= 256 ? 256 : 512;
+  static constexpr int kQB = QLayout<QT>::kQuantBytes;
+  static constexpr int kXS = QLayout<QT>::kScaleBytes + kNTP * kQChunkBytes;   // x slot: scales, then tokens
+  // two CTAs per SM (this projection and the next) at one and two tokens (Q4_0)
+  static constexpr bool kPair = QT == kQ4_0 && NT <= 2;
+  static constexpr int kBudget = kPair ? 110 * 1024 : 200 * 1024;
+  static constexpr int kEpi = NT * kTileRows * 4;                  // epilogue exchange [NT][128] f32
+  static constexpr int kFixed = kEpi + 16 * 4 + 16 + 320;          // + rstd, tmem slot, barriers
+  static constexpr int kSX = kPair ? 6 : 3;
+  static constexpr int kSW0 = (kBudget - kFixed - kSX * kXS) / kQB;
+  static constexpr int kSW = kSW0 > 8 ? 8 : kSW0;
+  static constexpr int kMinBlocks = kPair ? 2 : 1;
+  // shared-memory layout (the rings first; every slot 16-byte aligned)
+  static constexpr int kXOff = kSW * kQB;
+  static constexpr int kEpiOff = kXOff + kSX * kXS;
+  static constexpr int kRstdOff = kEpiOff + kEpi;
+  static constexpr int kSlotOff = kRstdOff + 16 * 4;
+  static constexpr int kBarOff = kSlotOff + 16;
+  // barriers: wfull[SW], wempty[SW], xfull[SX], xempty[SX], afull[2], afree[2], dfull[2], dfree[2], drain
+  static constexpr int kNumBars = 2 * kSW + 2 * kSX + 9;
+  static constexpr int kSmem = kBarOff + kNumBars * 8;
+  static_assert(kSW >= 2, "weight ring too shallow");
+  static_assert(kNumBars * 8 <= 320, "barrier area");
+  static_assert(kSmem <= kBudget, "shared-memory budget");
 };
 
 template <int QT, int NT>
@@ -627,96 +147,433 @@ constexpr int gemv_smem_bytes() {
   return GemvCfg<QT, NT>::kSmem;
 }
 
+// Non-blocking test of an mbarrier phase.
+QHL_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Stream-K tile counter: add 1 with release (this CTA's partial, published by
+// every update thread before the named barrier, becomes visible with it) and
+// acquire (the last contributor then sees every other partial).
+QHL_DEV int counter_add_acq_rel(int* p) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
+// f32 update of one (row, block, token): acc + d * s * sum_j q_j X_j, with the
+// exact integer sums H, M, L of the three digit planes.
+template <int QT>
+QHL_DEV float block_update(float acc, float d, float s, int H, int M, int L, int Sh, int Sml) {
+  int Hx = H, MLx = M * 256 + L;
+  if constexpr (QT == kQ4_0) {   // weights are nibble - 8
+    Hx -= 8 * Sh;
+    MLx -= 8 * Sml;
+  }
+  const float v = __fmaf_rn(__int2float_rn(Hx), 65536.f, __int2float_rn(MLx));
+  return __fmaf_rn(__fmul_rn(d, s), v, acc);
+}
+
+// Sum of squares of a 128-row tile held one row per thread by four warps
+// (quarter q = rows 32q .. 32q + 31): xor-butterfly per warp, then the four
+// warps in order.  The one definition used for the per-tile RMSNorm partials
+// everywhere, so a stage's result never depends on which kernel produced its
+// input.  `red` = shared [4] per token; `bar_id` names a barrier over the four
+// warps (128 threads).  Returns the sum in every thread.
+QHL_DEV float tile_sumsq(float v, float* red, int quarter, int lane, int bar_id) {
+  const float w = warp_sum(__fmul_rn(v, v));
+  if (lane == 0) red[quarter] = w;
+  named_sync(bar_id, 128);
+  const float s = __fadd_rn(__fadd_rn(__fadd_rn(red[0], red[1]), red[2]), red[3]);
+  named_sync(bar_id, 128);
+  return s;
+}
+
+// Epilogue of one finished tile by the four update warps, thread = tile row r
+// (quarter q = r / 32); v[t] = the tile's final sums for row r.
+template <int EPI, int NT>
+QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, const float (&v)[NT], const float* rstd, float* ex, int quarter,
+                           int lane) {
+  const int r = quarter * 32 + lane;
+  if constexpr (EPI == EPI_STORE) {
+    const int gr = tile * kTileRows + r;
+    if (gr < a.out_valid)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) a.y[(size_t)t * a.y_stride + gr] = __fmul_rn(v[t], rstd[t]);
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    // rows 0..63: gate rows of features 64 tile + r; rows 64..127 the matching up rows
+    if (r >= 64)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) ex[t * kTileRows + r - 64] = __fmul_rn(v[t], rstd[t]);
+    named_sync(kBarUpdate, 128);
+    if (r < 64) {
+      const int f = tile * 64 + r;
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float u = 0.f;
+        if (f < a.out_valid) {
+          const float g = __fmul_rn(v[t], rstd[t]);
+          const float up = ex[t * kTileRows + r];
+          u = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), up);   // silu(g) * up
+        }
+        qact_store_block(u, a.qout + (size_t)t * a.qout_stride, tile * 2 + quarter, lane);
+      }
+    }
+    named_sync(kBarUpdate, 128);
+  } else {
+    const int gr = tile * kTileRows + r;
+    const bool valid = gr < a.out_valid;
+    const float gam = a.qout && valid ? __ldg(a.gamma_next + gr) : 0.f;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float hn = 0.f;
+      if (valid) {
+        hn = __fadd_rn(__ldcg(a.y + (size_t)t * a.y_stride + gr), v[t]);
+        a.y[(size_t)t * a.y_stride + gr] = hn;
+      }
+      if (a.qout) qact_store_block(__fmul_rn(hn, gam), a.qout + (size_t)t * a.qout_stride, tile * 4 + quarter, lane);
+      if (a.ss_out) {
+        const float s = tile_sumsq(hn, ex + 4 * t, quarter, lane, kBarUpdate);
+        if (r == 0) a.ss_out[(size_t)t * a.ss_out_stride + tile] = s;
+      }
+    }
+  }
+}
+
+// Update warps: finish tile `tl` given this CTA's partial v (stream-K fix-up
+// if the tile is shared, then the epilogue).
+template <int EPI, int NT>
+QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int i0, int i1, int tl, float (&v)[NT],
+                              const float* rstd, float* ex, int* flag, int quarter, int lane) {
+  const int r = quarter * 32 + lane;
+  const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
+  if (t_lo >= i0 && t_hi <= i1) {
+    gemv_epilogue<EPI, NT>(a, tl, v, rstd, ex, quarter, lane);
+    return;
+  }
+  // publish this CTA's partial (slot 0: its first tile, slot 1: its last)
+  const int first_tile = i0 / a.chunks;
+  float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * kTileRows;
+#pragma unroll
+  for (int t = 0; t < NT; ++t) mine[t * kTileRows + r] = v[t];
+  __threadfence();
+  named_sync(kBarUpdate, 128);
+  const int cf = sk.owner(t_lo), cl = sk.owner(t_hi - 1);
+  if (r == 0) *flag = counter_add_acq_rel(&a.counters[tl]) == cl - cf ? 1 : 0;
+  named_sync(kBarUpdate, 128);
+  const int last = *flag;
+  named_sync(kBarUpdate, 128);
+  if (!last) return;
+  __threadfence();   // every thread orders its partial loads after the acquire above
+  // combine every contributor's partial in CTA order; tile tl is the first
+  // tile of every contributor after cf, and of cf exactly when cf's range
+  // starts at the tile's first item
+  const int cf_slot = sk.begin(cf) == t_lo ? 0 : 1;
+  float acc[NT];
+  constexpr int CB = 4;
+  for (int c0 = cf; c0 <= cl; c0 += CB) {
+    float pv[CB][NT];
+#pragma unroll
+    for (int k = 0; k < CB; ++k) {
+      const int c = c0 + k;
+      if (c <= cl) {
+        const float* pc = a.partials + (size_t)(2 * c + (c == cf ? cf_slot : 0)) * NT * kTileRows;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) pv[k][t] = c == cta ? v[t] : ld_cg_once(pc + t * kTileRows + r);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < CB; ++k)
+      if (c0 + k <= cl) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[t] = (c0 + k == cf) ? pv[k][t] : __fadd_rn(acc[t], pv[k][t]);
+      }
+  }
+  gemv_epilogue<EPI, NT>(a, tl, acc, rstd, ex, quarter, lane);
+  if (r == 0) a.counters[tl] = 0;
+}
+
 template <int QT, int NT, int EPI>
 __global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
   using C = GemvCfg<QT, NT>;
-  constexpr int S = C::kStages;
-  constexpr int IB = QLayout<QT>::kItemBytes;
-  constexpr int SB = C::kStageBytes;
-  constexpr int RB = TileRing<NT>::kBufs;
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* stages = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);   // full[S], empty[S], tile full[RB], tile free[RB]
-  const TileSync ts{reinterpret_cast<float*>(smem + C::kRedOff), bars + 2 * S, bars + 2 * S + RB};
-  float* fin = reinterpret_cast<float*>(smem + C::kFinOff);
-  float* rstd = reinterpret_cast<float*>(smem + C::kRstdOff);
+  constexpr int SW = C::kSW, SX = C::kSX, QB = C::kQB, XS = C::kXS;
+  extern __shared__ __align__(16) uint8_t gsmem[];
+  uint8_t* wring = gsmem;
+  uint8_t* xring = gsmem + C::kXOff;
+  float* ex = reinterpret_cast<float*>(gsmem + C::kEpiOff);
+  float* rstd = reinterpret_cast<float*>(gsmem + C::kRstdOff);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(gsmem + C::kSlotOff);
+  int* flag = reinterpret_cast<int*>(gsmem + C::kSlotOff + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gsmem + C::kBarOff);
+  uint64_t* wfull = bars;
+  uint64_t* wempty = bars + SW;
+  uint64_t* xfull = bars + 2 * SW;
+  uint64_t* xempty = bars + 2 * SW + SX;
+  uint64_t* afull = bars + 2 * SW + 2 * SX;
+  uint64_t* afree = afull + 2;
+  uint64_t* dfull = afull + 4;
+  uint64_t* dfree = afull + 6;
+  uint64_t* drain = afull + 8;
 
   const int cta = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) pdl_launch();
   if (cta >= a.workers) return;
   const StreamK sk(a.tiles * a.chunks, a.workers);
-  const int i0 = sk.begin(cta), n_local = sk.begin(cta + 1) - i0;
+  const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1), n = i1 - i0;
+  if (n == 0) return;
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&bars[s]), 1);
-      mbar_init(smem_u32(&bars[S + s]), kConsumerWarps);
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(smem_u32(&wfull[s]), 1);
+      mbar_init(smem_u32(&wempty[s]), 4);
     }
-    for (int b = 0; b < RB; ++b) {
-      mbar_init(smem_u32(&ts.full[b]), kConsumerWarps * 32);
-      mbar_init(smem_u32(&ts.free_[b]), 32);
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(smem_u32(&xfull[s]), 1);
+      mbar_init(smem_u32(&xempty[s]), 4);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&afull[b]), 4);
+      mbar_init(smem_u32(&afree[b]), 1);
+      mbar_init(smem_u32(&dfull[b]), 1);
+      mbar_init(smem_u32(&dfree[b]), 4);
+    }
+    mbar_init(smem_u32(drain), 1);
     fence_mbar_init();
   }
+  if (warp == kMmaWarp) tmem_alloc(tslot, C::kTmemCols);
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
 
   if (warp == kProducerWarp) {
-    // ---------------- producer: stream this CTA's items into the ring ----------
-    // Weights never depend on earlier kernels: the first S items' weights are
-    // requested before griddepcontrol.wait.  Their x chunks (written by the
-    // previous kernel) follow once the dependency is resolved.
+    // ---------------- producer: one thread streams this CTA's items ----------
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      const int pre = n_local < S ? n_local : S;
       const int c0 = i0 % a.chunks;
-      auto issue_x = [&](int k, int s) {
-        int c = c0 + k;                    // chunk of local item k, without 64-bit division
-        while (c >= a.chunks) c -= a.chunks;
-        const uint32_t full = smem_u32(&bars[s]);
-        for (int t = 0; t < NT; ++t)
-          bulk_g2s_plain(smem_u32(stages + s * SB + IB + t * kQChunkBytes),
-                         a.qx + (size_t)t * a.qx_stride + (size_t)c * kQChunkBytes, kQChunkBytes, full);
+      auto chunk_of = [&](int k) {   // chunk of local item k, without 64-bit division
+        int c = c0 + k % a.chunks;
+        return c >= a.chunks ? c - a.chunks : c;
       };
-      for (int k = 0; k < pre; ++k) {
-        const uint32_t full = smem_u32(&bars[k]);
-        mbar_arrive_expect_tx(full, SB);
-        bulk_g2s(smem_u32(stages + k * SB), a.W + (size_t)(i0 + k) * IB, IB, full, pol);
-      }
+      auto issue_w = [&](int k) {
+        const int s = k % SW;
+        if (cta == 0 && k == a.fault_item) return;   // injected failure: this slot never fills
+        mbar_arrive_expect_tx(smem_u32(&wfull[s]), QB);
+        bulk_g2s(smem_u32(wring + s * QB), a.W + (size_t)(i0 + k) * QLayout<QT>::kItemBytes, QB,
+                 smem_u32(&wfull[s]), pol);
+      };
+      auto issue_scales = [&](int k) {
+        const int s = k % SX;
+        mbar_arrive_expect_tx(smem_u32(&xfull[s]), QLayout<QT>::kScaleBytes + NT * kQChunkBytes);
+        bulk_g2s(smem_u32(xring + s * XS), a.W + (size_t)(i0 + k) * QLayout<QT>::kItemBytes + QB,
+                 QLayout<QT>::kScaleBytes, smem_u32(&xfull[s]), pol);
+      };
+      auto issue_x = [&](int k) {
+        const int s = k % SX, c = chunk_of(k);
+        for (int t = 0; t < NT; ++t)
+          bulk_g2s_plain(smem_u32(xring + s * XS + QLayout<QT>::kScaleBytes + t * kQChunkBytes),
+                         a.qx + (size_t)t * a.qx_stride + (size_t)c * kQChunkBytes, kQChunkBytes,
+                         smem_u32(&xfull[s]));
+      };
+      // weights never depend on earlier kernels: the first rings are requested
+      // before griddepcontrol.wait; the x columns (written by the previous
+      // kernel) once the dependency is resolved
+      int kw = 0, kx = 0;
+      for (; kw < n && kw < SW; ++kw) issue_w(kw);
+      for (int k = 0; k < n && k < SX; ++k) issue_scales(k);
       pdl_wait();
-      for (int k = 0; k < pre; ++k) issue_x(k, k);
-      for (int k = pre; k < n_local; ++k) {
-        const int s = k % S, round = k / S;
-        if (!mbar_wait(smem_u32(&bars[S + s]), (round - 1) & 1, a.err)) {
-          drain_inflight_copies();   // error path
-          return;
+      for (; kx < n && kx < SX; ++kx) issue_x(kx);
+      bool ok = true;
+      for (uint32_t spins = 0; ok && (kw < n || kx < n);) {
+        bool did = false;
+        if (kw < n && mbar_test(smem_u32(&wempty[kw % SW]), ((kw / SW) - 1) & 1u)) {
+          issue_w(kw++);
+          did = true;
         }
-        const uint32_t full = smem_u32(&bars[s]);
-        mbar_arrive_expect_tx(full, SB);
-        bulk_g2s(smem_u32(stages + s * SB), a.W + (size_t)(i0 + k) * IB, IB, full, pol);
-        issue_x(k, s);
+        if (kx < n && mbar_test(smem_u32(&xempty[kx % SX]), ((kx / SX) - 1) & 1u)) {
+          issue_scales(kx);
+          issue_x(kx++);
+          did = true;
+        }
+        if (did) {
+          spins = 0;
+        } else if (++spins > wait_limit(a.wait_limit)) {
+          atomicOr(a.err, ERR_WAIT_TIMEOUT);
+          ok = false;
+        } else {
+          __nanosleep(32);   // both rings full: poll lightly
+        }
       }
-      // every own item is on its way: warm L2 with the next projection's first
-      // items of this CTA index while the consumers finish (the next kernel's
-      // copies of them then hit L2)
-      if (a.next_W && cta < a.next_workers) {
+      if (ok && a.next_W && cta < a.next_workers) {
+        // every own item is on its way: warm L2 with the next projection's
+        // first items of this CTA index while the consumers finish
         const StreamK skn(a.next_items, a.next_workers);
-        const int j0 = skn.begin(cta), nj = min(S, skn.begin(cta + 1) - j0);
-        for (int k = 0; k < nj; ++k) bulk_prefetch_l2(a.next_W + (size_t)(j0 + k) * IB, IB);
+        const int j0 = skn.begin(cta), nj = min(SW, skn.begin(cta + 1) - j0);
+        for (int k = 0; k < nj; ++k) bulk_prefetch_l2(a.next_W + (size_t)(j0 + k) * QLayout<QT>::kItemBytes,
+                                                      QLayout<QT>::kItemBytes);
       }
+      if (!ok) drain_inflight_copies();   // error path
     }
-    return;
+    return;   // the producer takes no part in the tensor-memory teardown
   }
 
-  pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
-  uint32_t tc = 0;
   bool timed_out = false;
-  if (warp == kEpilogueWarp) {
-    gemv_finish<EPI, NT>(a, cta, ts, fin, rstd, tc, timed_out);
+  if (warp == kMmaWarp) {
+    // ---------------- MMA issuer: one thread ---------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(QT == kQ8_0, kTileRows, C::kN);
+      uint32_t gc = 0;
+      for (int k = 0; k < n && !timed_out; ++k) {
+        const int ab = k & 1, sx = k % SX;
+        if (!mbar_wait(smem_u32(&afull[ab]), (uint32_t)(k >> 1) & 1u, a.err, a.wait_limit) ||
+            !mbar_wait(smem_u32(&xfull[sx]), (uint32_t)(k / SX) & 1u, a.err, a.wait_limit)) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t xs = smem_u32(xring + sx * XS + QLayout<QT>::kScaleBytes);
+        for (int g = 0; g < C::kNG; ++g, ++gc) {
+          const int db = gc & 1;
+          if (gc >= 2 && !mbar_wait(smem_u32(&dfree[db]), ((gc >> 1) - 1) & 1u, a.err, a.wait_limit)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < C::kGB; ++j) {
+            const int b = g * C::kGB + j;
+            const uint64_t desc = smem_desc_kmajor(xs + b * kQBlockBytes, 128, kQChunkBytes);
+            mma_i8_ts(tmem + C::kDOff + db * C::kDCols + j * C::kN, tmem + ab * C::kACols + 8 * b, desc, idesc,
+                      false);
+          }
+          tc_commit(&dfull[db]);
+        }
+        if (!timed_out) tc_commit(&afree[ab]);
+      }
+      // every MMA this thread issued has completed before tensor memory goes
+      tc_commit(drain);
+      if (!mbar_wait(smem_u32(drain), 0, a.err, a.wait_limit)) timed_out = true;
+    }
+    __syncwarp();
+  } else if (warp < kUpdateWarp0) {
+    // ---------------- unpack: thread = row, A operand into tensor memory -----
+    const int quarter = warp & 3, r = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    for (int k = 0; k < n; ++k) {
+      const int ab = k & 1, sw = k % SW;
+      if (!mbar_wait(smem_u32(&wfull[sw]), (uint32_t)(k / SW) & 1u, a.err, a.wait_limit) ||
+          (k >= 2 && !mbar_wait(smem_u32(&afree[ab]), ((k >> 1) - 1) & 1u, a.err, a.wait_limit))) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const uint8_t* q = wring + sw * QB;
+      const uint32_t ta = tmem + lane_base + ab * C::kACols;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        uint32_t av[8];
+        if constexpr (QT == kQ4_0) {
+          q4_unpack(*reinterpret_cast<const uint4*>(q + q4_off(b, r)), av);
+        } else {
+          const uint4 w0 = *reinterpret_cast<const uint4*>(q + q8_off(b, 0, r));
+          const uint4 w1 = *reinterpret_cast<const uint4*>(q + q8_off(b, 1, r));
+          av[0] = w0.x; av[1] = w0.y; av[2] = w0.z; av[3] = w0.w;
+          av[4] = w1.x; av[5] = w1.y; av[6] = w1.z; av[7] = w1.w;
+        }
+        tmem_st8(ta + 8 * b, av);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&afull[ab]));
+        mbar_arrive(smem_u32(&wempty[sw]));
+      }
+    }
   } else {
-    int slot = 0;
-    uint32_t phase = 0;
-    gemv_consume<QT, NT, S>(a, cta, stages, bars, ts, slot, phase, tc, timed_out);
+    // ---------------- update: thread = row, f32 block updates, tile finish ---
+    const int quarter = warp & 3, r = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
+    for (int t = quarter; t < NT; t += 4) {
+      const float rs = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
+      if (lane == 0) rstd[t] = rs;
+    }
+    named_sync(kBarUpdate, 128);
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+    uint32_t gc = 0;
+    int tile = i0 / a.chunks;
+    for (int k = 0; k < n; ++k) {
+      const int item = i0 + k, sx = k % SX;
+      if (item / a.chunks != tile) {
+        gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, rstd, ex, flag, quarter, lane);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+        tile = item / a.chunks;
+      }
+      const uint8_t* xsl = xring + sx * XS;
+      uint4 sc4 = make_uint4(0, 0, 0, 0);
+      for (int g = 0; g < C::kNG; ++g, ++gc) {
+        const int db = gc & 1;
+        // the four warps share named barriers in the tile finish, so they
+        // decide together: all go on, or all stop
+        // (the first group also waits for the x slot itself: its scales and
+        // block metadata are read here, not only by the MMA)
+        const bool ok = mbar_wait(smem_u32(&dfull[db]), (gc >> 1) & 1u, a.err, a.wait_limit) &&
+                        (g > 0 || mbar_wait(smem_u32(&xfull[sx]), (uint32_t)(k / SX) & 1u, a.err, a.wait_limit));
+        if (!bar_and(kBarUpdate, 128, ok)) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
+        if (g == 0) sc4 = *reinterpret_cast<const uint4*>(xsl + r * 16);   // the row's 8 block scales
+        int dv[C::kGB][NT][4];
+#pragma unroll
+        for (int j = 0; j < C::kGB; ++j)
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            tmem_ld4(tmem + lane_base + C::kDOff + db * C::kDCols + j * C::kN + t * 8, dv[j][t]);
+        tmem_ld_wait();
+        const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+#pragma unroll
+        for (int j = 0; j < C::kGB; ++j) {
+          const int b = g * C::kGB + j;
+          const uint32_t w = scw[b >> 1];
+          const float d = __half2float(__ushort_as_half(static_cast<unsigned short>((b & 1) ? (w >> 16) : (w & 0xFFFFu))));
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const int4 m = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + t * kQChunkBytes +
+                                                          b * kQBlockBytes + kQMetaOff);
+            acc[t] = block_update<QT>(acc[t], d, __int_as_float(m.x), dv[j][t][0], dv[j][t][1], dv[j][t][2], m.y, m.z);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&dfree[db]));
+      }
+      if (timed_out) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&xempty[sx]));
+    }
+    if (!timed_out) gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, rstd, ex, flag, quarter, lane);
+  }
+  // ---------------- teardown: tensor memory back, after every MMA and load --
+  tc_fence_before();
+  named_sync(kBarTmem, kGemvCtaThreads - 32);
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
   }
   if (timed_out && lane == 0) drain_inflight_copies();   // error path
 }

@@ -92,13 +92,13 @@ struct stage {
   long long state_elems = 0;
   int committed = 0, pending_n = 0, pending_pos = 0;
   std::vector<int> cur;
-  cudaGraphExec_t exec[kMaxTok + 1] = {};
-  // persistent pass: per-layer step arguments on the device, grid-barrier counter
-  PassLayer* pass_layers = nullptr;
-  unsigned* bar = nullptr;
-  int n_phases = 0;
-  unsigned long long* trace = nullptr;   // [grid][n_phases][2], when tracing is on
-  int pass_mode = STAGE_PASS_KERNELS;
+  // one graph per (kind of pass, token count): kind 0 = forward (per-token
+  // snapshots), 1 = exact prefill, 2 = chunked prefill (DnMode)
+  cudaGraphExec_t exec[3][kMaxTok + 1] = {};
+  // failure injection for tests of the bounded waits (stage_debug_inject)
+  uint32_t dbg_wait_limit = 0;
+  int dbg_fault_item = -1;
+  int max_tiles = 0;
   size_t weight_bytes = 0;
   std::string last_error;
 };
@@ -140,8 +140,9 @@ stage_status dalloc_t(stage* st, T** p, size_t bytes) {
 void destroy(stage* st) {
   if (!st) return;
   if (st->stream || st->cap) cudaDeviceSynchronize();
-  for (auto& g : st->exec)
-    if (g) cudaGraphExecDestroy(g);
+  for (auto& row : st->exec)
+    for (auto& g : row)
+      if (g) cudaGraphExecDestroy(g);
   for (void* p : st->allocs) cudaFree(p);
   if (st->cap) cudaStreamDestroy(st->cap);
   delete st;
@@ -173,19 +174,29 @@ GemvArgs gemv_base(const stage* st) {
   a.err = st->err;
   a.eps = st->cfg.eps;
   a.inv_dim = 1.0f / (float)st->cfg.hidden;
+  a.wait_limit = st->dbg_wait_limit;
+  a.fault_item = -1;
   return a;
 }
 
-void set_workers(const stage* st, GemvArgs& a) { a.workers = gemv_workers(a.tiles, a.chunks, kCtasPerSm * st->sms); }
+void set_workers(const stage* st, GemvArgs& a) { a.workers = gemv_workers(a.tiles, a.chunks, st->sms); }
 
-// Arguments of every step of layer i (shared by both execution paths, so they
-// run the same units with the same split).
-PassLayer layer_args(const stage* st, size_t i) {
+// The steps of one layer: in-projection, out-projection, gate/up, down, and
+// the mixer between the first two.
+struct LayerSteps {
+  int attn;
+  GemvArgs g[4];
+  DnArgs dn;
+  AttnArgs at;
+};
+
+// Arguments of every step of layer i.
+LayerSteps layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
   const stage_config& c = st->cfg;
   const int H = c.hidden, F = c.ffn;
   const Layer& L = st->layers[i];
   const float* next_norm1 = i + 1 < st->layers.size() ? st->layers[i + 1].norm1 : nullptr;
-  PassLayer P = {};
+  LayerSteps P = {};
   P.attn = L.attn ? 1 : 0;
   // mixer in-projection with the RMSNorm1 scale folded into the epilogue
   GemvArgs a = gemv_base(st);
@@ -198,7 +209,7 @@ PassLayer layer_args(const stage* st, size_t i) {
   a.y_stride = st->y_stride;
   a.out_valid = L.in_rows;
   a.ss_in = st->ss;
-  a.ss_tiles = H / 64;
+  a.ss_tiles = H / kTileRows;
   a.ss_stride = st->ss_stride;
   set_workers(st, a);
   P.g[0] = a;
@@ -214,6 +225,7 @@ PassLayer layer_args(const stage* st, size_t i) {
     d.cur = st->ctrl + 1 + L.dn_slot;
     d.qo = st->qo;
     d.qo_stride = st->qo_stride;
+    d.mode = dn_mode;
   } else {
     AttnArgs& at = P.at;
     at.y = st->y;
@@ -263,7 +275,7 @@ PassLayer layer_args(const stage* st, size_t i) {
   a.qout = st->qu;
   a.qout_stride = st->qu_stride;
   a.ss_in = st->ss;
-  a.ss_tiles = H / 64;
+  a.ss_tiles = H / kTileRows;
   a.ss_stride = st->ss_stride;
   set_workers(st, a);
   P.g[2] = a;
@@ -291,15 +303,16 @@ PassLayer layer_args(const stage* st, size_t i) {
 
 // Record one pass of n tokens onto stream s (being captured) as a chain of
 // kernels: stage input, then per layer in-projection, mixer, out-projection,
-// gate/up, down.
-cudaError_t record_kernels(stage* st, int n, cudaStream_t s) {
+// gate/up, down.  Every kernel after the first is a programmatic dependent of
+// the one before.
+cudaError_t record_pass(stage* st, int n, int kind, cudaStream_t s) {
   const stage_config& c = st->cfg;
   const int qt = c.qtype;
   cudaError_t e = launch_stage_input(n, st->h, c.hidden, st->layers[0].norm1, st->qz, st->qz_stride, st->ss,
                                      st->ss_stride, s);
   if (e != cudaSuccess) return e;
   for (size_t i = 0; i < st->layers.size(); ++i) {
-    PassLayer P = layer_args(st, i);
+    LayerSteps P = layer_args(st, i, kind);
     // each projection warms L2 with the next one's first items
     auto chain = [](GemvArgs& a, const GemvArgs& next) {
       a.next_W = next.W;
@@ -310,6 +323,7 @@ cudaError_t record_kernels(stage* st, int n, cudaStream_t s) {
     chain(P.g[1], P.g[2]);
     chain(P.g[2], P.g[3]);
     if (i + 1 < st->layers.size()) chain(P.g[3], layer_args(st, i + 1).g[0]);
+    if (i == 0) P.g[0].fault_item = st->dbg_fault_item;   // injected failure (tests only)
     if ((e = launch_gemv(qt, n, EPI_STORE, P.g[0], P.g[0].workers, s, kUsePdl)) != cudaSuccess) return e;
     if (!P.attn) {
       if ((e = launch_dn_step(n, P.dn, c.dn_v_heads * (kDnDim / 32), s, kUsePdl)) != cudaSuccess) return e;
@@ -324,59 +338,9 @@ cudaError_t record_kernels(stage* st, int n, cudaStream_t s) {
   return cudaSuccess;
 }
 
-// Whether the n-token pass can run as one persistent kernel: n within the
-// instantiated range, two CTAs per SM resident, and the mixers' scratch within
-// the kernel's shared memory.
-bool pass_eligible(const stage* st, int n) {
-  if (n > kPassMaxTok || !st->pass_layers) return false;
-  const int qt = st->cfg.qtype;
-  int blocks = 0;
-  if (pass_occupancy(qt, n, &blocks) != cudaSuccess || blocks < 2) {
-    (void)cudaGetLastError();
-    return false;
-  }
-  const int rep = st->cfg.att_q_heads / st->cfg.att_kv_heads;
-  const int mix = pass_mix_bytes(qt, n);
-  const int need = std::max({n * 64 * 4, dn_smem_floats(n) * 4, st->nchunk * 3 * 4, st->nchunk ? attn_smem_bytes(std::min(n, kAttGroup), rep) : 0});
-  return need <= mix;
-}
-
-// Record one pass of n tokens as one cooperative persistent kernel (pass.cuh)
-// after zeroing its grid-barrier counter.
-cudaError_t record_persistent(stage* st, int n, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(st->bar, 0, sizeof(unsigned), s);
-  if (e != cudaSuccess) return e;
-  const stage_config& c = st->cfg;
-  PassArgs p = {};
-  p.layers = st->pass_layers;
-  p.n_layers = (int)st->layers.size();
-  p.h = st->h;
-  p.H = c.hidden;
-  p.gamma0 = st->layers[0].norm1;
-  p.qz = st->qz;
-  p.qz_stride = st->qz_stride;
-  p.ss = st->ss;
-  p.ss_stride = st->ss_stride;
-  p.kv_len = st->ctrl;
-  p.bar = st->bar;
-  p.grid = kCtasPerSm * st->sms;
-  p.dn_units = c.dn_v_heads * (kDnDim / 32);
-  p.Hq = c.att_q_heads;
-  p.Hkv = c.att_kv_heads;
-  p.err = st->err;
-  p.trace = st->trace;
-  p.n_phases = st->n_phases;
-  return launch_pass(c.qtype, n, p, s);
-}
-
-cudaError_t record_pass(stage* st, int n, cudaStream_t s) {
-  if (st->pass_mode == STAGE_PASS_PERSISTENT && pass_eligible(st, n)) return record_persistent(st, n, s);
-  return record_kernels(st, n, s);
-}
-
-stage_status build_graph(stage* st, int n) {
+stage_status build_graph(stage* st, int n, int kind) {
   CK(cudaStreamBeginCapture(st->cap, cudaStreamCaptureModeThreadLocal));
-  cudaError_t e = record_pass(st, n, st->cap);
+  cudaError_t e = record_pass(st, n, kind, st->cap);
   cudaGraph_t g = nullptr;
   cudaError_t e2 = cudaStreamEndCapture(st->cap, &g);
   if (e != cudaSuccess || e2 != cudaSuccess) {
@@ -388,7 +352,7 @@ stage_status build_graph(stage* st, int n) {
   e = cudaGraphInstantiate(&ex, g, 0);
   cudaGraphDestroy(g);
   if (e != cudaSuccess) return fail(st, STAGE_E_CUDA, cuda_msg("cudaGraphInstantiate", e));
-  st->exec[n] = ex;
+  st->exec[kind][n] = ex;
   return STAGE_OK;
 }
 
@@ -567,7 +531,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
   // --- activations and scratch --------------------------------------------
   const int y_rows = std::max(dn_in, at_in);
   st->y_stride = (y_rows + 63) / 64 * 64;
-  st->ss_stride = H / 64;
+  st->ss_stride = H / kTileRows;
   st->qz_stride = (int)qact_row_bytes(H);
   st->qo_stride = (int)qact_row_bytes(std::max(dn_o, at_o));
   st->qu_stride = (int)qact_row_bytes(F);
@@ -588,8 +552,9 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     if ((e = launch_rope_table(st->rope, c.max_ctx, c.rope_dims, c.rope_theta, nullptr)) != cudaSuccess)
       return bail(fail(st, STAGE_E_CUDA, cuda_msg("rope table", e)));
   }
-  const int max_tiles = std::max({packed_tiles(y_rows, false), packed_tiles(F, true), H / 64});
-  if ((s = dalloc_t(st, &st->partials, (size_t)2 * kCtasPerSm * st->sms * kMaxTok * 64 * 4)) != STAGE_OK ||
+  const int max_tiles = std::max({packed_tiles(y_rows, false), packed_tiles(F, true), H / kTileRows});
+  st->max_tiles = max_tiles;
+  if ((s = dalloc_t(st, &st->partials, (size_t)2 * st->sms * kMaxTok * kTileRows * 4)) != STAGE_OK ||
       (s = dalloc_t(st, &st->counters, (size_t)max_tiles * 4)) != STAGE_OK ||
       (s = dalloc_t(st, &st->err, 16)) != STAGE_OK ||
       (s = dalloc_t(st, &st->ctrl, (size_t)(1 + st->n_dn) * 4)) != STAGE_OK)
@@ -601,38 +566,20 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
   st->cur.assign(st->n_dn, 0);
 
-  // --- persistent pass: step arguments of every layer, phase numbering -------
-  if ((e = pass_prepare(qt)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("pass_prepare", e)));
-  {
-    std::vector<PassLayer> pl(st->layers.size());
-    int phase = 1;   // phase 0: stage input
-    for (size_t i = 0; i < pl.size(); ++i) {
-      pl[i] = layer_args(st, i);
-      pl[i].phase_in = phase;
-      phase += pl[i].attn ? 6 : 5;   // in-proj, mixer (attention: partials + combine), out, gate/up, down
-    }
-    st->n_phases = phase;
-    if ((s = dalloc_t(st, &st->pass_layers, pl.size() * sizeof(PassLayer))) != STAGE_OK ||
-        (s = dalloc_t(st, &st->bar, 16)) != STAGE_OK)
-      return bail(s);
-    if ((e = cudaMemcpy(st->pass_layers, pl.data(), pl.size() * sizeof(PassLayer), cudaMemcpyHostToDevice)) !=
-        cudaSuccess)
-      return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemcpy pass layers", e)));
-  }
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("load sync", e)));
   *out = st;
   return STAGE_OK;
 }
 
 // Checks shared by both forward entries; builds the n_tok graph on first use.
-static stage_status forward_begin(stage_t* st, const void* hidden_dev, int n_tok, int pos) {
+static stage_status forward_begin(stage_t* st, const void* hidden_dev, int n_tok, int pos, int kind = DN_SNAPSHOTS) {
   if (!st) return STAGE_E_ARG;
   if (!hidden_dev) return fail(st, STAGE_E_ARG, "hidden buffer is NULL");
   if (n_tok < 1 || n_tok > kMaxTok) return fail(st, STAGE_E_ARG, "n_tok must be in 1..16");
   if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending: commit or roll back first");
   if (pos != st->committed) return fail(st, STAGE_E_STATE, "pos must equal the committed length");
   if (pos + n_tok > st->cfg.max_ctx) return fail(st, STAGE_E_ARG, "pass would overflow max_ctx");
-  if (!st->exec[n_tok]) return build_graph(st, n_tok);
+  if (!st->exec[kind][n_tok]) return build_graph(st, n_tok, kind);
   return STAGE_OK;
 }
 
@@ -641,7 +588,7 @@ stage_status stage_forward(stage_t* st, float* hidden_dev, int n_tok, int pos) {
   if (s != STAGE_OK) return s;
   const size_t bytes = (size_t)n_tok * st->cfg.hidden * 4;
   CK(cudaMemcpyAsync(st->h, hidden_dev, bytes, cudaMemcpyDeviceToDevice, st->stream));
-  CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
+  CK(cudaGraphLaunch(st->exec[DN_SNAPSHOTS][n_tok], st->stream));
   CK(cudaMemcpyAsync(hidden_dev, st->h, bytes, cudaMemcpyDeviceToDevice, st->stream));
   st->pending_n = n_tok;
   st->pending_pos = pos;
@@ -655,7 +602,7 @@ stage_status stage_forward_host(stage_t* st, const float* hidden_in_host, float*
   if (s != STAGE_OK) return s;
   const size_t bytes = (size_t)n_tok * st->cfg.hidden * 4;
   CK(cudaMemcpyAsync(st->h, hidden_in_host, bytes, cudaMemcpyHostToDevice, st->stream));
-  CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
+  CK(cudaGraphLaunch(st->exec[DN_SNAPSHOTS][n_tok], st->stream));
   CK(cudaMemcpyAsync(hidden_out_host, st->h, bytes, cudaMemcpyDeviceToHost, st->stream));
   st->pending_n = n_tok;
   st->pending_pos = pos;
@@ -668,10 +615,28 @@ stage_status stage_forward_f16(stage_t* st, void* hidden_dev, int n_tok, int pos
   if (s != STAGE_OK) return s;
   const int n = n_tok * st->cfg.hidden;
   CK(launch_hidden_from_f16(hidden_dev, st->h, n, st->stream));
-  CK(cudaGraphLaunch(st->exec[n_tok], st->stream));
+  CK(cudaGraphLaunch(st->exec[DN_SNAPSHOTS][n_tok], st->stream));
   CK(launch_hidden_to_f16(st->h, hidden_dev, n, st->stream));
   st->pending_n = n_tok;
   st->pending_pos = pos;
+  return STAGE_OK;
+}
+
+stage_status stage_prefill(stage_t* st, float* hidden_dev, int n_tok, int pos, int mode) {
+  if (st && mode != STAGE_PREFILL_EXACT && mode != STAGE_PREFILL_CHUNKED)
+    return fail(st, STAGE_E_ARG, "mode must be STAGE_PREFILL_EXACT or STAGE_PREFILL_CHUNKED");
+  const int kind = mode == STAGE_PREFILL_CHUNKED ? DN_CHUNKED : DN_FINAL;
+  stage_status s = forward_begin(st, hidden_dev, n_tok, pos, kind);
+  if (s != STAGE_OK) return s;
+  const size_t bytes = (size_t)n_tok * st->cfg.hidden * 4;
+  CK(cudaMemcpyAsync(st->h, hidden_dev, bytes, cudaMemcpyDeviceToDevice, st->stream));
+  CK(cudaGraphLaunch(st->exec[kind][n_tok], st->stream));
+  CK(cudaMemcpyAsync(hidden_dev, st->h, bytes, cudaMemcpyDeviceToDevice, st->stream));
+  // the chunk is committed whole: each DeltaNet layer's final state sits in
+  // ring slot (cur + n_tok), the slot commit(n_tok) selects
+  CK(launch_commit(st->ctrl, n_tok, st->n_dn, kRing, st->stream));
+  st->committed = pos + n_tok;
+  for (int& v : st->cur) v = (v + n_tok) % kRing;
   return STAGE_OK;
 }
 
@@ -705,7 +670,10 @@ stage_status stage_sync(stage_t* st) {
   unsigned err = 0;
   CK(cudaMemcpy(&err, st->err, sizeof(err), cudaMemcpyDeviceToHost));
   if (err) {
+    // a kernel that gave up may have left stream-K tile counters part-way:
+    // clear them with the error word, so the next pass starts clean
     CK(cudaMemset(st->err, 0, sizeof(err)));
+    CK(cudaMemset(st->counters, 0, (size_t)st->max_tiles * sizeof(int)));
     return fail(st, STAGE_E_DEVICE, "device error word " + std::to_string(err) + " (bounded wait timed out)");
   }
   return STAGE_OK;
@@ -808,60 +776,28 @@ stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float
   return STAGE_OK;
 }
 
-stage_status stage_set_pass_mode(stage_t* st, int mode) {
-  if (!st) return STAGE_E_ARG;
-  if (mode != STAGE_PASS_KERNELS && mode != STAGE_PASS_PERSISTENT) return fail(st, STAGE_E_ARG, "unknown pass mode");
-  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
-  if (mode == st->pass_mode) return STAGE_OK;
+// Drop every recorded graph (the next forward of each token count records
+// it again with the current settings).
+static stage_status drop_graphs(stage_t* st) {
   CK(cudaStreamSynchronize(st->stream));
-  for (auto& g : st->exec)
-    if (g) {
-      CK(cudaGraphExecDestroy(g));
-      g = nullptr;
-    }
-  st->pass_mode = mode;
+  for (auto& row : st->exec)
+    for (auto& g : row)
+      if (g) {
+        CK(cudaGraphExecDestroy(g));
+        g = nullptr;
+      }
   return STAGE_OK;
 }
 
-stage_status stage_set_trace(stage_t* st, int enable) {
+stage_status stage_debug_inject(stage_t* st, int fault_item, unsigned wait_limit) {
   if (!st) return STAGE_E_ARG;
   if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
-  if ((enable != 0) == (st->trace != nullptr)) return STAGE_OK;
-  CK(cudaStreamSynchronize(st->stream));
-  for (auto& g : st->exec)
-    if (g) {
-      CK(cudaGraphExecDestroy(g));
-      g = nullptr;
-    }
-  if (enable) {
-    const size_t bytes = (size_t)kCtasPerSm * st->sms * st->n_phases * 2 * sizeof(unsigned long long);
-    stage_status s = dalloc_t(st, &st->trace, bytes);
-    if (s != STAGE_OK) return s;
-    CK(cudaMemset(st->trace, 0, bytes));
-  } else {
-    cudaFree(st->trace);
-    st->allocs.erase(std::remove(st->allocs.begin(), st->allocs.end(), (void*)st->trace), st->allocs.end());
-    st->trace = nullptr;
-  }
+  if (fault_item < -1) return fail(st, STAGE_E_ARG, "fault_item must be -1 or a local item index");
+  stage_status s = drop_graphs(st);
+  if (s != STAGE_OK) return s;
+  st->dbg_fault_item = fault_item;
+  st->dbg_wait_limit = wait_limit;
   return STAGE_OK;
-}
-
-stage_status stage_get_trace(stage_t* st, unsigned long long* host_dst, size_t count, int* grid, int* n_phases) {
-  if (!st) return STAGE_E_ARG;
-  if (!st->trace) return fail(st, STAGE_E_STATE, "tracing is off");
-  const size_t need = (size_t)kCtasPerSm * st->sms * st->n_phases * 2;
-  if (grid) *grid = kCtasPerSm * st->sms;
-  if (n_phases) *n_phases = st->n_phases;
-  if (!host_dst) return STAGE_OK;
-  if (count != need) return fail(st, STAGE_E_ARG, "count must be grid * n_phases * 2");
-  CK(cudaStreamSynchronize(st->stream));
-  CK(cudaMemcpy(host_dst, st->trace, need * sizeof(unsigned long long), cudaMemcpyDeviceToHost));
-  return STAGE_OK;
-}
-
-int stage_pass_persistent(stage_t* st, int n_tok) {
-  if (!st || n_tok < 1 || n_tok > kMaxTok) return -1;
-  return st->pass_mode == STAGE_PASS_PERSISTENT && pass_eligible(st, n_tok) ? 1 : 0;
 }
 
 size_t stage_weight_bytes(const stage_t* st) { return st ? st->weight_bytes : 0; }

@@ -12,12 +12,12 @@ TOL = 2e-3   # max relative error per output vector / per DeltaNet head state
 def gemv_error_bound(qtype, W, x):
     """Per-output bound on |y_gpu - y| for y = x W^T, derived from the arithmetic.
 
-    The CUDA GEMV carries x in 24-bit block fixed point: per token and 32-column
-    block, s = 2^(E - 22) with 2^E <= max |x| < 2^(E + 1), so an element is off
-    by at most one unit s (half a unit from rounding, one where the top code is
-    clamped).  Block sums over the integer codes are exact; turning a block's
-    sums into f32 takes two roundings, adding it to the accumulator one more,
-    and the warp, stream-K and epilogue sums a few more, each at most 2^-24 of
+    The CUDA GEMV carries x in block fixed point: per token and 32-column
+    block, s = 2^(E - 21) with 2^E <= max |x| < 2^(E + 1), so an element is off
+    by at most one unit s (half a unit from rounding; the codes never reach the
+    clamp at 2^22).  Block sums over the integer codes are exact; turning a
+    block's sums into f32 takes two roundings, adding it to the accumulator one
+    more, and the stream-K and epilogue sums a few more, each at most 2^-24 of
     the magnitudes involved.  Bound per output:
         sum_j |W_j| s_j + (blocks + 8) 2^-23 sum_j |W_j| (|x_j| + s_j).
     """
@@ -28,7 +28,7 @@ def gemv_error_bound(qtype, W, x):
     m = np.abs(x).reshape(n, cols // 32, 32).max(axis=2)         # block maxima
     E = np.frexp(m)[1] - 1                                        # 2^E <= m < 2^(E+1)
     E = np.where(m > 0, np.maximum(E, -100), -100)
-    step = np.repeat(np.ldexp(1.0, E - 22), 32, axis=1)          # [n, cols]
+    step = np.repeat(np.ldexp(1.0, E - 21), 32, axis=1)          # [n, cols]
     return step @ A.T + (cols // 32 + 8) * 2.0 ** -23 * ((np.abs(x) + step) @ A.T)
 
 

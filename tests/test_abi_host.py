@@ -66,13 +66,14 @@ def test_library_exports_every_declared_symbol(qhl):
 
 
 def test_packed_bytes_geometry(qhl):
-    # Q4_0 item: 64 rows x 256 cols in 9216 bytes; Q8_0: 17408 bytes
-    assert qhl.qhl_packed_bytes(2, 64, 256) == 9216
-    assert qhl.qhl_packed_bytes(8, 64, 256) == 17408
-    assert qhl.qhl_packed_bytes(2, 1024, 1024) == 16 * 4 * 9216
-    assert qhl.qhl_packed_bytes(2, 10336, 5120) == 162 * 20 * 9216       # ragged rows pad to 64
-    assert qhl.qhl_packed_bytes(2, 17408, 5120, paired=True) == 544 * 20 * 9216
-    # packed bytes equal GGUF bytes whenever rows are a multiple of 64
+    # Q4_0 item: 128 rows x 256 cols in 18432 bytes; Q8_0: 34816 bytes
+    assert qhl.qhl_packed_bytes(2, 128, 256) == 18432
+    assert qhl.qhl_packed_bytes(8, 128, 256) == 34816
+    assert qhl.qhl_packed_bytes(2, 64, 256) == 18432                        # a short tile pads to 128 rows
+    assert qhl.qhl_packed_bytes(2, 1024, 1024) == 8 * 4 * 18432
+    assert qhl.qhl_packed_bytes(2, 10336, 5120) == 81 * 20 * 18432       # ragged rows pad to 128
+    assert qhl.qhl_packed_bytes(2, 17408, 5120, paired=True) == 272 * 20 * 18432
+    # packed bytes equal GGUF bytes whenever rows are a multiple of 128
     assert qhl.qhl_packed_bytes(2, 5120, 17408) == 5120 * 17408 // 32 * 18
     assert qhl.qhl_packed_bytes(8, 5120, 6144) == 5120 * 6144 // 32 * 34
     assert qhl.qhl_packed_bytes(2, 64, 100) == 0                            # cols % 256

@@ -31,9 +31,8 @@ def test_pass_bytes_of_the_64_layer_stage():
 def test_launches_per_pass():
     # stage input, then per layer in-proj, mixer (DeltaNet step | attention
     # partials + combine), out-proj, gate/up, down
-    assert bench.launches_per_pass(FULL, range(64), persistent=False) == 1 + 48 * 5 + 16 * 6 == 337
-    assert bench.launches_per_pass(FULL, range(0, 4), persistent=False) == 1 + 3 * 5 + 6
-    assert bench.launches_per_pass(FULL, range(64), persistent=True) == 1
+    assert bench.launches_per_pass(FULL, range(64)) == 1 + 48 * 5 + 16 * 6 == 337
+    assert bench.launches_per_pass(FULL, range(0, 4)) == 1 + 3 * 5 + 6
 
 
 class _FakeSmi:
@@ -58,7 +57,25 @@ def test_clock_record_median_max_and_reasons():
     r = s.stop()
     assert r["sm_mhz"] == 1950 and r["sm_max_mhz"] == 1965 and r["samples"] == 3
     assert r["reasons"] == ["sw_power_cap"]
-    assert bench.ClockSampler(0).stop()["reasons"] == ["nvidia-smi unavailable"]
+    assert bench.ClockSampler(0).stop()["reasons"] == ["clock sampling unavailable"]
+
+
+def test_clock_record_from_nvml_samples():
+    s = bench.ClockSampler(0)
+
+    class _Done:
+        def set(self):
+            pass
+
+    class _Thread:
+        def join(self, timeout=None):
+            pass
+
+    s.thread, s.stop_ev, s.max_mhz = _Thread(), _Done(), 1965.0
+    s.samples = [(1965.0, set()), (1440.0, {"sw_power_cap"}), (1950.0, set()), (1960.0, {"hw_slowdown"})]
+    r = s.stop()
+    assert r["sm_mhz"] == 1955.0 and r["sm_max_mhz"] == 1965.0 and r["samples"] == 4
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
 
 
 def test_traffic_is_reported_only_for_the_sources_it_was_measured_on(monkeypatch):

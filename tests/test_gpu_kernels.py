@@ -55,8 +55,8 @@ def test_single_q4_0_gemv_1024(q):
     err = rel_err_rows(y, ref)
     assert max(err) <= TOL, err
     assert np.all(np.abs(y - ref) <= gemv_error_bound(Q4_0, W, x))
-    # x enters as 24-bit block fixed point (step <= 2^-22 of the block max): the
-    # error stays far inside the bound
+    # x enters as block fixed point (step <= 2^-21 of the block max): the error
+    # stays far inside the bound
     assert max(err) <= 2e-4
 
 
@@ -77,8 +77,9 @@ def test_gemv_batched_is_bit_identical_to_single_tokens(q, qtype):
     rows, cols = 1500, 2304
     W, x = synth.gemv_problem(21, rows, cols, 16, qtype)
     P = packed_on_gpu(q, qtype, W)
-    # n >= 4 runs the integer tensor-core path, n < 4 the dp4a path: both form
-    # the same exact block sums, so every n equals the single-token results
+    # every n forms the same exact integer block sums on the tensor cores (MMA
+    # N = 8 rows per token) and the same f32 updates, so every n equals the
+    # single-token results
     for n in (16, 9, 8, 7, 5, 4, 3, 2):
         yb = gemv_gpu(q, qtype, P, rows, cols, x[:n])
         for t in range(n):
@@ -184,3 +185,27 @@ def test_deltanet_batched_equals_sequential_and_rollback_prefix(q):
     j = synth.accepted_prefix(1, 0, n)
     kept = S0 if j == 0 else snaps_b[j - 1]
     assert np.array_equal(kept, seq[j])
+
+
+def test_qgemv_wait_that_runs_out_is_reported_by_qhl_sync(q):
+    """qhl_debug_inject makes CTA 0 skip one item of the next qhl_qgemv calls
+    with every wait capped short: the call returns, qhl_sync raises
+    STAGE_E_DEVICE once (clearing the error word and the tile counters), and
+    with injection off the next call gives the reference bits again."""
+    import torch
+    rows, cols = 1000, 5120
+    W, x = synth.gemv_problem(71, rows, cols, 1)
+    P = packed_on_gpu(q, Q4_0, W)
+    ref = gemv_gpu(q, Q4_0, P, rows, cols, x)
+    q.qhl_sync()
+    try:
+        q.qhl_debug_inject(0, 4096)
+        gemv_gpu(q, Q4_0, P, rows, cols, x)
+        with pytest.raises(q.StageError) as e:
+            q.qhl_sync()
+        assert e.value.code == -7
+        q.qhl_sync()
+    finally:
+        q.qhl_debug_inject(-1, 0)
+    assert np.array_equal(gemv_gpu(q, Q4_0, P, rows, cols, x), ref)
+    q.qhl_sync()

@@ -2,12 +2,15 @@
 
 * one hybrid stage of 4 layers (DeltaNet, DeltaNet, DeltaNet, attention) at
   hidden 5120, Q4_0, n_tok 1 from cached position 4096 (seed 2),
-* speculative verify passes of 4 and 16 tokens from position 4096 with a seeded
-  accepted prefix, commit and rollback, Q4_0 and Q8_0 (seed 3): batched output
-  bit-identical to sequential decoding, post-commit state bit-identical to the
-  sequential state at that prefix, rollback restoring the state exactly,
+* speculative verify passes of 4 and 16 tokens (and 5, 7, 13) from position
+  4096 with a seeded accepted prefix, commit and rollback, Q4_0 and Q8_0
+  (seed 3): batched output bit-identical to sequential decoding, post-commit
+  state bit-identical to the sequential state at that prefix, rollback
+  restoring the state exactly,
 * split equals whole (layers [0,4) = [0,2) then [2,4)),
-* protocol and format errors leave the stage unchanged.
+* the f16 boundary against the oracle and against the f32 pass,
+* protocol and format errors leave the stage unchanged; a bounded wait that is
+  made to run out is reported and the stage recovers.
 """
 import numpy as np
 import pytest
@@ -95,7 +98,11 @@ def _states(st, begin, end):
     return {l: st.get_dn_state(l) for l in dn_layers(begin, end)}
 
 
-@pytest.mark.parametrize("qtype,n", [(Q4_0, 4), (Q4_0, 16), (Q8_0, 4)])
+# 4 and 16 draft tokens (config 4), Q8_0 at both, and the ragged counts 5, 7
+# and 13 (a partial last attention group of 4, and 8-token MMA groups that a
+# 16-token pass pads)
+@pytest.mark.parametrize("qtype,n", [(Q4_0, 4), (Q4_0, 16), (Q8_0, 4), (Q8_0, 16), (Q4_0, 5), (Q4_0, 7),
+                                     (Q4_0, 13)])
 def test_verify_pass_commit_and_rollback(q, qtype, n):
     seed = 3
     st, orc, _ = make_pair(FULL, qtype, seed, 0, 4, MAX_CTX, CTX)
@@ -235,80 +242,6 @@ def test_load_rejects_missing_or_misshaped_tensors(q):
     st.free()
 
 
-@pytest.mark.parametrize("qtype,ns", [(Q4_0, (1, 2, 3, 4)), (Q8_0, (1, 3))])
-def test_persistent_pass_equals_kernel_chain(q, qtype, ns):
-    """The one-kernel persistent pass and the chain of per-step kernels run the
-    same units with the same split: outputs and committed states are
-    bit-identical."""
-    import torch
-    seed = 7
-    st, _, _ = make_pair(FULL, qtype, seed, 0, 4, MAX_CTX, CTX, with_oracle=False)
-    try:
-        assert not st.pass_persistent(1)                      # the chain of kernels by default
-        assert not st.pass_persistent(16)
-        S0 = _states(st, 0, 4)
-        kv0 = {l: st.get_kv(l) for l in attn_layers(0, 4)}
-        for n in ns:
-            st.set_pass_mode(q.PASS_PERSISTENT)
-            assert st.pass_persistent(n), n
-            h = synth.hidden(FULL, seed, n, n)
-            res = {}
-            for mode in (q.PASS_PERSISTENT, q.PASS_KERNELS):
-                st.set_pass_mode(mode)
-                out = run(st, h, CTX)
-                st.commit(n)
-                res[mode] = (out, _states(st, 0, 4), {l: st.get_kv(l) for l in attn_layers(0, 4)})
-                for l, S in S0.items():                       # back to the starting state
-                    st.set_dn_state(l, S)
-                for l, (K, V) in kv0.items():
-                    st.set_kv(l, K, V)
-                st.set_kv_len(CTX)
-            out_p, S_p, kv_p = res[q.PASS_PERSISTENT]
-            out_k, S_k, kv_k = res[q.PASS_KERNELS]
-            assert np.array_equal(out_p, out_k), n
-            for l in S_p:
-                assert np.array_equal(S_p[l], S_k[l]), (n, l)
-            for l in kv_p:
-                assert np.array_equal(kv_p[l][0], kv_k[l][0]) and np.array_equal(kv_p[l][1], kv_k[l][1]), (n, l)
-        st.set_pass_mode(q.PASS_PERSISTENT)
-        st.forward(torch.zeros((1, FULL.hidden), device="cuda"), CTX)
-        with pytest.raises(q.StageError) as e:
-            st.set_pass_mode(q.PASS_KERNELS)          # refused while a pass is pending
-        assert e.value.code == -2
-        st.rollback()
-        with pytest.raises(q.StageError) as e:
-            st.set_pass_mode(5)
-        assert e.value.code == -1
-    finally:
-        st.free()
-
-
-def test_persistent_pass_trace_shows_the_grid_barriers(q):
-    """With tracing on, every CTA records each phase; no CTA starts a phase
-    before every CTA has finished the previous one (the grid barrier)."""
-    st, _, _ = make_pair(FULL, Q4_0, 8, 0, 4, MAX_CTX, CTX, with_oracle=False)
-    try:
-        with pytest.raises(q.StageError):
-            st.get_trace()                                   # off by default
-        st.set_pass_mode(q.PASS_PERSISTENT)
-        st.set_trace(True)
-        h = synth.hidden(FULL, 8, 0, 1)
-        run(st, h, CTX)
-        st.rollback()
-        tr = st.get_trace().astype(np.int64)
-        grid, n_phases, _ = tr.shape
-        assert n_phases == 1 + 3 * 5 + 6                      # input, 3 DeltaNet layers, 1 attention layer
-        assert (tr > 0).all()
-        assert (tr[:, :, 1] >= tr[:, :, 0]).all()
-        for ph in range(1, n_phases):
-            assert tr[:, ph, 0].min() >= tr[:, ph - 1, 1].max(), ph
-        st.set_trace(False)
-        run(st, h, CTX)                                       # still runs without the trace buffer
-        st.rollback()
-    finally:
-        st.free()
-
-
 def test_zero_weight_stage_is_the_identity(q):
     """All quants at the Q4_0 zero point (nibble 8): every projection is 0, so
     each layer adds exact zeros and the stage returns its input bit for bit
@@ -392,3 +325,136 @@ def test_forward_from_host_buffers_equals_the_device_pass(q, stage3):
     st.rollback()
     assert np.array_equal(hp.numpy(), ref)
     assert st.committed_len == pos
+
+
+def test_f16_boundary_matches_the_oracle(q, stage3):
+    """The wire form end to end against the oracle: the oracle runs the same
+    layers on the f16 input values and its f64 output, rounded once to f16, is
+    what the f16 entry must return within the tolerance (rounding to f16 adds
+    at most 2^-11 relative, inside 2e-3)."""
+    import torch
+    st, orc, _ = stage3
+    pos = st.committed_len
+    h16 = synth.hidden(FULL, 14, 0, 2).astype(np.float16)
+    x16 = torch.from_numpy(h16.copy()).cuda()
+    st.forward_f16(x16, pos)
+    torch.cuda.synchronize()
+    st.sync()
+    got = x16.cpu().numpy().astype(np.float64)
+    st.rollback()
+    ref = orc.forward(h16.astype(np.float64), pos)
+    orc.rollback()
+    assert np.isfinite(got).all()
+    assert max(rel_err_rows(got, ref.astype(np.float16).astype(np.float64))) <= TOL
+    assert max(rel_err_rows(got, ref)) <= TOL
+    assert st.committed_len == pos
+
+
+def test_a_wait_that_runs_out_is_reported_and_the_stage_recovers(q):
+    """Failure detection without a GPU fault.  stage_debug_inject makes CTA 0
+    of the first in-projection skip one item's quants, with every GEMV wait
+    capped at a few thousand iterations: that wait runs out, every kernel of
+    the pass still finishes, stage_sync reports STAGE_E_DEVICE once, and after
+    rollback, with injection off, the next pass gives the reference bits."""
+    import torch
+    seed = 13
+    st, _, _ = make_pair(FULL, Q4_0, seed, 0, 4, MAX_CTX, CTX, with_oracle=False)
+    try:
+        h = synth.hidden(FULL, seed, 0, 2)
+        ref = run(st, h, CTX)
+        st.rollback()
+        S0 = _states(st, 0, 4)
+        st.debug_inject(fault_item=1, wait_limit=4096)
+        x = torch.from_numpy(h.copy()).cuda()
+        st.forward(x, CTX)
+        with pytest.raises(q.StageError) as e:
+            st.sync()
+        assert e.value.code == -7                               # STAGE_E_DEVICE
+        st.sync()                                               # reported once, then cleared
+        st.rollback()
+        for l, S in _states(st, 0, 4).items():                  # the committed state is untouched
+            assert np.array_equal(S, S0[l])
+        with pytest.raises(q.StageError) as e:
+            st.debug_inject(fault_item=-2)
+        assert e.value.code == -1
+        st.debug_inject(-1, 0)
+        out = run(st, h, CTX)
+        assert np.array_equal(out, ref)
+        st.rollback()
+    finally:
+        st.free()
+
+
+def _prefill(st, h, pos, chunked):
+    import torch
+    x = torch.from_numpy(np.ascontiguousarray(h, dtype=np.float32)).cuda()
+    st.prefill(x, pos, chunked=chunked)
+    torch.cuda.synchronize()
+    st.sync()
+    return x.cpu().numpy()
+
+
+@pytest.mark.parametrize("n", [5, 16])
+def test_exact_prefill_equals_forward_and_commit(q, n):
+    """stage_prefill(EXACT) keeps only each DeltaNet layer's final state but
+    runs the same arithmetic: output, committed states and KV rows are those of
+    stage_forward + stage_commit(n), bit for bit, and nothing is pending."""
+    seed = 15
+    st, _, _ = make_pair(FULL, Q4_0, seed, 0, 4, MAX_CTX, CTX, with_oracle=False)
+    try:
+        S0 = _states(st, 0, 4)
+        kv0 = {l: st.get_kv(l) for l in attn_layers(0, 4)}
+        h = synth.hidden(FULL, seed, n, n)
+        ref = run(st, h, CTX)
+        st.commit(n)
+        S_ref = _states(st, 0, 4)
+        kv_ref = {l: st.get_kv(l) for l in attn_layers(0, 4)}
+        for l, S in S0.items():
+            st.set_dn_state(l, S)
+        for l, (K, V) in kv0.items():
+            st.set_kv(l, K, V)
+        st.set_kv_len(CTX)
+        got = _prefill(st, h, CTX, chunked=False)
+        assert np.array_equal(got, ref)
+        assert st.committed_len == CTX + n and st.pending == 0
+        for l, S in _states(st, 0, 4).items():
+            assert np.array_equal(S, S_ref[l]), l
+        for l in attn_layers(0, 4):
+            K, V = st.get_kv(l)
+            assert np.array_equal(K[:, :CTX + n], kv_ref[l][0][:, :CTX + n])
+            assert np.array_equal(V[:, :CTX + n], kv_ref[l][1][:, :CTX + n])
+        with pytest.raises(q.StageError) as e:
+            _prefill(st, h, CTX, chunked=False)          # pos must be the committed length
+        assert e.value.code == -2
+    finally:
+        st.free()
+
+
+@pytest.mark.parametrize("qtype,n", [(Q4_0, 16), (Q8_0, 16), (Q4_0, 7)])
+def test_chunked_prefill_matches_oracle(q, qtype, n):
+    """stage_prefill(CHUNKED): the chunked closed form of the DeltaNet
+    recurrence for a prompt chunk, against the oracle's token-by-token steps:
+    every hidden vector, every DeltaNet head state and the new KV rows within
+    the tolerance; decoding then continues from the committed chunk."""
+    seed = 16
+    st, orc, _ = make_pair(FULL, qtype, seed, 0, 4, MAX_CTX, CTX)
+    try:
+        h = synth.hidden(FULL, seed, 300 + n, n)
+        got = _prefill(st, h, CTX, chunked=True)
+        ref = orc.forward(h, CTX)
+        orc.commit(n)
+        assert max(rel_err_rows(got, ref)) <= TOL
+        assert st.committed_len == CTX + n and st.pending == 0
+        for l in dn_layers(0, 4):
+            assert max(rel_err_heads(st.get_dn_state(l), orc.S[l])) <= TOL, l
+        for l in attn_layers(0, 4):
+            K, V = st.get_kv(l)
+            for X, R in ((K, orc.K[l]), (V, orc.V[l])):
+                for p in range(CTX, CTX + n):
+                    assert max(rel_err_rows(X[:, p].astype(np.float64), R[:, p].astype(np.float64))) <= TOL
+        h2 = synth.hidden(FULL, seed, 400 + n, 1)
+        got2 = run(st, h2, CTX + n)
+        assert max(rel_err_rows(got2, orc.forward(h2, CTX + n))) <= TOL
+        st.rollback()
+    finally:
+        st.free()

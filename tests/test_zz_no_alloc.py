@@ -24,8 +24,9 @@ def test_noalloc_rejects_problems_beyond_its_static_scratch():
     from quantized_hybrid_layer_b200 import build as b
     b.build()
     lib = q.lib()
-    # 16 tokens x 20480 columns need 1.05 MiB of input scratch (limit 1 MiB): refused before any device work
-    assert lib.qhl_qgemv_noalloc(2, 64, 20480, 16, 16, 16, 16, None) == -1
+    # 16 tokens x 18688 columns need 73 chunks x 2048 bytes x 16 = 2.28 MiB of input
+    # scratch, one chunk past the 2.25 MiB region: refused before any device work
+    assert lib.qhl_qgemv_noalloc(2, 64, 18688, 16, 16, 16, 16, None) == -1
     assert b"exceeds" in lib.qhl_last_error()
     assert lib.qhl_qgemv_noalloc(2, 64, 256, None, None, 1, None, None) == -1
 
@@ -43,7 +44,10 @@ def test_noalloc_gemv_matches_the_regular_entry_point_on_two_calls():
         q.qhl_repack(qtype, rows, nb * 32, g, P)
         return P
 
-    for seed, qtype, rows, cols, n in ((61, Q4_0, 1000, 5120, 1), (62, Q8_0, 700, 17408, 16)):
+    # the last case fills the input region exactly: 16 tokens x 72 chunks x 2048
+    # bytes = 2.25 MiB, the largest problem the static array accepts
+    for seed, qtype, rows, cols, n in ((61, Q4_0, 1000, 5120, 1), (62, Q8_0, 700, 17408, 16),
+                                       (63, Q4_0, 130, 18432, 16)):
         W, x = synth.gemv_problem(seed, rows, cols, n, qtype)
         P = packed(qtype, W)
         xt = torch.from_numpy(x).cuda()
