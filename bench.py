@@ -127,9 +127,11 @@ def pass_bytes(shape, qtype, layers, ctx: int, n_tok: int = 1) -> dict:
     return {"weights": w, "kv": kv, "state": state, "total": w + kv + state}
 
 
-def launches_per_pass(shape, layers) -> int:
-    """Kernels the stage launches per pass: input + per layer (in-proj, mixer
-    kernel(s), out-proj, gate/up, down)."""
+def launches_per_pass(shape, layers, persistent: bool = False) -> int:
+    """Kernels the stage launches per pass: one persistent kernel, or input +
+    per layer (in-proj, mixer kernel(s), out-proj, gate/up, down)."""
+    if persistent:
+        return 1
     n = 1
     for l in layers:
         n += 6 if shape.is_attention(l) else 5
@@ -384,6 +386,8 @@ def run_ours(args, rank, world, local, pg):
     cfg = q.config_from_shape(shape, qtype, max_ctx)
     with torch.cuda.stream(stream):
         st = q.stage_load(cfg, tensors, 0, args.layers, stream=stream)
+        st.set_pass_mode(q.PASS_PERSISTENT if args.pass_mode == "persistent" else q.PASS_KERNELS)
+        persistent = st.pass_persistent(1)
         for l in layers:
             if shape.is_attention(l):
                 K, V = synth.kv_prefill(shape, SEED, l, CTX0, max_ctx)
@@ -504,7 +508,8 @@ def run_ours(args, rank, world, local, pg):
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (launches_per_pass(shape, layers) + 1) * args.steps,
+        "gpu_launches": (launches_per_pass(shape, layers, persistent) + 1) * args.steps,
+        "pass_mode": "persistent" if persistent else "kernels",
         "clocks": clk,
     }
     return res
@@ -562,6 +567,8 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-roofline", action="store_true")
+    ap.add_argument("--pass-mode", choices=("kernels", "persistent"), default="kernels",
+                    help="decode pass as a chain of kernels (CUDA graph) or as one persistent kernel")
     ap.add_argument("--only-kernel-roofline", action="store_true",
                     help="time only the dominant kernel alone (the GEMV roofline leg) and print it")
     args = ap.parse_args(argv)

@@ -232,6 +232,26 @@ stage_status stage_set_kv_len(stage_t* st, int kv_len);
  * dequantise bit-exactly. */
 stage_status stage_debug_dequant(stage_t* st, const char* tensor, int row, float* host_dst, size_t dst_elems);
 
+/* How a forward pass runs on the device.
+ *   STAGE_PASS_KERNELS (default): one kernel per step (stage input, then per
+ *     layer in-projection, mixer, out-projection, gate/up, down), recorded in
+ *     a CUDA graph, each a programmatic dependent of the one before.
+ *   STAGE_PASS_PERSISTENT: one cooperative kernel of one CTA per SM runs the
+ *     whole pass, its phases separated by a grid-wide arrival counter; its
+ *     producer streams every projection's weights across phase boundaries.
+ *     Used for n_tok 1..4 when the mixers' scratch fits (attention context of
+ *     at most ~3400 chunks of 64 rows); other passes and prefill run as
+ *     kernels.
+ * Both run the same units with the same split and reduction order, so they
+ * give bit-identical results.  Refused while a pass is pending; waits for the
+ * stage's stream and drops the recorded graphs. */
+typedef enum { STAGE_PASS_KERNELS = 0, STAGE_PASS_PERSISTENT = 1 } stage_pass_mode;
+stage_status stage_set_pass_mode(stage_t* st, int mode);
+
+/* 1 if an n_tok-token forward would run as the persistent kernel, 0 if as a
+ * chain of kernels, -1 for a NULL stage or n_tok outside 1..16. */
+int stage_pass_persistent(stage_t* st, int n_tok);
+
 /* Failure injection for tests of the device-side error path (no counterpart
  * on the pages; the stage's kernels bound every wait, and this makes one run
  * out without faulting anything).  fault_item >= 0: in the next recorded

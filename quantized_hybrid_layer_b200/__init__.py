@@ -23,6 +23,7 @@ STAGE_Q4_0 = 2
 STAGE_Q8_0 = 8
 MAX_TOK = 16
 PREFILL_EXACT, PREFILL_CHUNKED = 0, 1
+PASS_KERNELS, PASS_PERSISTENT = 0, 1
 
 STATUS = {
     0: "STAGE_OK", -1: "STAGE_E_ARG", -2: "STAGE_E_STATE", -3: "STAGE_E_OOM", -4: "STAGE_E_CUDA",
@@ -33,7 +34,8 @@ STATUS = {
 EXPORTS = (
     "stage_load", "stage_forward", "stage_forward_host", "stage_forward_f16", "stage_prefill", "stage_commit", "stage_rollback", "stage_reset", "stage_sync",
     "stage_committed_len", "stage_pending", "stage_get_dn_state", "stage_set_dn_state", "stage_get_kv",
-    "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_debug_inject",
+    "stage_set_kv", "stage_set_kv_len", "stage_debug_dequant", "stage_set_pass_mode", "stage_pass_persistent",
+    "stage_debug_inject",
     "stage_weight_bytes", "stage_last_error",
     "stage_free", "qhl_packed_bytes", "qhl_repack", "qhl_dequant", "qhl_qgemv", "qhl_deltanet_step",
     "qhl_qgemv_noalloc", "qhl_sync", "qhl_debug_inject", "qhl_last_error",
@@ -91,6 +93,8 @@ def lib() -> ctypes.CDLL:
             "stage_set_kv": (i, [vp, i, vp, vp, sz]),
             "stage_set_kv_len": (i, [vp, i]),
             "stage_debug_dequant": (i, [vp, ctypes.c_char_p, i, vp, sz]),
+            "stage_set_pass_mode": (i, [vp, i]),
+            "stage_pass_persistent": (i, [vp, i]),
             "stage_debug_inject": (i, [vp, i, ctypes.c_uint]),
             "stage_weight_bytes": (sz, [vp]),
             "stage_last_error": (ctypes.c_char_p, [vp]),
@@ -228,6 +232,15 @@ class Stage:
     @property
     def pending(self) -> int:
         return lib().stage_pending(self._h)
+
+    def set_pass_mode(self, mode: int):
+        """PASS_KERNELS (one kernel per step, the default) or PASS_PERSISTENT
+        (one cooperative kernel per forward pass where eligible)."""
+        self._check(lib().stage_set_pass_mode(self._h, mode))
+
+    def pass_persistent(self, n_tok: int) -> bool:
+        """Whether an n_tok forward runs as the persistent kernel."""
+        return lib().stage_pass_persistent(self._h, n_tok) == 1
 
     def debug_inject(self, fault_item: int = -1, wait_limit: int = 0):
         """Failure injection for tests of the bounded waits (stage_debug_inject)."""

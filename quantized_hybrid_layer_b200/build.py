@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqhl_stage.so")
-SOURCES = ["gemv.cu", "mixers.cu", "stage.cu", "kernel_abi.cu", "noalloc.cu"]
+SOURCES = ["gemv.cu", "pass.cu", "mixers.cu", "stage.cu", "kernel_abi.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 

@@ -157,7 +157,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t
     reinterpret_cast<float4*>(qs + job * kAttDim)[2 * lane + 1] = reinterpret_cast<const float4*>(vec)[2 * lane + 1];
     __syncwarp();
   }
-  named_sync(1, 256);   // new cache rows and queries visible to all 256 threads
+  named_sync(kBarMix, 256);   // new cache rows and queries visible to all 256 threads
 
   // K rows are loaded up front and V rows right after the scores (through L2,
   // each in one round), so the unit pays the memory latency about twice.  Scores: lane quad (lane >> 2) of warp w owns key
@@ -218,7 +218,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t
     const int kk = half * 32 + i;
     vr[i] = kk < nkeys ? ld_cg_once(reinterpret_cast<const uint32_t*>(a.V + (head_base + k0 + kk) * kAttDim) + pair) : 0u;
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
 
   // chunk softmax statistics, one warp per query
   for (int job = warp; job < njobs; job += 8) {
@@ -240,7 +240,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t
       a.pl[idx] = l;
     }
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
 
   // exp-weighted V: per (query, dim) the keys of each half in order, then
   // half 0 + half 1; 4 queries at a time (vec_all holds half 1's sums), so
@@ -275,7 +275,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t
       for (int jj = 0; jj < JB; ++jj)
         reinterpret_cast<float2*>(part + jj * kAttDim)[pair] = make_float2(o0[jj], o1[jj]);
     }
-    named_sync(1, 256);
+    named_sync(kBarMix, 256);
     if (half == 0) {
 #pragma unroll
       for (int jj = 0; jj < JB; ++jj) {
@@ -288,7 +288,7 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t
         }
       }
     }
-    named_sync(1, 256);
+    named_sync(kBarMix, 256);
   }
 }
 
@@ -322,12 +322,12 @@ QHL_DEV void combine_unit(const AttnArgs& a, int t, int head, int pos, float* cs
     cm[c] = __ldcg(a.pm + base + c);
     cl[c] = __ldcg(a.pl + base + c);
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
   float M = -INFINITY;
   for (int c = lane; c < nc; c += 32) M = fmaxf(M, cm[c]);
   M = warp_max(M);
   for (int c = dim; c < nc; c += 256) cw[c] = expf(__fsub_rn(cm[c], M));
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
   float L = 0.f;
   for (int c = lane; c < nc; c += 32) L = __fmaf_rn(cl[c], cw[c], L);
   L = warp_sum(L);
@@ -347,7 +347,7 @@ QHL_DEV void combine_unit(const AttnArgs& a, int t, int head, int pos, float* cs
   if (a.out) a.out[(size_t)t * a.out_stride + head * kAttDim + dim] = r;
   if (a.qout)   // warp w holds dims 32w..32w+31: one block
     qact_store_block(r, a.qout + (size_t)t * a.qout_stride, head * (kAttDim / 32) + (dim >> 5), dim & 31);
-  named_sync(1, 256);   // cs reusable by the caller
+  named_sync(kBarMix, 256);   // cs reusable by the caller
 }
 
 template <int NT>

@@ -142,6 +142,10 @@ QHL_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 QHL_DEV void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- named barrier among a subset of warps ---------------------------------
+// Barrier 0 is __syncthreads.  The mixer units (DeltaNet step, attention,
+// stage input) synchronise their 256 (or 128) threads on kBarMix, so they can
+// run beside warps that use other named barriers.
+constexpr int kBarMix = 5;
 QHL_DEV void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -117,7 +117,7 @@ QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
     sb[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_b + h);
     sa[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_a + h);
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
 
   for (int t = 0; t < NT; ++t) {
     float4 q = reinterpret_cast<const float4*>(sq + t * kDnDim)[lane];
@@ -151,11 +151,11 @@ QHL_DEV void dn_run(const DnArgs& a, int unit, float4 (&S)[4], float* sm) {
       if (keep) reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = S[r];
     }
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
   if (a.qo)
     for (int t = warp; t < NT; t += 8)
       qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (unit & 3), lane);
-  named_sync(1, 256);   // sm reusable by the caller
+  named_sync(kBarMix, 256);   // sm reusable by the caller
 }
 
 // Chunked form of the same recurrence for a prefill chunk whose tokens are
@@ -208,7 +208,7 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
     sb[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_b + h);
     sa[tid] = __ldcg(a.y + (size_t)tid * a.y_stride + off_a + h);
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
   // q, k normalised in place (warp w: tokens w, w + 8); decays by thread 0
   for (int t = warp; t < NT; t += 8) {
     float4 q = reinterpret_cast<const float4*>(sq + t * kDnDim)[lane];
@@ -232,7 +232,7 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
     }
     for (int t = 0; t < NT; ++t) ef[t] = expf(__fsub_rn(cl[NT - 1], cl[t]));
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
   for (int p = warp; p < NT * NT; p += 8) {
     const int t = p / NT, j = p % NT;
     const float4 kj = reinterpret_cast<const float4*>(sk + j * kDnDim)[lane];
@@ -244,7 +244,7 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
       Pm[p] = __fmul_rn(e, qk);
     }
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
 
   float* dst = a.cur ? a.ring + (size_t)((cur + NT) % a.ring_size) * a.state_elems
                      : a.ring + (size_t)(NT - 1) * a.state_elems;
@@ -286,11 +286,11 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
     }
     reinterpret_cast<float4*>(dst + ((size_t)h * kDnDim + row0 + r) * kDnDim)[lane] = sn;
   }
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
   if (a.qo)
     for (int t = warp; t < NT; t += 8)
       qact_store_block(ob[t][lane], a.qo + (size_t)t * a.qo_stride, h * (kDnDim / 32) + (unit & 3), lane);
-  named_sync(1, 256);
+  named_sync(kBarMix, 256);
 }
 
 template <int NT>

@@ -10,6 +10,7 @@
 #include "attention.cuh"
 #include "deltanet.cuh"
 #include "input.cuh"
+#include "pass.cuh"
 #include "qgemv.cuh"
 
 namespace qhl {
@@ -55,6 +56,11 @@ cudaError_t launch_dequant(int qt, const uint8_t* packed, int rows, int cols, in
 cudaError_t launch_rope_table(float2* tab, int max_ctx, int rope_dims, double theta, cudaStream_t s);
 cudaError_t launch_commit(int* ctrl, int n_accepted, int n_dn, int ring, cudaStream_t s);
 cudaError_t launch_set_int(int* p, int v, cudaStream_t s);
+
+// Persistent pass (pass.cuh, instantiated in pass.cu for n_tok 1..kPassMaxTok).
+cudaError_t pass_prepare(int qt);
+cudaError_t pass_occupancy(int qt, int nt, int* blocks);   // co-resident CTAs per SM (0: not instantiated)
+cudaError_t launch_pass(int qt, int nt, const PassArgs& p, cudaStream_t s);
 
 // CTAs that own items of a tiles x chunks GEMV on `cap` CTAs (one per SM).
 // When the CTAs can own whole tiles -- a divisor of `tiles` no smaller than

@@ -18,7 +18,7 @@ __global__ void __launch_bounds__(128) stage_input_kernel(const float* h, int H,
                                                           int qz_stride, float* ss, int ss_stride) {
   __shared__ float red[4];
   if (threadIdx.x == 0) pdl_launch();
-  input_unit<NT>(h, H, gamma, qz, qz_stride, ss, ss_stride, blockIdx.x, red, 1);
+  input_unit<NT>(h, H, gamma, qz, qz_stride, ss, ss_stride, blockIdx.x, red, kBarMix);
 }
 
 // f32 rows -> block fixed point, one warp per (token, 32-column block).  The

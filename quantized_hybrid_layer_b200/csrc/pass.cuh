@@ -1,0 +1,362 @@
+// The whole layer-stage pass in one persistent, cooperative kernel.
+//
+// The pages submit one command buffer per token (SwarmLLM README, paragraph
+// after the peer diagram), and every token reads all of the weights once.
+// Here one grid of one CTA per SM runs every phase of the pass -- the stage
+// input, then per layer the mixer in-projection, the DeltaNet step or the
+// attention partials + combine, the out-projection, gate/up and down -- with
+// the phases separated by a grid-wide arrival counter.  What a chain of
+// kernels cannot do, this does: the weight stream never stops at a phase
+// boundary.  The producer thread knows the pass's whole schedule of items
+// and keeps both rings full across phases; only an item's x columns wait for
+// the phase that writes them, and the unpack warps turn the next
+// projection's weights into MMA operands while the previous phase finishes.
+//
+// Warp roles of the CTA (18 warps):
+//   0..7    mixer units (stage input, DeltaNet step, attention partials and
+//           combine), the same device functions as the separate kernels
+//   8       producer (one thread): bulk copies of every projection's items
+//   9       MMA issuer (one thread) and tensor-memory owner
+//   10..13  unpack, 14..17 update: the GEMV roles of qgemv.cuh
+// Each CTA arrives once per phase (the update warps for a projection, the
+// mixer warps for a mixer phase); phase p may start once the counter reaches
+// p * grid.  Every wait is bounded; any recorded error makes every wait of
+// the pass give up.
+#pragma once
+
+#include "attention.cuh"
+#include "deltanet.cuh"
+#include "input.cuh"
+#include "qgemv.cuh"
+
+namespace qhl {
+
+struct PassLayer {
+  int attn;            // 1: full-attention layer, 0: gated DeltaNet
+  int phase_in;        // phase of the mixer in-projection
+  GemvArgs g[4];       // in-projection, out-projection, gate/up, down
+  DnArgs dn;
+  AttnArgs at;
+};
+
+struct PassArgs {
+  const PassLayer* layers;
+  int n_layers;
+  const float* h;      // stage input [NT][H]
+  int H;
+  const float* gamma0; // first layer's RMSNorm weight
+  uint8_t* qz;
+  int qz_stride;
+  float* ss;
+  int ss_stride;
+  const int* kv_len;   // position of token 0
+  unsigned* bar;       // phase arrival counter, zero at launch
+  int grid;            // CTAs (all co-resident)
+  int dn_units;        // Hv * 4
+  int Hq, Hkv;
+  unsigned* err;
+  uint32_t wait_limit; // 0: the default cap
+};
+
+// Mixer scratch of the persistent kernel: attention at up to 4 tokens with up
+// to 6 query heads per KV head, the combine's chunk statistics, the DeltaNet
+// unit, the stage input.
+constexpr int kPassMixBytes = 40 * 1024;
+constexpr int kPassXQueueBytes = 32 * 16;   // the producer's x-job queue, after the mixer scratch
+constexpr int kPassMaxTok = 4;
+
+constexpr int kPassMixWarps = 8;
+constexpr int kPassProducerWarp = 8;
+constexpr int kPassMmaWarp = 9;
+constexpr int kPassUnpackWarp0 = 10;
+constexpr int kPassUpdateWarp0 = 14;
+constexpr int kPassThreads = 18 * 32;
+
+template <int QT, int NT>
+struct PassCfg : GemvGeom<QT, NT, 221 * 1024, 8, 4, 4, 12, kPassMixBytes + kPassXQueueBytes> {};
+
+template <int QT, int NT>
+constexpr int pass_smem_bytes() {
+  return PassCfg<QT, NT>::kSmem;
+}
+
+QHL_DEV unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+QHL_DEV unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+QHL_DEV void red_release_gpu(unsigned* p) { asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p) : "memory"); }
+// Order this thread's earlier global writes before later async-proxy (bulk
+// copy) reads of them, and acquired global data before later bulk copies.
+QHL_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// One thread: wait until phase `ph` may start (every CTA arrived for the
+// phases before it).  False if an error was recorded anywhere or the wait ran
+// out.
+QHL_DEV bool phase_wait(const PassArgs& p, int ph) {
+  const unsigned target = (unsigned)ph * (unsigned)p.grid;
+  const uint32_t limit = wait_limit(p.wait_limit);
+  for (uint32_t i = 0;; ++i) {
+    if (ld_acquire_gpu(p.bar) >= target) return true;
+    if ((i & 63u) == 63u && ld_relaxed_gpu(p.err)) return false;
+    if (i >= limit) {
+      atomicOr(p.err, ERR_WAIT_TIMEOUT);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+// The threads of one role (`nthreads` on named barrier `bar_id`) wait for a
+// phase together: thread `leader` polls, all get the same answer.
+QHL_DEV bool group_phase_wait(const PassArgs& p, int ph, int bar_id, int nthreads, bool leader) {
+  bool ok = true;
+  if (leader) ok = phase_wait(p, ph);
+  return bar_and(bar_id, nthreads, ok);
+}
+
+// The group's arrival for a phase after its writes: every thread orders its
+// global writes before later bulk-copy reads by other CTAs, then the leader
+// releases the arrival.
+QHL_DEV void group_arrive(const PassArgs& p, int bar_id, int nthreads, bool leader) {
+  fence_proxy_async_global();
+  __threadfence();
+  named_sync(bar_id, nthreads);
+  if (leader) red_release_gpu(p.bar);
+}
+
+// Producer (one thread): every projection item of this CTA in pass order.
+// The quants go as soon as a weight slot is free; the scales and x columns of
+// an item wait in a small queue until its phase may start and an x slot is
+// free.  The queue is serviced whenever the thread would otherwise wait.
+// An x part waiting in the producer's queue (shared memory).
+struct XJob {
+  int gemv;            // layer * 4 + projection
+  int item, chunk, phase;
+};
+constexpr int kPassXQueue = 32;
+
+template <class C>
+QHL_DEV bool pass_produce(const PassArgs& p, const GemvSmem<C>& S, int cta, XJob* q) {
+  constexpr int SW = C::kSW, SX = C::kSX;
+  constexpr int kQ = kPassXQueue;   // x jobs whose quants are issued, oldest first
+  int qh = 0, qn = 0;
+  uint32_t KX = 0;        // x parts issued so far
+  unsigned ready = 0;     // phases known to have started
+  // The counter is polled with relaxed loads whose value is read at the next
+  // call, so a poll never stalls the weight copies issued in between; once the
+  // target is seen, one acquiring load orders the phase's data before the x
+  // copies.
+  unsigned polled = 0;
+  bool poll_out = false;
+  uint32_t polls = 0;
+  const uint64_t pol = policy_evict_first();
+  const uint32_t limit = wait_limit(p.wait_limit);
+  // issue the ready head of the queue; false only on an error seen
+  auto service = [&]() -> bool {
+    while (qn > 0) {
+      const XJob& j = q[qh];
+      if ((unsigned)j.phase > ready) {
+        const unsigned target = (unsigned)j.phase * (unsigned)p.grid;
+        if (!poll_out) {
+          polled = ld_relaxed_gpu(p.bar);
+          poll_out = true;
+          return true;
+        }
+        poll_out = false;
+        if (polled < target) return (++polls & 63u) != 0 || ld_relaxed_gpu(p.err) == 0;
+        (void)ld_acquire_gpu(p.bar);
+        ready = (unsigned)j.phase;
+        fence_proxy_async_global();
+      }
+      if (KX >= (uint32_t)SX && !mbar_test(smem_u32(&S.xempty[KX % SX]), ((KX / SX) - 1) & 1u)) return true;
+      const GemvArgs& a = p.layers[j.gemv >> 2].g[j.gemv & 3];
+      issue_scales<C>(a, S, j.item, KX, pol);
+      issue_x<C>(a, S, j.chunk, KX);
+      ++KX;
+      qh = qh + 1 == kQ ? 0 : qh + 1;
+      --qn;
+    }
+    return true;
+  };
+  uint32_t K = 0;         // quants issued so far
+  for (int l = 0; l < p.n_layers; ++l) {
+    const PassLayer& L = p.layers[l];
+    const int ph_out = L.phase_in + (L.attn ? 3 : 2);
+    const int phases[4] = {L.phase_in, ph_out, ph_out + 1, ph_out + 2};
+    for (int gi = 0; gi < 4; ++gi) {
+      const GemvArgs& a = L.g[gi];
+      if (cta >= a.workers) continue;
+      const StreamK sk(a.tiles * a.chunks, a.workers);
+      const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1);
+      int c = i0 % a.chunks;
+      for (int it = i0; it < i1; ++it, ++K) {
+        // a free weight slot and room in the queue; service the queue meanwhile
+        for (uint32_t spins = 0;; ++spins) {
+          const bool wfree = K < (uint32_t)SW || mbar_test(smem_u32(&S.wempty[K % SW]), ((K / SW) - 1) & 1u);
+          if (wfree && qn < kQ) break;
+          if (!service()) return false;
+          if (spins >= limit) {
+            atomicOr(p.err, ERR_WAIT_TIMEOUT);
+            return false;
+          }
+          __nanosleep(32);
+        }
+        issue_weights<C>(a, S, it, K, pol);
+        int qt = qh + qn;
+        if (qt >= kQ) qt -= kQ;
+        q[qt] = XJob{l * 4 + gi, it, c, phases[gi]};
+        ++qn;
+        if (++c == a.chunks) c = 0;
+        if (!service()) return false;
+      }
+    }
+  }
+  for (uint32_t spins = 0; qn > 0; ++spins) {
+    if (!service()) return false;
+    if (spins >= limit) {
+      atomicOr(p.err, ERR_WAIT_TIMEOUT);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  return true;
+}
+
+template <int QT, int NT>
+__global__ void __maxnreg__(112) stage_pass_kernel(const PassArgs p) {
+  using C = PassCfg<QT, NT>;
+  extern __shared__ __align__(16) uint8_t gsmem[];
+  const GemvSmem<C> S(gsmem);
+  uint8_t* mix = S.extra;
+  const int cta = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) S.init();
+  if (warp == kPassMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *S.tslot;
+  bool ok = true;
+
+  if (warp == kPassProducerWarp) {
+    if (lane == 0 && !pass_produce<C>(p, S, cta, reinterpret_cast<XJob*>(mix + kPassMixBytes)))
+      drain_inflight_copies();   // error path
+    return;   // the producer takes no part in the tensor-memory teardown
+  }
+  if (warp < kPassMixWarps) {
+    // ---------------- mixer warps: stage input, DeltaNet, attention ----------
+    const bool lead = tid == 0;
+    // phase 0: the stage input (four warps, 128-row tiles)
+    if (warp < 4)
+      for (int u = cta; u < p.H / kTileRows; u += p.grid)
+        input_unit<NT>(p.h, p.H, p.gamma0, p.qz, p.qz_stride, p.ss, p.ss_stride, u, reinterpret_cast<float*>(mix),
+                       kBarMix);
+    group_arrive(p, kBarMix + 1, 256, lead);
+    for (int l = 0; l < p.n_layers && ok; ++l) {
+      const PassLayer& L = p.layers[l];
+      const int ph = L.phase_in + 1;
+      if (!L.attn) {
+        float4 Sr[4];
+        const int u0 = cta;
+        if (u0 < p.dn_units) dn_load<NT>(L.dn, u0, Sr);   // the state rows never depend on this pass
+        if (!(ok = group_phase_wait(p, ph, kBarMix + 1, 256, lead))) break;
+        for (int u = u0; u < p.dn_units; u += p.grid) {
+          if (u != u0) dn_load<NT>(L.dn, u, Sr);
+          if (L.dn.mode == DN_CHUNKED)
+            dn_run_chunked<NT>(L.dn, u, Sr, reinterpret_cast<float*>(mix));
+          else
+            dn_run<NT>(L.dn, u, Sr, reinterpret_cast<float*>(mix));
+        }
+        group_arrive(p, kBarMix + 1, 256, lead);
+      } else {
+        if (!(ok = group_phase_wait(p, ph, kBarMix + 1, 256, lead))) break;
+        const int pos = *p.kv_len;
+        constexpr int kGroups = (NT + kAttGroup - 1) / kAttGroup;
+        const int units = (pos + NT + kAttChunk - 1) / kAttChunk * p.Hkv * kGroups;
+        for (int u = cta; u < units; u += p.grid) {
+          const int grp = u % kGroups, rest = u / kGroups, t0 = grp * kAttGroup;
+          const int c = rest / p.Hkv, g = rest % p.Hkv;
+          if (c * kAttChunk < pos + t0 + min(kAttGroup, NT - t0)) attn_unit<NT>(L.at, c, g, pos, t0, mix);
+        }
+        group_arrive(p, kBarMix + 1, 256, lead);
+        if (!(ok = group_phase_wait(p, ph + 1, kBarMix + 1, 256, lead))) break;
+        for (int u = cta; u < NT * p.Hq; u += p.grid)
+          combine_unit<NT>(L.at, u / p.Hq, u % p.Hq, pos, reinterpret_cast<float*>(mix));
+        group_arrive(p, kBarMix + 1, 256, lead);
+      }
+    }
+    if (!ok && tid == 0) drain_inflight_copies();
+    return;   // the mixer warps take no part in the tensor-memory teardown
+  }
+
+  uint32_t K = 0;   // this CTA's items so far, over every projection of the pass
+  if (warp == kPassMmaWarp) {
+    if (lane == 0) {
+      for (int l = 0; l < p.n_layers && ok; ++l)
+        for (int gi = 0; gi < 4 && ok; ++gi) {
+          const GemvArgs& a = p.layers[l].g[gi];
+          if (cta >= a.workers) continue;
+          const StreamK sk(a.tiles * a.chunks, a.workers);
+          const int n = sk.begin(cta + 1) - sk.begin(cta);
+          ok = mma_items<C>(a, S, tmem, n, K);
+          K += n;
+        }
+      // every MMA this thread issued has completed before tensor memory goes
+      tc_commit(S.drain);
+      if (!mbar_wait(smem_u32(S.drain), 0, p.err, p.wait_limit)) ok = false;
+    }
+    __syncwarp();
+  } else if (warp < kPassUpdateWarp0) {
+    for (int l = 0; l < p.n_layers && ok; ++l)
+      for (int gi = 0; gi < 4 && ok; ++gi) {
+        const GemvArgs& a = p.layers[l].g[gi];
+        if (cta >= a.workers) continue;
+        const StreamK sk(a.tiles * a.chunks, a.workers);
+        const int n = sk.begin(cta + 1) - sk.begin(cta);
+        ok = unpack_items<C>(a, S, tmem, n, K, warp & 3, lane);
+        K += n;
+      }
+  } else {
+    // ---------------- update warps: one projection phase after another ------
+    const bool lead = warp == kPassUpdateWarp0 && lane == 0;
+    for (int l = 0; l < p.n_layers && ok; ++l) {
+      const PassLayer& L = p.layers[l];
+      const int ph_out = L.phase_in + (L.attn ? 3 : 2);
+      const int phases[4] = {L.phase_in, ph_out, ph_out + 1, ph_out + 2};
+      for (int gi = 0; gi < 4 && ok; ++gi) {
+        const GemvArgs& a = L.g[gi];
+        if (!(ok = group_phase_wait(p, phases[gi], kBarUpdate, 128, lead))) break;
+        if (cta < a.workers) {
+          const StreamK sk(a.tiles * a.chunks, a.workers);
+          const int i0 = sk.begin(cta), n = sk.begin(cta + 1) - i0;
+          load_rstd<C>(a, S, warp & 3, lane);
+          switch (gi) {
+            case 0: ok = update_items<C, EPI_STORE>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+            case 1: ok = update_items<C, EPI_RESID>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+            case 2: ok = update_items<C, EPI_SWIGLU>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+            default: ok = update_items<C, EPI_RESID>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+          }
+          K += n;
+        }
+        if (ok) group_arrive(p, kBarUpdate, 128, lead);
+      }
+    }
+  }
+  // ---------------- teardown: tensor memory back, after every MMA and load --
+  tc_fence_before();
+  named_sync(kBarTmem, 9 * 32);
+  if (warp == kPassMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+  if (!ok && lane == 0) drain_inflight_copies();   // error path
+}
+
+}  // namespace qhl

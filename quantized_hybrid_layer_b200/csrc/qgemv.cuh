@@ -106,40 +106,53 @@ constexpr int kGemvCtaThreads = 320;
 constexpr int kBarUpdate = 1;
 constexpr int kBarTmem = 2;
 
-// Geometry and shared-memory layout of one (weight type, token count).
-template <int QT, int NT>
-struct GemvCfg {
-  static constexpr int kN = NT == 1 ? 8 : 16 * ((NT + 1) / 2);   // MMA N: 8 rows per token, padded
-  static constexpr int kNTP = kN / 8;                              // token regions in an x slot
+// Geometry and shared-memory layout of one GEMV configuration: weight type,
+// token count, shared-memory budget, x-ring depth SX, tensor-memory A and D
+// buffers NA and ND, the deepest weight ring to use, and `EXTRA` bytes of
+// shared memory left for the caller after the GEMV's own regions.
+template <int QT_, int NT_, int BUDGET, int SX_, int NA_, int ND_, int SWMAX, int EXTRA>
+struct GemvGeom {
+  static constexpr int kQT = QT_, kNT = NT_;
+  static constexpr int kN = NT_ == 1 ? 8 : 16 * ((NT_ + 1) / 2);   // MMA N: 8 rows per token, padded
+  static constexpr int kNTP = kN / 8;                               // token regions in an x slot
   static constexpr int kGB = (64 / kN) >= 8 ? 8 : ((64 / kN) >= 1 ? 64 / kN : 1);   // blocks per D group
-  static constexpr int kNG = 8 / kGB;                              // D groups per item
-  static constexpr int kDCols = kGB * kN;                          // tensor-memory columns of a D buffer
-  static constexpr int kACols = 64;                                // 8 blocks x 32 bytes / 4
-  static constexpr int kDOff = 2 * kACols;
-  static constexpr int kTmemCols = kDOff + 2 * kDCols <= 256 ? 256 : 512;
-  static constexpr int kQB = QLayout<QT>::kQuantBytes;
-  static constexpr int kXS = QLayout<QT>::kScaleBytes + kNTP * kQChunkBytes;   // x slot: scales, then tokens
-  // two CTAs per SM (this projection and the next) at one and two tokens (Q4_0)
-  static constexpr bool kPair = QT == kQ4_0 && NT <= 2;
-  static constexpr int kBudget = kPair ? 110 * 1024 : 200 * 1024;
-  static constexpr int kEpi = NT * kTileRows * 4;                  // epilogue exchange [NT][128] f32
-  static constexpr int kFixed = kEpi + 16 * 4 + 16 + 320;          // + rstd, tmem slot, barriers
-  static constexpr int kSX = kPair ? 6 : 3;
-  static constexpr int kSW0 = (kBudget - kFixed - kSX * kXS) / kQB;
-  static constexpr int kSW = kSW0 > 8 ? 8 : kSW0;
-  static constexpr int kMinBlocks = kPair ? 2 : 1;
+  static constexpr int kNG = 8 / kGB;                               // D groups per item
+  static constexpr int kDCols = kGB * kN;                           // tensor-memory columns of a D buffer
+  static constexpr int kACols = 64;                                 // 8 blocks x 32 bytes / 4
+  static constexpr int kNA = NA_, kND = ND_;
+  static constexpr int kDOff = kNA * kACols;
+  static constexpr int kTmemNeed = kDOff + kND * kDCols;
+  static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
+  static constexpr int kQB = QLayout<QT_>::kQuantBytes;
+  static constexpr int kXS = QLayout<QT_>::kScaleBytes + kNTP * kQChunkBytes;   // x slot: scales, then tokens
+  static constexpr int kSX = SX_;
+  static constexpr int kEpi = NT_ * kTileRows * 4;                  // epilogue exchange [NT][128] f32
+  static constexpr int kNumBars = 2 * 16 + 2 * SX_ + 2 * NA_ + 2 * ND_ + 1;   // upper bound (SW <= 16)
+  static constexpr int kFixed = kEpi + 16 * 4 + 16 + kNumBars * 8 + EXTRA;
+  static constexpr int kSW0 = (BUDGET - kFixed - SX_ * kXS) / kQB;
+  static constexpr int kSW = kSW0 > SWMAX ? SWMAX : kSW0;
   // shared-memory layout (the rings first; every slot 16-byte aligned)
   static constexpr int kXOff = kSW * kQB;
   static constexpr int kEpiOff = kXOff + kSX * kXS;
-  static constexpr int kRstdOff = kEpiOff + kEpi;
+  static constexpr int kExtraOff = kEpiOff + kEpi;
+  static constexpr int kRstdOff = kExtraOff + (EXTRA + 15) / 16 * 16;
   static constexpr int kSlotOff = kRstdOff + 16 * 4;
   static constexpr int kBarOff = kSlotOff + 16;
-  // barriers: wfull[SW], wempty[SW], xfull[SX], xempty[SX], afull[2], afree[2], dfull[2], dfree[2], drain
-  static constexpr int kNumBars = 2 * kSW + 2 * kSX + 9;
-  static constexpr int kSmem = kBarOff + kNumBars * 8;
-  static_assert(kSW >= 2, "weight ring too shallow");
-  static_assert(kNumBars * 8 <= 320, "barrier area");
-  static_assert(kSmem <= kBudget, "shared-memory budget");
+  // barriers: wfull[SW], wempty[SW], xfull[SX], xempty[SX], afull[NA], afree[NA], dfull[ND], dfree[ND], drain
+  static constexpr int kSmem = kBarOff + (2 * kSW + 2 * kSX + 2 * kNA + 2 * kND + 1) * 8;
+  static_assert(kSW >= 2 && kSW <= 16, "weight ring depth");
+  static_assert(kTmemNeed <= 512, "tensor memory");
+  static_assert(kSmem <= BUDGET, "shared-memory budget");
+};
+
+// The stand-alone projection kernel's configuration: one CTA per SM with a
+// deep weight ring (the bytes in flight per SM decide the streaming rate) and
+// four A and four D buffers in tensor memory, so the unpack warps, the MMA
+// thread and the update warps each run up to four items apart instead of
+// waiting on one another's latencies.
+template <int QT, int NT>
+struct GemvCfg : GemvGeom<QT, NT, 200 * 1024, NT <= 2 ? 6 : 3, 4, NT <= 8 ? 4 : 2, 12, 0> {
+  static constexpr int kMinBlocks = 1;
 };
 
 template <int QT, int NT>
@@ -301,272 +314,345 @@ QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int
   if (r == 0) a.counters[tl] = 0;
 }
 
-template <int QT, int NT, int EPI>
-__global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
-  using C = GemvCfg<QT, NT>;
-  constexpr int SW = C::kSW, SX = C::kSX, QB = C::kQB, XS = C::kXS;
-  extern __shared__ __align__(16) uint8_t gsmem[];
-  uint8_t* wring = gsmem;
-  uint8_t* xring = gsmem + C::kXOff;
-  float* ex = reinterpret_cast<float*>(gsmem + C::kEpiOff);
-  float* rstd = reinterpret_cast<float*>(gsmem + C::kRstdOff);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(gsmem + C::kSlotOff);
-  int* flag = reinterpret_cast<int*>(gsmem + C::kSlotOff + 4);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gsmem + C::kBarOff);
-  uint64_t* wfull = bars;
-  uint64_t* wempty = bars + SW;
-  uint64_t* xfull = bars + 2 * SW;
-  uint64_t* xempty = bars + 2 * SW + SX;
-  uint64_t* afull = bars + 2 * SW + 2 * SX;
-  uint64_t* afree = afull + 2;
-  uint64_t* dfull = afull + 4;
-  uint64_t* dfree = afull + 6;
-  uint64_t* drain = afull + 8;
-
-  const int cta = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) pdl_launch();
-  if (cta >= a.workers) return;
-  const StreamK sk(a.tiles * a.chunks, a.workers);
-  const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1), n = i1 - i0;
-  if (n == 0) return;
-
-  if (tid == 0) {
-    for (int s = 0; s < SW; ++s) {
+// Pointers of one CTA's GEMV machinery in shared memory (layout of config C).
+template <class C>
+struct GemvSmem {
+  uint8_t* wring;
+  uint8_t* xring;
+  float* ex;
+  uint8_t* extra;
+  float* rstd;
+  uint32_t* tslot;
+  int* flag;
+  uint64_t *wfull, *wempty, *xfull, *xempty, *afull, *afree, *dfull, *dfree, *drain;
+  QHL_DEV explicit GemvSmem(uint8_t* base) {
+    wring = base;
+    xring = base + C::kXOff;
+    ex = reinterpret_cast<float*>(base + C::kEpiOff);
+    extra = base + C::kExtraOff;
+    rstd = reinterpret_cast<float*>(base + C::kRstdOff);
+    tslot = reinterpret_cast<uint32_t*>(base + C::kSlotOff);
+    flag = reinterpret_cast<int*>(base + C::kSlotOff + 4);
+    wfull = reinterpret_cast<uint64_t*>(base + C::kBarOff);
+    wempty = wfull + C::kSW;
+    xfull = wfull + 2 * C::kSW;
+    xempty = xfull + C::kSX;
+    afull = xempty + C::kSX;
+    afree = afull + C::kNA;
+    dfull = afree + C::kNA;
+    dfree = dfull + C::kND;
+    drain = dfree + C::kND;
+  }
+  // barrier set-up by one thread
+  QHL_DEV void init() const {
+    for (int s = 0; s < C::kSW; ++s) {
       mbar_init(smem_u32(&wfull[s]), 1);
       mbar_init(smem_u32(&wempty[s]), 4);
     }
-    for (int s = 0; s < SX; ++s) {
+    for (int s = 0; s < C::kSX; ++s) {
       mbar_init(smem_u32(&xfull[s]), 1);
       mbar_init(smem_u32(&xempty[s]), 4);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kNA; ++b) {
       mbar_init(smem_u32(&afull[b]), 4);
       mbar_init(smem_u32(&afree[b]), 1);
+    }
+    for (int b = 0; b < C::kND; ++b) {
       mbar_init(smem_u32(&dfull[b]), 1);
       mbar_init(smem_u32(&dfree[b]), 4);
     }
     mbar_init(smem_u32(drain), 1);
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) tmem_alloc(tslot, C::kTmemCols);
+};
+
+// The roles below process this CTA's items [i0, i0 + n) of one projection.  K0
+// is the running count of items the CTA has taken through its rings before
+// this projection: ring slots, buffer indices and barrier phases follow from
+// the running count K0 + k, so consecutive projections can share one CTA's
+// rings and buffers.
+
+// Copies of one item's parts into the rings (producer thread).
+template <class C>
+QHL_DEV void issue_weights(const GemvArgs& a, const GemvSmem<C>& S, int item, uint32_t K, uint64_t pol) {
+  constexpr int QT = C::kQT;
+  const int s = K % C::kSW;
+  mbar_arrive_expect_tx(smem_u32(&S.wfull[s]), C::kQB);
+  bulk_g2s(smem_u32(S.wring + s * C::kQB), a.W + (size_t)item * QLayout<QT>::kItemBytes, C::kQB,
+           smem_u32(&S.wfull[s]), pol);
+}
+template <class C>
+QHL_DEV void issue_scales(const GemvArgs& a, const GemvSmem<C>& S, int item, uint32_t K, uint64_t pol) {
+  constexpr int QT = C::kQT, NT = C::kNT;
+  const int s = K % C::kSX;
+  mbar_arrive_expect_tx(smem_u32(&S.xfull[s]), QLayout<QT>::kScaleBytes + NT * kQChunkBytes);
+  bulk_g2s(smem_u32(S.xring + s * C::kXS), a.W + (size_t)item * QLayout<QT>::kItemBytes + C::kQB,
+           QLayout<QT>::kScaleBytes, smem_u32(&S.xfull[s]), pol);
+}
+template <class C>
+QHL_DEV void issue_x(const GemvArgs& a, const GemvSmem<C>& S, int chunk, uint32_t K) {
+  constexpr int QT = C::kQT, NT = C::kNT;
+  const int s = K % C::kSX;
+  for (int t = 0; t < NT; ++t)
+    bulk_g2s_plain(smem_u32(S.xring + s * C::kXS + QLayout<QT>::kScaleBytes + t * kQChunkBytes),
+                   a.qx + (size_t)t * a.qx_stride + (size_t)chunk * kQChunkBytes, kQChunkBytes,
+                   smem_u32(&S.xfull[s]));
+}
+
+// Producer of one stand-alone projection (one thread; K0 = 0).  The weights
+// never depend on earlier kernels: the first rings are requested before
+// griddepcontrol.wait, the x columns (written by the previous kernel) once the
+// dependency is resolved.  Returns false on a timeout.
+template <class C>
+QHL_DEV bool produce_items(const GemvArgs& a, const GemvSmem<C>& S, int cta, int i0, int n) {
+  constexpr int QT = C::kQT;
+  constexpr int SW = C::kSW, SX = C::kSX;
+  const uint64_t pol = policy_evict_first();
+  const int c0 = i0 % a.chunks;
+  auto chunk_of = [&](int k) {   // chunk of local item k, without 64-bit division
+    int c = c0 + k % a.chunks;
+    return c >= a.chunks ? c - a.chunks : c;
+  };
+  auto w = [&](int k) {
+    if (cta == 0 && k == a.fault_item) return;   // injected failure: this slot never fills
+    issue_weights<C>(a, S, i0 + k, (uint32_t)k, pol);
+  };
+  int kw = 0, kx = 0;
+  for (; kw < n && kw < SW; ++kw) w(kw);
+  for (int k = 0; k < n && k < SX; ++k) issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
+  pdl_wait();
+  for (; kx < n && kx < SX; ++kx) issue_x<C>(a, S, chunk_of(kx), (uint32_t)kx);
+  for (uint32_t spins = 0; kw < n || kx < n;) {
+    bool did = false;
+    if (kw < n && mbar_test(smem_u32(&S.wempty[kw % SW]), ((kw / SW) - 1) & 1u)) {
+      w(kw++);
+      did = true;
+    }
+    if (kx < n && mbar_test(smem_u32(&S.xempty[kx % SX]), ((kx / SX) - 1) & 1u)) {
+      issue_scales<C>(a, S, i0 + kx, (uint32_t)kx, pol);
+      issue_x<C>(a, S, chunk_of(kx), (uint32_t)kx);
+      ++kx;
+      did = true;
+    }
+    if (did) {
+      spins = 0;
+    } else if (++spins > wait_limit(a.wait_limit)) {
+      atomicOr(a.err, ERR_WAIT_TIMEOUT);
+      return false;
+    } else {
+      __nanosleep(32);   // both rings full: poll lightly
+    }
+  }
+  if (a.next_W && cta < a.next_workers) {
+    // every own item is on its way: warm L2 with the next projection's first
+    // items of this CTA index while the consumers finish
+    const StreamK skn(a.next_items, a.next_workers);
+    const int j0 = skn.begin(cta), nj = min(SW, skn.begin(cta + 1) - j0);
+    for (int k = 0; k < nj; ++k)
+      bulk_prefetch_l2(a.next_W + (size_t)(j0 + k) * QLayout<QT>::kItemBytes, QLayout<QT>::kItemBytes);
+  }
+  return true;
+}
+
+// Unpack warps (thread = row r of quarter `quarter`): each item's quants into
+// the A operand in tensor memory.  Returns false on a timeout.
+template <class C>
+QHL_DEV bool unpack_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int n, uint32_t K0, int quarter,
+                          int lane) {
+  constexpr int QT = C::kQT;
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+  for (int k = 0; k < n; ++k) {
+    const uint32_t K = K0 + k;
+    const int ab = K % C::kNA, sw = K % C::kSW;
+    if (!mbar_wait(smem_u32(&S.wfull[sw]), (K / C::kSW) & 1u, a.err, a.wait_limit) ||
+        (K >= C::kNA && !mbar_wait(smem_u32(&S.afree[ab]), ((K / C::kNA) - 1) & 1u, a.err, a.wait_limit)))
+      return false;
+    tc_fence_after();
+    const uint8_t* q = S.wring + sw * C::kQB;
+    const uint32_t ta = tmem + lane_base + ab * C::kACols;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      uint32_t av[8];
+      if constexpr (QT == kQ4_0) {
+        q4_unpack(*reinterpret_cast<const uint4*>(q + q4_off(b, r)), av);
+      } else {
+        const uint4 w0 = *reinterpret_cast<const uint4*>(q + q8_off(b, 0, r));
+        const uint4 w1 = *reinterpret_cast<const uint4*>(q + q8_off(b, 1, r));
+        av[0] = w0.x; av[1] = w0.y; av[2] = w0.z; av[3] = w0.w;
+        av[4] = w1.x; av[5] = w1.y; av[6] = w1.z; av[7] = w1.w;
+      }
+      tmem_st8(ta + 8 * b, av);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(smem_u32(&S.afull[ab]));
+      mbar_arrive(smem_u32(&S.wempty[sw]));
+    }
+  }
+  return true;
+}
+
+// MMA issuer (one thread): per item and block one M = 128, N = 8 per token,
+// K = 32 integer MMA into a D buffer.  Returns false on a timeout.
+template <class C>
+QHL_DEV bool mma_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int n, uint32_t K0) {
+  constexpr int QT = C::kQT;
+  constexpr uint32_t idesc = idesc_i8(QT == kQ8_0, kTileRows, C::kN);
+  for (int k = 0; k < n; ++k) {
+    const uint32_t K = K0 + k;
+    const int ab = K % C::kNA, sx = K % C::kSX;
+    if (!mbar_wait(smem_u32(&S.afull[ab]), (K / C::kNA) & 1u, a.err, a.wait_limit) ||
+        !mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit))
+      return false;
+    tc_fence_after();
+    const uint32_t xs = smem_u32(S.xring + sx * C::kXS + QLayout<QT>::kScaleBytes);
+    for (int g = 0; g < C::kNG; ++g) {
+      const uint32_t gc = K * C::kNG + g;
+      const int db = gc % C::kND;
+      if (gc >= C::kND && !mbar_wait(smem_u32(&S.dfree[db]), ((gc / C::kND) - 1) & 1u, a.err, a.wait_limit))
+        return false;
+      tc_fence_after();
+#pragma unroll
+      for (int j = 0; j < C::kGB; ++j) {
+        const int b = g * C::kGB + j;
+        const uint64_t desc = smem_desc_kmajor(xs + b * kQBlockBytes, 128, kQChunkBytes);
+        mma_i8_ts(tmem + C::kDOff + db * C::kDCols + j * C::kN, tmem + ab * C::kACols + 8 * b, desc, idesc, false);
+      }
+      tc_commit(&S.dfull[db]);
+    }
+    tc_commit(&S.afree[ab]);
+  }
+  return true;
+}
+
+// Update warps (thread = row r of quarter `quarter`, the four warps of
+// kBarUpdate): f32 block updates of every item in order, then the tile finish
+// at each tile boundary.  rstd[] must hold the input's RMS scale.  The four
+// warps take every decision together.  Returns false on a timeout.
+template <class C, int EPI>
+QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int cta, int i0, int n,
+                          uint32_t K0, int quarter, int lane) {
+  constexpr int QT = C::kQT, NT = C::kNT;
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+  const StreamK sk(a.tiles * a.chunks, a.workers);
+  const int i1 = i0 + n;
+  float acc[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+  int tile = i0 / a.chunks;
+  bool timed_out = false;
+  for (int k = 0; k < n; ++k) {
+    const uint32_t K = K0 + k;
+    const int item = i0 + k, sx = K % C::kSX;
+    if (item / a.chunks != tile) {
+      if (!bar_and(kBarUpdate, 128, !timed_out)) return false;
+      gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+      tile = item / a.chunks;
+    }
+    const uint8_t* xsl = S.xring + sx * C::kXS;
+    uint4 sc4 = make_uint4(0, 0, 0, 0);
+    for (int g = 0; g < C::kNG; ++g) {
+      const uint32_t gc = K * C::kNG + g;
+      const int db = gc % C::kND;
+      // (the first group also waits for the x slot itself: its scales and
+      // block metadata are read here, not only by the MMA).  After a timeout
+      // this warp waits for nothing more; the four warps agree on stopping at
+      // the next tile boundary, before any named barrier they share.
+      if (!timed_out)
+        timed_out = !(mbar_wait(smem_u32(&S.dfull[db]), (gc / C::kND) & 1u, a.err, a.wait_limit) &&
+                      (g > 0 || mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit)));
+      if (timed_out) continue;
+      tc_fence_after();
+      if (g == 0) sc4 = *reinterpret_cast<const uint4*>(xsl + r * 16);   // the row's 8 block scales
+      int dv[C::kGB][NT][4];
+#pragma unroll
+      for (int j = 0; j < C::kGB; ++j)
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          tmem_ld4(tmem + lane_base + C::kDOff + db * C::kDCols + j * C::kN + t * 8, dv[j][t]);
+      tmem_ld_wait();
+      const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+#pragma unroll
+      for (int j = 0; j < C::kGB; ++j) {
+        const int b = g * C::kGB + j;
+        const uint32_t w = scw[b >> 1];
+        const float d = __half2float(__ushort_as_half(static_cast<unsigned short>((b & 1) ? (w >> 16) : (w & 0xFFFFu))));
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const int4 m = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + t * kQChunkBytes +
+                                                        b * kQBlockBytes + kQMetaOff);
+          acc[t] = block_update<QT>(acc[t], d, __int_as_float(m.x), dv[j][t][0], dv[j][t][1], dv[j][t][2], m.y, m.z);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.dfree[db]));
+    }
+    __syncwarp();
+    if (!timed_out && lane == 0) mbar_arrive(smem_u32(&S.xempty[sx]));
+  }
+  if (!bar_and(kBarUpdate, 128, !timed_out)) return false;
+  gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane);
+  return true;
+}
+
+// The input's RMS scale per token into S.rstd (update warps; after the
+// dependency on the kernel that wrote ss_in is resolved).
+template <class C>
+QHL_DEV void load_rstd(const GemvArgs& a, const GemvSmem<C>& S, int quarter, int lane) {
+  constexpr int NT = C::kNT;
+  for (int t = quarter; t < NT; t += 4) {
+    const float rs = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
+    if (lane == 0) S.rstd[t] = rs;
+  }
+  named_sync(kBarUpdate, 128);
+}
+
+template <int QT, int NT, int EPI>
+__global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
+  using C = GemvCfg<QT, NT>;
+  extern __shared__ __align__(16) uint8_t gsmem[];
+  const GemvSmem<C> S(gsmem);
+  const int cta = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) pdl_launch();
+  if (cta >= a.workers) return;
+  const StreamK sk(a.tiles * a.chunks, a.workers);
+  const int i0 = sk.begin(cta), n = sk.begin(cta + 1) - i0;
+  if (n == 0) return;
+
+  if (tid == 0) S.init();
+  if (warp == kMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;
+  const uint32_t tmem = *S.tslot;
 
   if (warp == kProducerWarp) {
-    // ---------------- producer: one thread streams this CTA's items ----------
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      const int c0 = i0 % a.chunks;
-      auto chunk_of = [&](int k) {   // chunk of local item k, without 64-bit division
-        int c = c0 + k % a.chunks;
-        return c >= a.chunks ? c - a.chunks : c;
-      };
-      auto issue_w = [&](int k) {
-        const int s = k % SW;
-        if (cta == 0 && k == a.fault_item) return;   // injected failure: this slot never fills
-        mbar_arrive_expect_tx(smem_u32(&wfull[s]), QB);
-        bulk_g2s(smem_u32(wring + s * QB), a.W + (size_t)(i0 + k) * QLayout<QT>::kItemBytes, QB,
-                 smem_u32(&wfull[s]), pol);
-      };
-      auto issue_scales = [&](int k) {
-        const int s = k % SX;
-        mbar_arrive_expect_tx(smem_u32(&xfull[s]), QLayout<QT>::kScaleBytes + NT * kQChunkBytes);
-        bulk_g2s(smem_u32(xring + s * XS), a.W + (size_t)(i0 + k) * QLayout<QT>::kItemBytes + QB,
-                 QLayout<QT>::kScaleBytes, smem_u32(&xfull[s]), pol);
-      };
-      auto issue_x = [&](int k) {
-        const int s = k % SX, c = chunk_of(k);
-        for (int t = 0; t < NT; ++t)
-          bulk_g2s_plain(smem_u32(xring + s * XS + QLayout<QT>::kScaleBytes + t * kQChunkBytes),
-                         a.qx + (size_t)t * a.qx_stride + (size_t)c * kQChunkBytes, kQChunkBytes,
-                         smem_u32(&xfull[s]));
-      };
-      // weights never depend on earlier kernels: the first rings are requested
-      // before griddepcontrol.wait; the x columns (written by the previous
-      // kernel) once the dependency is resolved
-      int kw = 0, kx = 0;
-      for (; kw < n && kw < SW; ++kw) issue_w(kw);
-      for (int k = 0; k < n && k < SX; ++k) issue_scales(k);
-      pdl_wait();
-      for (; kx < n && kx < SX; ++kx) issue_x(kx);
-      bool ok = true;
-      for (uint32_t spins = 0; ok && (kw < n || kx < n);) {
-        bool did = false;
-        if (kw < n && mbar_test(smem_u32(&wempty[kw % SW]), ((kw / SW) - 1) & 1u)) {
-          issue_w(kw++);
-          did = true;
-        }
-        if (kx < n && mbar_test(smem_u32(&xempty[kx % SX]), ((kx / SX) - 1) & 1u)) {
-          issue_scales(kx);
-          issue_x(kx++);
-          did = true;
-        }
-        if (did) {
-          spins = 0;
-        } else if (++spins > wait_limit(a.wait_limit)) {
-          atomicOr(a.err, ERR_WAIT_TIMEOUT);
-          ok = false;
-        } else {
-          __nanosleep(32);   // both rings full: poll lightly
-        }
-      }
-      if (ok && a.next_W && cta < a.next_workers) {
-        // every own item is on its way: warm L2 with the next projection's
-        // first items of this CTA index while the consumers finish
-        const StreamK skn(a.next_items, a.next_workers);
-        const int j0 = skn.begin(cta), nj = min(SW, skn.begin(cta + 1) - j0);
-        for (int k = 0; k < nj; ++k) bulk_prefetch_l2(a.next_W + (size_t)(j0 + k) * QLayout<QT>::kItemBytes,
-                                                      QLayout<QT>::kItemBytes);
-      }
-      if (!ok) drain_inflight_copies();   // error path
-    }
+    if (lane == 0 && !produce_items<C>(a, S, cta, i0, n)) drain_inflight_copies();   // error path
     return;   // the producer takes no part in the tensor-memory teardown
   }
-
-  bool timed_out = false;
+  bool ok = true;
   if (warp == kMmaWarp) {
-    // ---------------- MMA issuer: one thread ---------------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(QT == kQ8_0, kTileRows, C::kN);
-      uint32_t gc = 0;
-      for (int k = 0; k < n && !timed_out; ++k) {
-        const int ab = k & 1, sx = k % SX;
-        if (!mbar_wait(smem_u32(&afull[ab]), (uint32_t)(k >> 1) & 1u, a.err, a.wait_limit) ||
-            !mbar_wait(smem_u32(&xfull[sx]), (uint32_t)(k / SX) & 1u, a.err, a.wait_limit)) {
-          timed_out = true;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t xs = smem_u32(xring + sx * XS + QLayout<QT>::kScaleBytes);
-        for (int g = 0; g < C::kNG; ++g, ++gc) {
-          const int db = gc & 1;
-          if (gc >= 2 && !mbar_wait(smem_u32(&dfree[db]), ((gc >> 1) - 1) & 1u, a.err, a.wait_limit)) {
-            timed_out = true;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < C::kGB; ++j) {
-            const int b = g * C::kGB + j;
-            const uint64_t desc = smem_desc_kmajor(xs + b * kQBlockBytes, 128, kQChunkBytes);
-            mma_i8_ts(tmem + C::kDOff + db * C::kDCols + j * C::kN, tmem + ab * C::kACols + 8 * b, desc, idesc,
-                      false);
-          }
-          tc_commit(&dfull[db]);
-        }
-        if (!timed_out) tc_commit(&afree[ab]);
-      }
+      ok = mma_items<C>(a, S, tmem, n, 0);
       // every MMA this thread issued has completed before tensor memory goes
-      tc_commit(drain);
-      if (!mbar_wait(smem_u32(drain), 0, a.err, a.wait_limit)) timed_out = true;
+      tc_commit(S.drain);
+      if (!mbar_wait(smem_u32(S.drain), 0, a.err, a.wait_limit)) ok = false;
     }
     __syncwarp();
   } else if (warp < kUpdateWarp0) {
-    // ---------------- unpack: thread = row, A operand into tensor memory -----
-    const int quarter = warp & 3, r = quarter * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    for (int k = 0; k < n; ++k) {
-      const int ab = k & 1, sw = k % SW;
-      if (!mbar_wait(smem_u32(&wfull[sw]), (uint32_t)(k / SW) & 1u, a.err, a.wait_limit) ||
-          (k >= 2 && !mbar_wait(smem_u32(&afree[ab]), ((k >> 1) - 1) & 1u, a.err, a.wait_limit))) {
-        timed_out = true;
-        break;
-      }
-      tc_fence_after();
-      const uint8_t* q = wring + sw * QB;
-      const uint32_t ta = tmem + lane_base + ab * C::kACols;
-#pragma unroll
-      for (int b = 0; b < 8; ++b) {
-        uint32_t av[8];
-        if constexpr (QT == kQ4_0) {
-          q4_unpack(*reinterpret_cast<const uint4*>(q + q4_off(b, r)), av);
-        } else {
-          const uint4 w0 = *reinterpret_cast<const uint4*>(q + q8_off(b, 0, r));
-          const uint4 w1 = *reinterpret_cast<const uint4*>(q + q8_off(b, 1, r));
-          av[0] = w0.x; av[1] = w0.y; av[2] = w0.z; av[3] = w0.w;
-          av[4] = w1.x; av[5] = w1.y; av[6] = w1.z; av[7] = w1.w;
-        }
-        tmem_st8(ta + 8 * b, av);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(smem_u32(&afull[ab]));
-        mbar_arrive(smem_u32(&wempty[sw]));
-      }
-    }
+    ok = unpack_items<C>(a, S, tmem, n, 0, warp & 3, lane);
   } else {
-    // ---------------- update: thread = row, f32 block updates, tile finish ---
-    const int quarter = warp & 3, r = quarter * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
-    for (int t = quarter; t < NT; t += 4) {
-      const float rs = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
-      if (lane == 0) rstd[t] = rs;
-    }
-    named_sync(kBarUpdate, 128);
-    float acc[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-    uint32_t gc = 0;
-    int tile = i0 / a.chunks;
-    for (int k = 0; k < n; ++k) {
-      const int item = i0 + k, sx = k % SX;
-      if (item / a.chunks != tile) {
-        gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, rstd, ex, flag, quarter, lane);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-        tile = item / a.chunks;
-      }
-      const uint8_t* xsl = xring + sx * XS;
-      uint4 sc4 = make_uint4(0, 0, 0, 0);
-      for (int g = 0; g < C::kNG; ++g, ++gc) {
-        const int db = gc & 1;
-        // the four warps share named barriers in the tile finish, so they
-        // decide together: all go on, or all stop
-        // (the first group also waits for the x slot itself: its scales and
-        // block metadata are read here, not only by the MMA)
-        const bool ok = mbar_wait(smem_u32(&dfull[db]), (gc >> 1) & 1u, a.err, a.wait_limit) &&
-                        (g > 0 || mbar_wait(smem_u32(&xfull[sx]), (uint32_t)(k / SX) & 1u, a.err, a.wait_limit));
-        if (!bar_and(kBarUpdate, 128, ok)) {
-          timed_out = true;
-          break;
-        }
-        tc_fence_after();
-        if (g == 0) sc4 = *reinterpret_cast<const uint4*>(xsl + r * 16);   // the row's 8 block scales
-        int dv[C::kGB][NT][4];
-#pragma unroll
-        for (int j = 0; j < C::kGB; ++j)
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            tmem_ld4(tmem + lane_base + C::kDOff + db * C::kDCols + j * C::kN + t * 8, dv[j][t]);
-        tmem_ld_wait();
-        const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
-#pragma unroll
-        for (int j = 0; j < C::kGB; ++j) {
-          const int b = g * C::kGB + j;
-          const uint32_t w = scw[b >> 1];
-          const float d = __half2float(__ushort_as_half(static_cast<unsigned short>((b & 1) ? (w >> 16) : (w & 0xFFFFu))));
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            const int4 m = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + t * kQChunkBytes +
-                                                          b * kQBlockBytes + kQMetaOff);
-            acc[t] = block_update<QT>(acc[t], d, __int_as_float(m.x), dv[j][t][0], dv[j][t][1], dv[j][t][2], m.y, m.z);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&dfree[db]));
-      }
-      if (timed_out) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&xempty[sx]));
-    }
-    if (!timed_out) gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, rstd, ex, flag, quarter, lane);
+    load_rstd<C>(a, S, warp & 3, lane);
+    ok = update_items<C, EPI>(a, S, tmem, cta, i0, n, 0, warp & 3, lane);
   }
   // ---------------- teardown: tensor memory back, after every MMA and load --
   tc_fence_before();
@@ -575,7 +661,7 @@ __global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) 
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
-  if (timed_out && lane == 0) drain_inflight_copies();   // error path
+  if (!ok && lane == 0) drain_inflight_copies();   // error path
 }
 
 }  // namespace qhl

@@ -52,6 +52,7 @@ struct Layer {
   int out_cols = 0;
   uint8_t* w_gu = nullptr;
   uint8_t* w_down = nullptr;
+  size_t in_bytes = 0, out_bytes = 0, gu_bytes = 0, down_bytes = 0;   // packed sizes, for the launch checks
   float* norm1 = nullptr;
   float* norm2 = nullptr;
   float* qn = nullptr;
@@ -95,6 +96,11 @@ struct stage {
   // one graph per (kind of pass, token count): kind 0 = forward (per-token
   // snapshots), 1 = exact prefill, 2 = chunked prefill (DnMode)
   cudaGraphExec_t exec[3][kMaxTok + 1] = {};
+  // persistent pass: per-layer step arguments on the device, phase counter
+  PassLayer* pass_layers = nullptr;
+  unsigned* bar = nullptr;
+  int n_phases = 0;
+  int pass_mode = STAGE_PASS_KERNELS;
   // failure injection for tests of the bounded waits (stage_debug_inject)
   uint32_t dbg_wait_limit = 0;
   int dbg_fault_item = -1;
@@ -181,22 +187,16 @@ GemvArgs gemv_base(const stage* st) {
 
 void set_workers(const stage* st, GemvArgs& a) { a.workers = gemv_workers(a.tiles, a.chunks, st->sms); }
 
-// The steps of one layer: in-projection, out-projection, gate/up, down, and
-// the mixer between the first two.
-struct LayerSteps {
-  int attn;
-  GemvArgs g[4];
-  DnArgs dn;
-  AttnArgs at;
-};
-
 // Arguments of every step of layer i.
-LayerSteps layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
+// Arguments of the steps of layer i (both execution paths use these, so they
+// run the same units with the same split): in-projection, out-projection,
+// gate/up, down, and the mixer between the first two.
+PassLayer layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
   const stage_config& c = st->cfg;
   const int H = c.hidden, F = c.ffn;
   const Layer& L = st->layers[i];
   const float* next_norm1 = i + 1 < st->layers.size() ? st->layers[i + 1].norm1 : nullptr;
-  LayerSteps P = {};
+  PassLayer P = {};
   P.attn = L.attn ? 1 : 0;
   // mixer in-projection with the RMSNorm1 scale folded into the epilogue
   GemvArgs a = gemv_base(st);
@@ -250,7 +250,7 @@ LayerSteps layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
   // out-projection + residual; z = h * norm2 (block fixed point) and its tile sums of squares
   a = gemv_base(st);
   a.W = L.w_out;
-  a.tiles = H / 64;
+  a.tiles = packed_tiles(H, false);
   a.chunks = L.out_cols / kChunkCols;
   a.qx = st->qo;
   a.qx_stride = st->qo_stride;
@@ -267,7 +267,7 @@ LayerSteps layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
   // gate/up with the RMSNorm2 scale and the SwiGLU epilogue
   a = gemv_base(st);
   a.W = L.w_gu;
-  a.tiles = (F + 31) / 32;
+  a.tiles = packed_tiles(F, true);
   a.chunks = H / kChunkCols;
   a.qx = st->qz;
   a.qx_stride = st->qz_stride;
@@ -282,7 +282,7 @@ LayerSteps layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
   // down + residual; z for the next layer's RMSNorm1
   a = gemv_base(st);
   a.W = L.w_down;
-  a.tiles = H / 64;
+  a.tiles = packed_tiles(H, false);
   a.chunks = F / kChunkCols;
   a.qx = st->qu;
   a.qx_stride = st->qu_stride;
@@ -305,14 +305,68 @@ LayerSteps layer_args(const stage* st, size_t i, int dn_mode = DN_SNAPSHOTS) {
 // kernels: stage input, then per layer in-projection, mixer, out-projection,
 // gate/up, down.  Every kernel after the first is a programmatic dependent of
 // the one before.
+// Every projection streams exactly its packed matrix and writes inside its
+// output: checked on the host before a pass is recorded, so a geometry error
+// fails the recording instead of reaching the device.
+bool gemv_fits(const stage* st, const GemvArgs& a, size_t packed, int out_cap) {
+  const size_t streamed = (size_t)a.tiles * a.chunks * item_bytes(st->cfg.qtype);
+  return streamed == packed && a.workers >= 1 && a.workers <= st->sms && a.out_valid <= out_cap &&
+         a.tiles * (long long)kTileRows >= a.out_valid;
+}
+
+// Whether an n-token forward can run as the one persistent kernel: n within
+// the instantiated range, one CTA per SM resident, and every mixer unit's
+// scratch within the kernel's.
+bool pass_eligible(const stage* st, int n) {
+  if (n > kPassMaxTok || !st->pass_layers) return false;
+  int blocks = 0;
+  if (pass_occupancy(st->cfg.qtype, n, &blocks) != cudaSuccess || blocks < 1) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  const int rep = st->cfg.att_q_heads / st->cfg.att_kv_heads;
+  const int need = std::max({dn_smem_floats(n) * 4, st->nchunk * 3 * 4,
+                             st->nchunk ? attn_smem_bytes(std::min(n, kAttGroup), rep) : 0});
+  return need <= kPassMixBytes;
+}
+
+// One persistent kernel for the whole pass, after zeroing its phase counter.
+cudaError_t record_persistent(stage* st, int n, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(st->bar, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  const stage_config& c = st->cfg;
+  PassArgs p = {};
+  p.layers = st->pass_layers;
+  p.n_layers = (int)st->layers.size();
+  p.h = st->h;
+  p.H = c.hidden;
+  p.gamma0 = st->layers[0].norm1;
+  p.qz = st->qz;
+  p.qz_stride = st->qz_stride;
+  p.ss = st->ss;
+  p.ss_stride = st->ss_stride;
+  p.kv_len = st->ctrl;
+  p.bar = st->bar;
+  p.grid = st->sms;
+  p.dn_units = c.dn_v_heads * (kDnDim / 32);
+  p.Hq = c.att_q_heads;
+  p.Hkv = c.att_kv_heads;
+  p.err = st->err;
+  p.wait_limit = st->dbg_wait_limit;
+  return launch_pass(c.qtype, n, p, s);
+}
+
 cudaError_t record_pass(stage* st, int n, int kind, cudaStream_t s) {
   const stage_config& c = st->cfg;
   const int qt = c.qtype;
+  if (kind == DN_SNAPSHOTS && st->pass_mode == STAGE_PASS_PERSISTENT && st->dbg_fault_item < 0 &&
+      pass_eligible(st, n))
+    return record_persistent(st, n, s);
   cudaError_t e = launch_stage_input(n, st->h, c.hidden, st->layers[0].norm1, st->qz, st->qz_stride, st->ss,
                                      st->ss_stride, s);
   if (e != cudaSuccess) return e;
   for (size_t i = 0; i < st->layers.size(); ++i) {
-    LayerSteps P = layer_args(st, i, kind);
+    PassLayer P = layer_args(st, i, kind);
     // each projection warms L2 with the next one's first items
     auto chain = [](GemvArgs& a, const GemvArgs& next) {
       a.next_W = next.W;
@@ -324,6 +378,10 @@ cudaError_t record_pass(stage* st, int n, int kind, cudaStream_t s) {
     chain(P.g[2], P.g[3]);
     if (i + 1 < st->layers.size()) chain(P.g[3], layer_args(st, i + 1).g[0]);
     if (i == 0) P.g[0].fault_item = st->dbg_fault_item;   // injected failure (tests only)
+    const Layer& L = st->layers[i];
+    if (!gemv_fits(st, P.g[0], L.in_bytes, st->y_stride) || !gemv_fits(st, P.g[1], L.out_bytes, c.hidden) ||
+        !gemv_fits(st, P.g[2], L.gu_bytes, c.ffn) || !gemv_fits(st, P.g[3], L.down_bytes, c.hidden))
+      return cudaErrorInvalidValue;
     if ((e = launch_gemv(qt, n, EPI_STORE, P.g[0], P.g[0].workers, s, kUsePdl)) != cudaSuccess) return e;
     if (!P.attn) {
       if ((e = launch_dn_step(n, P.dn, c.dn_v_heads * (kDnDim / 32), s, kUsePdl)) != cudaSuccess) return e;
@@ -467,9 +525,10 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     L.index = l;
     L.attn = l % c.attn_every == c.attn_every - 1;
     auto T = [&](const char* tag) { return by_name["blk." + std::to_string(l) + "." + tag]; };
-    auto qmat = [&](const stage_tensor* t, int rows, int cols, uint8_t** dst) -> stage_status {
+    auto qmat = [&](const stage_tensor* t, int rows, int cols, uint8_t** dst, size_t* bytes) -> stage_status {
       stage_status r;
       const size_t pb = packed_bytes(qt, rows, cols, false);
+      *bytes = pb;
       if ((r = dalloc_t(st, dst, pb)) != STAGE_OK) return r;
       if ((r = upload(st, stage_a, t)) != STAGE_OK) return r;
       cudaError_t ee = launch_repack(qt, stage_a, nullptr, rows, cols, *dst, nullptr);
@@ -488,8 +547,8 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     if (L.attn) {
       L.in_rows = at_in;
       L.out_cols = at_o;
-      if ((s = qmat(T("attn_in"), at_in, H, &L.w_in)) != STAGE_OK) return bail(s);
-      if ((s = qmat(T("attn_out"), H, at_o, &L.w_out)) != STAGE_OK) return bail(s);
+      if ((s = qmat(T("attn_in"), at_in, H, &L.w_in, &L.in_bytes)) != STAGE_OK) return bail(s);
+      if ((s = qmat(T("attn_out"), H, at_o, &L.w_out, &L.out_bytes)) != STAGE_OK) return bail(s);
       if ((s = vec(T("attn_q_norm"), &L.qn)) != STAGE_OK || (s = vec(T("attn_k_norm"), &L.kn)) != STAGE_OK)
         return bail(s);
       if ((s = dalloc_t(st, &L.K, kv_elems * 2)) != STAGE_OK || (s = dalloc_t(st, &L.V, kv_elems * 2)) != STAGE_OK)
@@ -499,8 +558,8 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     } else {
       L.in_rows = dn_in;
       L.out_cols = dn_o;
-      if ((s = qmat(T("dn_in"), dn_in, H, &L.w_in)) != STAGE_OK) return bail(s);
-      if ((s = qmat(T("dn_out"), H, dn_o, &L.w_out)) != STAGE_OK) return bail(s);
+      if ((s = qmat(T("dn_in"), dn_in, H, &L.w_in, &L.in_bytes)) != STAGE_OK) return bail(s);
+      if ((s = qmat(T("dn_out"), H, dn_o, &L.w_out, &L.out_bytes)) != STAGE_OK) return bail(s);
       const size_t rb = (size_t)kRing * st->state_elems * 4;
       if ((s = dalloc_t(st, &L.ring, rb)) != STAGE_OK) return bail(s);
       if ((e = cudaMemset(L.ring, 0, rb)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
@@ -510,6 +569,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     {
       // gate and up, interleaved tile by tile for the SwiGLU epilogue
       const size_t pb = packed_bytes(qt, F, H, true);
+      L.gu_bytes = pb;
       if ((s = dalloc_t(st, &L.w_gu, pb)) != STAGE_OK) return bail(s);
       if ((s = upload(st, stage_a, T("ffn_gate"))) != STAGE_OK) return bail(s);
       if ((s = upload(st, stage_b, T("ffn_up"))) != STAGE_OK) return bail(s);
@@ -518,7 +578,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
         return bail(fail(st, STAGE_E_CUDA, cuda_msg("repack gate/up", e)));
       st->weight_bytes += pb;
     }
-    if ((s = qmat(T("ffn_down"), H, F, &L.w_down)) != STAGE_OK) return bail(s);
+    if ((s = qmat(T("ffn_down"), H, F, &L.w_down, &L.down_bytes)) != STAGE_OK) return bail(s);
     st->layers.push_back(L);
   }
   // staging no longer needed
@@ -566,6 +626,24 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
     return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemset", e)));
   st->cur.assign(st->n_dn, 0);
 
+  // --- persistent pass: step arguments of every layer, phase numbering -------
+  if ((e = pass_prepare(qt)) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("pass_prepare", e)));
+  {
+    std::vector<PassLayer> pl(st->layers.size());
+    int phase = 1;   // phase 0: stage input
+    for (size_t i = 0; i < pl.size(); ++i) {
+      pl[i] = layer_args(st, i);
+      pl[i].phase_in = phase;
+      phase += pl[i].attn ? 6 : 5;   // in-proj, mixer (attention: partials + combine), out, gate/up, down
+    }
+    st->n_phases = phase;
+    if ((s = dalloc_t(st, &st->pass_layers, pl.size() * sizeof(PassLayer))) != STAGE_OK ||
+        (s = dalloc_t(st, &st->bar, 16)) != STAGE_OK)
+      return bail(s);
+    if ((e = cudaMemcpy(st->pass_layers, pl.data(), pl.size() * sizeof(PassLayer), cudaMemcpyHostToDevice)) !=
+        cudaSuccess)
+      return bail(fail(st, STAGE_E_CUDA, cuda_msg("cudaMemcpy pass layers", e)));
+  }
   if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(fail(st, STAGE_E_CUDA, cuda_msg("load sync", e)));
   *out = st;
   return STAGE_OK;
@@ -787,6 +865,22 @@ static stage_status drop_graphs(stage_t* st) {
         g = nullptr;
       }
   return STAGE_OK;
+}
+
+stage_status stage_set_pass_mode(stage_t* st, int mode) {
+  if (!st) return STAGE_E_ARG;
+  if (mode != STAGE_PASS_KERNELS && mode != STAGE_PASS_PERSISTENT) return fail(st, STAGE_E_ARG, "unknown pass mode");
+  if (st->pending_n) return fail(st, STAGE_E_STATE, "a pass is pending");
+  if (mode == st->pass_mode) return STAGE_OK;
+  stage_status s = drop_graphs(st);
+  if (s != STAGE_OK) return s;
+  st->pass_mode = mode;
+  return STAGE_OK;
+}
+
+int stage_pass_persistent(stage_t* st, int n_tok) {
+  if (!st || n_tok < 1 || n_tok > kMaxTok) return -1;
+  return st->pass_mode == STAGE_PASS_PERSISTENT && st->dbg_fault_item < 0 && pass_eligible(st, n_tok) ? 1 : 0;
 }
 
 stage_status stage_debug_inject(stage_t* st, int fault_item, unsigned wait_limit) {

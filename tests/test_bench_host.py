@@ -33,6 +33,7 @@ def test_launches_per_pass():
     # partials + combine), out-proj, gate/up, down
     assert bench.launches_per_pass(FULL, range(64)) == 1 + 48 * 5 + 16 * 6 == 337
     assert bench.launches_per_pass(FULL, range(0, 4)) == 1 + 3 * 5 + 6
+    assert bench.launches_per_pass(FULL, range(64), persistent=True) == 1
 
 
 class _FakeSmi:

@@ -2,7 +2,7 @@
 hidden 5120, FFN 17408, Q4_0, seed 4) against the oracle, through the C ABI, in
 the launch configuration `bench.py` times (one CUDA graph of kernels per
 token, n_tok 1 from cached position 4096), and in its prefill configuration
-(16-token chunks from position 0).
+(a 16-token chunk from position 0 through stage_prefill, chunked DeltaNet form).
 
 The oracle computes every step on the host's cores (about 8 s per decoded
 token): every element of each output hidden vector is compared, and the
@@ -68,17 +68,22 @@ def test_64_layer_decode_steps_and_prefill_chunk_match_oracle():
                 assert np.array_equal(X[:, :CTX], R[:, :CTX])
 
         # prefill: a new sequence, one 16-token chunk from position 0 (zero
-        # recurrent states, empty cache), against a fresh oracle stage
+        # recurrent states, empty cache) through stage_prefill with the chunked
+        # DeltaNet form (what bench.py times), against a fresh oracle stage
+        # running the token-by-token recurrence
         st.reset()
         orc0 = oracle.OracleStage(FULL, Q4_0, tensors, 0, LAYERS, MAX_CTX)
         h = synth.hidden(FULL, SEED, 500, CHUNK)
-        got = _run(st, h, 0)
+        x = torch.from_numpy(np.ascontiguousarray(h, dtype=np.float32)).cuda()
+        st.prefill(x, 0, chunked=True)
+        torch.cuda.synchronize()
+        st.sync()
+        got = x.cpu().numpy()
         ref = orc0.forward(h, 0)
         errs = rel_err_rows(got, ref)
         assert max(errs) <= TOL, errs
-        st.commit(CHUNK)
         orc0.commit(CHUNK)
-        assert st.committed_len == CHUNK
+        assert st.committed_len == CHUNK and st.pending == 0
         for l in (0, 62):
             assert max(rel_err_heads(st.get_dn_state(l), orc0.S[l])) <= TOL, l
     finally:

@@ -72,9 +72,11 @@ def test_gemv_ragged_shapes(q, qtype, rows, cols, n):
     assert np.all(np.abs(y - ref) <= gemv_error_bound(qtype, W, x))
 
 
+# (1500, 2304): one item per CTA; (4000, 5120): four or five items per CTA
+# through the rings, with stream-K fix-ups
 @pytest.mark.parametrize("qtype", [Q4_0, Q8_0])
-def test_gemv_batched_is_bit_identical_to_single_tokens(q, qtype):
-    rows, cols = 1500, 2304
+@pytest.mark.parametrize("rows,cols", [(1500, 2304), (4000, 5120)])
+def test_gemv_batched_is_bit_identical_to_single_tokens(q, qtype, rows, cols):
     W, x = synth.gemv_problem(21, rows, cols, 16, qtype)
     P = packed_on_gpu(q, qtype, W)
     # every n forms the same exact integer block sums on the tensor cores (MMA
@@ -91,15 +93,16 @@ def test_gemv_batched_is_bit_identical_to_single_tokens(q, qtype):
                                        (FULL.attn_in_rows, FULL.hidden), (FULL.ffn, FULL.hidden),
                                        (FULL.hidden, FULL.ffn)])
 @pytest.mark.parametrize("n", [1, 16])
-def test_gemv_full_size_sampled_rows(q, rows, cols, n):
-    W, x = synth.gemv_problem(31, rows, cols, n)
-    P = packed_on_gpu(q, Q4_0, W)
-    y = gemv_gpu(q, Q4_0, P, rows, cols, x)
+@pytest.mark.parametrize("qtype", [Q4_0, Q8_0])
+def test_gemv_full_size_sampled_rows(q, rows, cols, n, qtype):
+    W, x = synth.gemv_problem(31, rows, cols, n, qtype)
+    P = packed_on_gpu(q, qtype, W)
+    y = gemv_gpu(q, qtype, P, rows, cols, x)
     idx = np.sort(np.random.default_rng(rows + cols).choice(rows, size=min(rows, 192), replace=False))
     idx = np.unique(np.concatenate([idx, [0, rows - 1]]))
-    ref = oracle.qgemv(Q4_0, W[idx], x)             # the oracle computes just these rows
+    ref = oracle.qgemv(qtype, W[idx], x)            # the oracle computes just these rows
     assert max(rel_err_rows(y[:, idx], ref)) <= TOL
-    assert np.all(np.abs(y[:, idx] - ref) <= gemv_error_bound(Q4_0, W[idx], x))
+    assert np.all(np.abs(y[:, idx] - ref) <= gemv_error_bound(qtype, W[idx], x))
 
 
 # ------------------------------------------------------------- dequant --

@@ -458,3 +458,51 @@ def test_chunked_prefill_matches_oracle(q, qtype, n):
         st.rollback()
     finally:
         st.free()
+
+
+@pytest.mark.parametrize("qtype,ns", [(Q4_0, (1, 2, 3, 4)), (Q8_0, (1, 3))])
+def test_persistent_pass_equals_kernel_chain(q, qtype, ns):
+    """The one-kernel persistent pass and the chain of per-step kernels run the
+    same units with the same split: outputs, committed states and new KV rows
+    are bit-identical."""
+    import torch
+    seed = 7
+    st, _, _ = make_pair(FULL, qtype, seed, 0, 4, MAX_CTX, CTX, with_oracle=False)
+    try:
+        assert not st.pass_persistent(1)                      # the chain of kernels by default
+        S0 = _states(st, 0, 4)
+        kv0 = {l: st.get_kv(l) for l in attn_layers(0, 4)}
+        for n in ns:
+            h = synth.hidden(FULL, seed, n, n)
+            res = {}
+            for mode in (q.PASS_PERSISTENT, q.PASS_KERNELS):
+                st.set_pass_mode(mode)
+                assert st.pass_persistent(n) == (mode == q.PASS_PERSISTENT), (n, mode)
+                out = run(st, h, CTX)
+                st.commit(n)
+                res[mode] = (out, _states(st, 0, 4), {l: st.get_kv(l) for l in attn_layers(0, 4)})
+                for l, S in S0.items():                       # back to the starting state
+                    st.set_dn_state(l, S)
+                for l, (K, V) in kv0.items():
+                    st.set_kv(l, K, V)
+                st.set_kv_len(CTX)
+            out_p, S_p, kv_p = res[q.PASS_PERSISTENT]
+            out_k, S_k, kv_k = res[q.PASS_KERNELS]
+            assert np.array_equal(out_p, out_k), n
+            for l in S_p:
+                assert np.array_equal(S_p[l], S_k[l]), (n, l)
+            for l in kv_p:
+                assert np.array_equal(kv_p[l][0], kv_k[l][0]) and np.array_equal(kv_p[l][1], kv_k[l][1]), (n, l)
+        st.set_pass_mode(q.PASS_PERSISTENT)
+        assert not st.pass_persistent(16)                     # 16-token passes run as kernels
+        st.forward(torch.zeros((1, FULL.hidden), device="cuda"), CTX)
+        with pytest.raises(q.StageError) as e:
+            st.set_pass_mode(q.PASS_KERNELS)                  # refused while a pass is pending
+        assert e.value.code == -2
+        st.rollback()
+        with pytest.raises(q.StageError) as e:
+            st.set_pass_mode(5)
+        assert e.value.code == -1
+        st.set_pass_mode(q.PASS_KERNELS)
+    finally:
+        st.free()
