@@ -242,6 +242,11 @@ class Stage:
         """Whether an n_tok forward runs as the persistent kernel."""
         return lib().stage_pass_persistent(self._h, n_tok) == 1
 
+    @property
+    def last_error(self) -> str:
+        """The stage's last error message (stage_last_error)."""
+        return lib().stage_last_error(self._h).decode()
+
     def debug_inject(self, fault_item: int = -1, wait_limit: int = 0):
         """Failure injection for tests of the bounded waits (stage_debug_inject)."""
         self._check(lib().stage_debug_inject(self._h, fault_item, wait_limit))

@@ -7,7 +7,7 @@ namespace {
 
 template <int QT, int NT, int EPI>
 cudaError_t one(const GemvArgs& a, int grid, cudaStream_t s, bool pdl) {
-  return launch_ex(qgemv_kernel<QT, NT, EPI>, dim3(grid), dim3(kGemvCtaThreads), (size_t)gemv_smem_bytes<QT, NT>(), s,
+  return launch_ex(qgemv_kernel<QT, NT, EPI>, dim3(grid), dim3(GemvCfg<QT, NT>::kThreads), (size_t)gemv_smem_bytes<QT, NT>(), s,
                    pdl, a);
 }
 

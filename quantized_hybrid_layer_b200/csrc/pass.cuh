@@ -12,12 +12,18 @@
 // the phase that writes them, and the unpack warps turn the next
 // projection's weights into MMA operands while the previous phase finishes.
 //
-// Warp roles of the CTA (18 warps):
-//   0..7    mixer units (stage input, DeltaNet step, attention partials and
-//           combine), the same device functions as the separate kernels
+// Warp roles of the CTA (14 warps):
+//   0..3    update (the GEMV role of qgemv.cuh, thread = tile row) during the
+//           projection phases, and with 4..7 the mixer units (stage input,
+//           DeltaNet step, attention partials and combine, the same device
+//           functions as the separate kernels) during the mixer phases
+//   4..7    mixer units only
 //   8       producer (one thread): bulk copies of every projection's items
 //   9       MMA issuer (one thread) and tensor-memory owner
-//   10..13  unpack, 14..17 update: the GEMV roles of qgemv.cuh
+//   10..13  unpack
+// The update and the mixer phases of a layer are strictly ordered, so one set
+// of warps serves both; fourteen warps of up to 128 registers fit the
+// register file of an SM's four sub-partitions (at most four warps each).
 // Each CTA arrives once per phase (the update warps for a projection, the
 // mixer warps for a mixer phase); phase p may start once the counter reaches
 // p * grid.  Every wait is bounded; any recorded error makes every wait of
@@ -65,15 +71,17 @@ constexpr int kPassMixBytes = 40 * 1024;
 constexpr int kPassXQueueBytes = 32 * 16;   // the producer's x-job queue, after the mixer scratch
 constexpr int kPassMaxTok = 4;
 
-constexpr int kPassMixWarps = 8;
+constexpr int kPassMixWarps = 8;      // warps 0..7; 0..3 are also the update warps
 constexpr int kPassProducerWarp = 8;
 constexpr int kPassMmaWarp = 9;
 constexpr int kPassUnpackWarp0 = 10;
-constexpr int kPassUpdateWarp0 = 14;
-constexpr int kPassThreads = 18 * 32;
+constexpr int kPassThreads = 14 * 32;
 
 template <int QT, int NT>
-struct PassCfg : GemvGeom<QT, NT, 221 * 1024, 8, 4, 4, 12, kPassMixBytes + kPassXQueueBytes> {};
+struct PassCfg : GemvGeom<QT, NT, 221 * 1024, 8, 4, 4, 12, kPassMixBytes + kPassXQueueBytes> {
+  static constexpr int kUnpackWarps = 4;
+  static constexpr int kMmaThreads = 1;
+};
 
 template <int QT, int NT>
 constexpr int pass_smem_bytes() {
@@ -229,7 +237,7 @@ QHL_DEV bool pass_produce(const PassArgs& p, const GemvSmem<C>& S, int cta, XJob
 }
 
 template <int QT, int NT>
-__global__ void __maxnreg__(112) stage_pass_kernel(const PassArgs p) {
+__global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
   using C = PassCfg<QT, NT>;
   extern __shared__ __align__(16) uint8_t gsmem[];
   const GemvSmem<C> S(gsmem);
@@ -250,22 +258,48 @@ __global__ void __maxnreg__(112) stage_pass_kernel(const PassArgs p) {
       drain_inflight_copies();   // error path
     return;   // the producer takes no part in the tensor-memory teardown
   }
+  uint32_t K = 0;   // this CTA's items so far, over every projection of the pass
   if (warp < kPassMixWarps) {
-    // ---------------- mixer warps: stage input, DeltaNet, attention ----------
+    // ------------- warps 0..7: projection updates (0..3) and mixer units -----
+    const bool upd = warp < 4;
     const bool lead = tid == 0;
-    // phase 0: the stage input (four warps, 128-row tiles)
-    if (warp < 4)
+    // one projection's update (warps 0..3): wait for its phase, run this
+    // CTA's items, arrive
+    auto update = [&](const GemvArgs& a, int gi, int ph) -> bool {
+      if (!group_phase_wait(p, ph, kBarUpdate, 128, lead)) return false;
+      bool good = true;
+      if (cta < a.workers) {
+        const StreamK sk(a.tiles * a.chunks, a.workers);
+        const int i0 = sk.begin(cta), n = sk.begin(cta + 1) - i0;
+        load_rstd<C>(a, S, warp & 3, lane);
+        switch (gi) {
+          case 0: good = update_items<C, EPI_STORE>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+          case 1: good = update_items<C, EPI_RESID>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+          case 2: good = update_items<C, EPI_SWIGLU>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+          default: good = update_items<C, EPI_RESID>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
+        }
+        K += n;
+      }
+      if (good) group_arrive(p, kBarUpdate, 128, lead);
+      return good;
+    };
+    // phase 0: the stage input (warps 0..3, 128-row tiles)
+    if (upd)
       for (int u = cta; u < p.H / kTileRows; u += p.grid)
         input_unit<NT>(p.h, p.H, p.gamma0, p.qz, p.qz_stride, p.ss, p.ss_stride, u, reinterpret_cast<float*>(mix),
                        kBarMix);
     group_arrive(p, kBarMix + 1, 256, lead);
-    for (int l = 0; l < p.n_layers && ok; ++l) {
+    for (int l = 0; l < p.n_layers; ++l) {
       const PassLayer& L = p.layers[l];
       const int ph = L.phase_in + 1;
+      const int ph_out = L.phase_in + (L.attn ? 3 : 2);
+      if (upd && ok) ok = update(L.g[0], 0, L.phase_in);
+      float4 Sr[4];
+      const int u0 = cta;
+      if (!L.attn && ok && u0 < p.dn_units) dn_load<NT>(L.dn, u0, Sr);   // the state rows never depend on this pass
+      // the eight warps agree on going on before any barrier of the mixer
+      if (!(ok = bar_and(kBarMix + 1, 256, ok))) break;
       if (!L.attn) {
-        float4 Sr[4];
-        const int u0 = cta;
-        if (u0 < p.dn_units) dn_load<NT>(L.dn, u0, Sr);   // the state rows never depend on this pass
         if (!(ok = group_phase_wait(p, ph, kBarMix + 1, 256, lead))) break;
         for (int u = u0; u < p.dn_units; u += p.grid) {
           if (u != u0) dn_load<NT>(L.dn, u, Sr);
@@ -291,13 +325,16 @@ __global__ void __maxnreg__(112) stage_pass_kernel(const PassArgs p) {
           combine_unit<NT>(L.at, u / p.Hq, u % p.Hq, pos, reinterpret_cast<float*>(mix));
         group_arrive(p, kBarMix + 1, 256, lead);
       }
+      // out-projection, gate/up, down (warps 0..3; 4..7 go on to the next
+      // layer's agreement, where these four join them)
+      if (upd)
+        for (int gi = 1; gi < 4 && ok; ++gi) ok = update(L.g[gi], gi, ph_out + gi - 1);
     }
-    if (!ok && tid == 0) drain_inflight_copies();
-    return;   // the mixer warps take no part in the tensor-memory teardown
-  }
-
-  uint32_t K = 0;   // this CTA's items so far, over every projection of the pass
-  if (warp == kPassMmaWarp) {
+    if (!upd) {
+      if (!ok && lane == 0) drain_inflight_copies();
+      return;   // warps 4..7 take no part in the tensor-memory teardown
+    }
+  } else if (warp == kPassMmaWarp) {
     if (lane == 0) {
       for (int l = 0; l < p.n_layers && ok; ++l)
         for (int gi = 0; gi < 4 && ok; ++gi) {
@@ -305,7 +342,7 @@ __global__ void __maxnreg__(112) stage_pass_kernel(const PassArgs p) {
           if (cta >= a.workers) continue;
           const StreamK sk(a.tiles * a.chunks, a.workers);
           const int n = sk.begin(cta + 1) - sk.begin(cta);
-          ok = mma_items<C>(a, S, tmem, n, K);
+          ok = mma_items<C>(a, S, tmem, n, K, 0);
           K += n;
         }
       // every MMA this thread issued has completed before tensor memory goes
@@ -313,41 +350,16 @@ __global__ void __maxnreg__(112) stage_pass_kernel(const PassArgs p) {
       if (!mbar_wait(smem_u32(S.drain), 0, p.err, p.wait_limit)) ok = false;
     }
     __syncwarp();
-  } else if (warp < kPassUpdateWarp0) {
+  } else {
     for (int l = 0; l < p.n_layers && ok; ++l)
       for (int gi = 0; gi < 4 && ok; ++gi) {
         const GemvArgs& a = p.layers[l].g[gi];
         if (cta >= a.workers) continue;
         const StreamK sk(a.tiles * a.chunks, a.workers);
         const int n = sk.begin(cta + 1) - sk.begin(cta);
-        ok = unpack_items<C>(a, S, tmem, n, K, warp & 3, lane);
+        ok = unpack_items<C>(a, S, tmem, n, K, warp & 3, 0, lane);
         K += n;
       }
-  } else {
-    // ---------------- update warps: one projection phase after another ------
-    const bool lead = warp == kPassUpdateWarp0 && lane == 0;
-    for (int l = 0; l < p.n_layers && ok; ++l) {
-      const PassLayer& L = p.layers[l];
-      const int ph_out = L.phase_in + (L.attn ? 3 : 2);
-      const int phases[4] = {L.phase_in, ph_out, ph_out + 1, ph_out + 2};
-      for (int gi = 0; gi < 4 && ok; ++gi) {
-        const GemvArgs& a = L.g[gi];
-        if (!(ok = group_phase_wait(p, phases[gi], kBarUpdate, 128, lead))) break;
-        if (cta < a.workers) {
-          const StreamK sk(a.tiles * a.chunks, a.workers);
-          const int i0 = sk.begin(cta), n = sk.begin(cta + 1) - i0;
-          load_rstd<C>(a, S, warp & 3, lane);
-          switch (gi) {
-            case 0: ok = update_items<C, EPI_STORE>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
-            case 1: ok = update_items<C, EPI_RESID>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
-            case 2: ok = update_items<C, EPI_SWIGLU>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
-            default: ok = update_items<C, EPI_RESID>(a, S, tmem, cta, i0, n, K, warp & 3, lane); break;
-          }
-          K += n;
-        }
-        if (ok) group_arrive(p, kBarUpdate, 128, lead);
-      }
-    }
   }
   // ---------------- teardown: tensor memory back, after every MMA and load --
   tc_fence_before();

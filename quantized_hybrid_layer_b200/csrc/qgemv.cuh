@@ -96,12 +96,13 @@ struct StreamK {
   }
 };
 
-// Warp roles.
+// Warp roles: weight producer, MMA issuer, C::kUnpackWarps unpack warps
+// (eight, two per tensor-memory lane quarter and half an item each, where
+// registers allow it; else four), the four update warps, the x producer and
+// the second MMA issuer.
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
-constexpr int kUnpackWarp0 = 2;   // warps 2..5
-constexpr int kUpdateWarp0 = 6;   // warps 6..9
-constexpr int kGemvCtaThreads = 320;
+constexpr int kUnpackWarp0 = 2;
 // Named barriers: 1 = the four update warps, 2 = every warp that touches tensor memory.
 constexpr int kBarUpdate = 1;
 constexpr int kBarTmem = 2;
@@ -120,6 +121,9 @@ struct GemvGeom {
   static constexpr int kDCols = kGB * kN;                           // tensor-memory columns of a D buffer
   static constexpr int kACols = 64;                                 // 8 blocks x 32 bytes / 4
   static constexpr int kNA = NA_, kND = ND_;
+  // One D group per item and as many A as D buffers: a single commit per item
+  // (on dfull) also tells the unpack warps that the item's A buffer is free.
+  static constexpr bool kOneCommit = kNG == 1 && NA_ == ND_;
   static constexpr int kDOff = kNA * kACols;
   static constexpr int kTmemNeed = kDOff + kND * kDCols;
   static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
@@ -127,7 +131,7 @@ struct GemvGeom {
   static constexpr int kXS = QLayout<QT_>::kScaleBytes + kNTP * kQChunkBytes;   // x slot: scales, then tokens
   static constexpr int kSX = SX_;
   static constexpr int kEpi = NT_ * kTileRows * 4;                  // epilogue exchange [NT][128] f32
-  static constexpr int kNumBars = 2 * 16 + 2 * SX_ + 2 * NA_ + 2 * ND_ + 1;   // upper bound (SW <= 16)
+  static constexpr int kNumBars = 2 * 16 + 3 * SX_ + 2 * NA_ + 2 * ND_ + 1;   // upper bound (SW <= 16)
   static constexpr int kFixed = kEpi + 16 * 4 + 16 + kNumBars * 8 + EXTRA;
   static constexpr int kSW0 = (BUDGET - kFixed - SX_ * kXS) / kQB;
   static constexpr int kSW = kSW0 > SWMAX ? SWMAX : kSW0;
@@ -138,8 +142,9 @@ struct GemvGeom {
   static constexpr int kRstdOff = kExtraOff + (EXTRA + 15) / 16 * 16;
   static constexpr int kSlotOff = kRstdOff + 16 * 4;
   static constexpr int kBarOff = kSlotOff + 16;
-  // barriers: wfull[SW], wempty[SW], xfull[SX], xempty[SX], afull[NA], afree[NA], dfull[ND], dfree[ND], drain
-  static constexpr int kSmem = kBarOff + (2 * kSW + 2 * kSX + 2 * kNA + 2 * kND + 1) * 8;
+  // barriers: wfull[SW], wempty[SW], xfull[SX], sfull[SX], xempty[SX], afull[NA], afree[NA], dfull[ND],
+  // dfree[ND], drain
+  static constexpr int kSmem = kBarOff + (2 * kSW + 3 * kSX + 2 * kNA + 2 * kND + 1) * 8;
   static_assert(kSW >= 2 && kSW <= 16, "weight ring depth");
   static_assert(kTmemNeed <= 512, "tensor memory");
   static_assert(kSmem <= BUDGET, "shared-memory budget");
@@ -151,8 +156,19 @@ struct GemvGeom {
 // thread and the update warps each run up to four items apart instead of
 // waiting on one another's latencies.
 template <int QT, int NT>
-struct GemvCfg : GemvGeom<QT, NT, 200 * 1024, NT <= 2 ? 6 : 3, 4, NT <= 8 ? 4 : 2, 12, 0> {
+struct GemvCfg : GemvGeom<QT, NT, 200 * 1024, NT <= 2 ? 16 : (NT <= 8 ? 4 : 2), 4, NT <= 8 ? 4 : 2, 12, 0> {
   static constexpr int kMinBlocks = 1;
+  // Sixteen warps leave 128 registers a thread (four warps per SM
+  // sub-partition), enough up to eight tokens; beyond, twelve warps.
+  static constexpr int kUnpackWarps = NT <= 8 ? 8 : 4;
+  static constexpr int kUpdateWarp0 = kUnpackWarp0 + kUnpackWarps;
+  static constexpr int kXWarp = kUpdateWarp0 + 4;
+  static constexpr int kMma2Warp = kXWarp + 1;
+  static constexpr int kMmaThreads = 2;
+  static constexpr int kThreads = (kMma2Warp + 1) * 32;
+  // each MMA thread waits on its own half of the A, D and x slots (item K
+  // uses A slot K % NA and x slot K % SX, both even counts)
+  static_assert(GemvCfg::kNA % 2 == 0 && GemvCfg::kND % 2 == 0 && GemvCfg::kSX % 2 == 0, "slots per MMA thread");
 };
 
 template <int QT, int NT>
@@ -169,6 +185,40 @@ QHL_DEV bool mbar_test(uint32_t bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of two / three mbarrier phases at once: the tests go out
+// back to back, so a check of barriers that have already completed (the
+// common case in a full pipeline) costs one shared-memory round trip, not one
+// per barrier.  A parity of ((K / depth) - 1) & 1 with K < depth names the
+// phase before a fresh barrier's first, which counts as complete.
+QHL_DEV bool mbar_test2(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q0, q1;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
+      "and.pred q0, q0, q1;\n\t"
+      "selp.u32 %0, 1, 0, q0;\n\t}"
+      : "=r"(ok)
+      : "r"(b0), "r"(p0), "r"(b1), "r"(p1)
+      : "memory");
+  return ok != 0;
+}
+QHL_DEV bool mbar_test3(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1, uint32_t b2, uint32_t p2) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred q0, q1, q2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q2, [%5], %6;\n\t"
+      "and.pred q0, q0, q1;\n\t"
+      "and.pred q0, q0, q2;\n\t"
+      "selp.u32 %0, 1, 0, q0;\n\t}"
+      : "=r"(ok)
+      : "r"(b0), "r"(p0), "r"(b1), "r"(p1), "r"(b2), "r"(p2)
       : "memory");
   return ok != 0;
 }
@@ -324,7 +374,7 @@ struct GemvSmem {
   float* rstd;
   uint32_t* tslot;
   int* flag;
-  uint64_t *wfull, *wempty, *xfull, *xempty, *afull, *afree, *dfull, *dfree, *drain;
+  uint64_t *wfull, *wempty, *xfull, *sfull, *xempty, *afull, *afree, *dfull, *dfree, *drain;
   QHL_DEV explicit GemvSmem(uint8_t* base) {
     wring = base;
     xring = base + C::kXOff;
@@ -336,7 +386,8 @@ struct GemvSmem {
     wfull = reinterpret_cast<uint64_t*>(base + C::kBarOff);
     wempty = wfull + C::kSW;
     xfull = wfull + 2 * C::kSW;
-    xempty = xfull + C::kSX;
+    sfull = xfull + C::kSX;
+    xempty = sfull + C::kSX;
     afull = xempty + C::kSX;
     afree = afull + C::kNA;
     dfull = afree + C::kNA;
@@ -347,24 +398,44 @@ struct GemvSmem {
   QHL_DEV void init() const {
     for (int s = 0; s < C::kSW; ++s) {
       mbar_init(smem_u32(&wfull[s]), 1);
-      mbar_init(smem_u32(&wempty[s]), 4);
+      mbar_init(smem_u32(&wempty[s]), C::kUnpackWarps);
     }
     for (int s = 0; s < C::kSX; ++s) {
       mbar_init(smem_u32(&xfull[s]), 1);
+      mbar_init(smem_u32(&sfull[s]), 1);
       mbar_init(smem_u32(&xempty[s]), 4);
     }
     for (int b = 0; b < C::kNA; ++b) {
-      mbar_init(smem_u32(&afull[b]), 4);
+      mbar_init(smem_u32(&afull[b]), C::kUnpackWarps);
       mbar_init(smem_u32(&afree[b]), 1);
     }
     for (int b = 0; b < C::kND; ++b) {
       mbar_init(smem_u32(&dfull[b]), 1);
       mbar_init(smem_u32(&dfree[b]), 4);
     }
-    mbar_init(smem_u32(drain), 1);
+    mbar_init(smem_u32(drain), C::kMmaThreads);
     fence_mbar_init();
   }
 };
+
+// D buffer of group g of item K and the index of that use among the
+// buffer's uses (its barrier phase).  With two MMA threads each owns half of
+// the buffers (thread K & 1 takes item K), so that every barrier is waited on
+// by one thread, one phase at a time: a parity wait cannot tell a phase from
+// the one two before it.
+template <class C>
+QHL_DEV void d_slot(uint32_t K, int g, int& db, uint32_t& use) {
+  if constexpr (C::kMmaThreads == 1) {
+    const uint32_t gc = K * C::kNG + g;
+    db = gc % C::kND;
+    use = gc / C::kND;
+  } else {
+    constexpr int kOwn = C::kND / 2;
+    const uint32_t lg = (K >> 1) * C::kNG + g;   // the group's index among its thread's groups
+    db = (int)(K & 1u) + 2 * (int)(lg % kOwn);
+    use = lg / kOwn;
+  }
+}
 
 // The roles below process this CTA's items [i0, i0 + n) of one projection.  K0
 // is the running count of items the CTA has taken through its rings before
@@ -383,65 +454,40 @@ QHL_DEV void issue_weights(const GemvArgs& a, const GemvSmem<C>& S, int item, ui
 }
 template <class C>
 QHL_DEV void issue_scales(const GemvArgs& a, const GemvSmem<C>& S, int item, uint32_t K, uint64_t pol) {
-  constexpr int QT = C::kQT, NT = C::kNT;
+  constexpr int QT = C::kQT;
   const int s = K % C::kSX;
-  mbar_arrive_expect_tx(smem_u32(&S.xfull[s]), QLayout<QT>::kScaleBytes + NT * kQChunkBytes);
+  mbar_arrive_expect_tx(smem_u32(&S.sfull[s]), QLayout<QT>::kScaleBytes);
   bulk_g2s(smem_u32(S.xring + s * C::kXS), a.W + (size_t)item * QLayout<QT>::kItemBytes + C::kQB,
-           QLayout<QT>::kScaleBytes, smem_u32(&S.xfull[s]), pol);
+           QLayout<QT>::kScaleBytes, smem_u32(&S.sfull[s]), pol);
 }
 template <class C>
 QHL_DEV void issue_x(const GemvArgs& a, const GemvSmem<C>& S, int chunk, uint32_t K) {
   constexpr int QT = C::kQT, NT = C::kNT;
   const int s = K % C::kSX;
+  mbar_arrive_expect_tx(smem_u32(&S.xfull[s]), NT * kQChunkBytes);
   for (int t = 0; t < NT; ++t)
     bulk_g2s_plain(smem_u32(S.xring + s * C::kXS + QLayout<QT>::kScaleBytes + t * kQChunkBytes),
                    a.qx + (size_t)t * a.qx_stride + (size_t)chunk * kQChunkBytes, kQChunkBytes,
                    smem_u32(&S.xfull[s]));
 }
 
-// Producer of one stand-alone projection (one thread; K0 = 0).  The weights
-// never depend on earlier kernels: the first rings are requested before
-// griddepcontrol.wait, the x columns (written by the previous kernel) once the
-// dependency is resolved.  Returns false on a timeout.
+// Producers of one stand-alone projection (K0 = 0), two threads in two warps
+// so that neither ring waits for the other's slots.  The weight thread keeps
+// the weight ring full: it requests the first SW items at once (the weights
+// never depend on earlier kernels) and then each item as soon as its slot is
+// released, sleeping in the barrier wait in between.  The x thread does the
+// same for the x ring (an item's block scales and x columns); the x columns
+// are written by the previous kernel, so they are requested only once
+// griddepcontrol.wait has returned.  Each returns false on a timeout.
 template <class C>
-QHL_DEV bool produce_items(const GemvArgs& a, const GemvSmem<C>& S, int cta, int i0, int n) {
+QHL_DEV bool produce_weights(const GemvArgs& a, const GemvSmem<C>& S, int cta, int i0, int n) {
   constexpr int QT = C::kQT;
-  constexpr int SW = C::kSW, SX = C::kSX;
+  constexpr int SW = C::kSW;
   const uint64_t pol = policy_evict_first();
-  const int c0 = i0 % a.chunks;
-  auto chunk_of = [&](int k) {   // chunk of local item k, without 64-bit division
-    int c = c0 + k % a.chunks;
-    return c >= a.chunks ? c - a.chunks : c;
-  };
-  auto w = [&](int k) {
-    if (cta == 0 && k == a.fault_item) return;   // injected failure: this slot never fills
+  for (int k = 0; k < n; ++k) {
+    if (k >= SW && !mbar_wait(smem_u32(&S.wempty[k % SW]), ((k / SW) - 1) & 1u, a.err, a.wait_limit)) return false;
+    if (cta == 0 && k == a.fault_item) continue;   // injected failure: this slot never fills
     issue_weights<C>(a, S, i0 + k, (uint32_t)k, pol);
-  };
-  int kw = 0, kx = 0;
-  for (; kw < n && kw < SW; ++kw) w(kw);
-  for (int k = 0; k < n && k < SX; ++k) issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
-  pdl_wait();
-  for (; kx < n && kx < SX; ++kx) issue_x<C>(a, S, chunk_of(kx), (uint32_t)kx);
-  for (uint32_t spins = 0; kw < n || kx < n;) {
-    bool did = false;
-    if (kw < n && mbar_test(smem_u32(&S.wempty[kw % SW]), ((kw / SW) - 1) & 1u)) {
-      w(kw++);
-      did = true;
-    }
-    if (kx < n && mbar_test(smem_u32(&S.xempty[kx % SX]), ((kx / SX) - 1) & 1u)) {
-      issue_scales<C>(a, S, i0 + kx, (uint32_t)kx, pol);
-      issue_x<C>(a, S, chunk_of(kx), (uint32_t)kx);
-      ++kx;
-      did = true;
-    }
-    if (did) {
-      spins = 0;
-    } else if (++spins > wait_limit(a.wait_limit)) {
-      atomicOr(a.err, ERR_WAIT_TIMEOUT);
-      return false;
-    } else {
-      __nanosleep(32);   // both rings full: poll lightly
-    }
   }
   if (a.next_W && cta < a.next_workers) {
     // every own item is on its way: warm L2 with the next projection's first
@@ -453,36 +499,92 @@ QHL_DEV bool produce_items(const GemvArgs& a, const GemvSmem<C>& S, int cta, int
   }
   return true;
 }
+template <class C>
+QHL_DEV bool produce_x(const GemvArgs& a, const GemvSmem<C>& S, int i0, int n) {
+  constexpr int SX = C::kSX;
+  const uint64_t pol = policy_evict_first();
+  int c = i0 % a.chunks;   // chunk of the current item, stepped without division
+  for (int k = 0; k < n && k < SX; ++k) issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
+  pdl_wait();
+  for (int k = 0; k < n; ++k) {
+    if (k >= SX) {
+      if (!mbar_wait(smem_u32(&S.xempty[k % SX]), ((k / SX) - 1) & 1u, a.err, a.wait_limit)) return false;
+      issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
+    }
+    issue_x<C>(a, S, c, (uint32_t)k);
+    if (++c == a.chunks) c = 0;
+  }
+  return true;
+}
 
 // Unpack warps (thread = row r of quarter `quarter`): each item's quants into
-// the A operand in tensor memory.  Returns false on a timeout.
+// the A operand in tensor memory.  With C::kUnpackWarps = 8 two warps share a
+// lane quarter and `part` 0 / 1 takes blocks 0..3 / 4..7 of every item.
+// Returns false on a timeout.
 template <class C>
 QHL_DEV bool unpack_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int n, uint32_t K0, int quarter,
-                          int lane) {
+                          int part, int lane) {
   constexpr int QT = C::kQT;
+  constexpr int kHalves = 8 / C::kUnpackWarps;   // groups of four blocks per warp and item
+  static_assert(C::kUnpackWarps == 4 || C::kUnpackWarps == 8, "unpack warps");
   const int r = quarter * 32 + lane;
   const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
   for (int k = 0; k < n; ++k) {
     const uint32_t K = K0 + k;
     const int ab = K % C::kNA, sw = K % C::kSW;
-    if (!mbar_wait(smem_u32(&S.wfull[sw]), (K / C::kSW) & 1u, a.err, a.wait_limit) ||
-        (K >= C::kNA && !mbar_wait(smem_u32(&S.afree[ab]), ((K / C::kNA) - 1) & 1u, a.err, a.wait_limit)))
+    // the A buffer is free once the MMAs of item K - NA have completed: its
+    // afree barrier, or with one commit per item the dfull barrier of its D
+    // buffer; for K < NA the weight barrier stands in (nothing to wait for)
+    uint32_t b_free = smem_u32(&S.wfull[sw]), p_free = (K / C::kSW) & 1u;
+    if (K >= (uint32_t)C::kNA) {
+      if constexpr (C::kOneCommit) {
+        int db;
+        uint32_t use;
+        d_slot<C>(K - C::kNA, 0, db, use);
+        b_free = smem_u32(&S.dfull[db]);
+        p_free = use & 1u;
+      } else {
+        b_free = smem_u32(&S.afree[ab]);
+        p_free = ((K / C::kNA) - 1) & 1u;
+      }
+    }
+    if (!mbar_test2(smem_u32(&S.wfull[sw]), (K / C::kSW) & 1u, b_free, p_free) &&
+        (!mbar_wait(smem_u32(&S.wfull[sw]), (K / C::kSW) & 1u, a.err, a.wait_limit) ||
+         !mbar_wait(b_free, p_free, a.err, a.wait_limit)))
       return false;
     tc_fence_after();
     const uint8_t* q = S.wring + sw * C::kQB;
     const uint32_t ta = tmem + lane_base + ab * C::kACols;
+    // the row's loads of four blocks first (one round of shared-memory
+    // latency), then one tensor-memory store of the four
 #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      uint32_t av[8];
+    for (int hh = 0; hh < kHalves; ++hh) {
+      const int h = part * kHalves + hh;
+      uint32_t av[32];
       if constexpr (QT == kQ4_0) {
-        q4_unpack(*reinterpret_cast<const uint4*>(q + q4_off(b, r)), av);
+        uint4 w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const uint4*>(q + q4_off(4 * h + j, r));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t blk[8];
+          q4_unpack(w[j], blk);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) av[8 * j + i] = blk[i];
+        }
       } else {
-        const uint4 w0 = *reinterpret_cast<const uint4*>(q + q8_off(b, 0, r));
-        const uint4 w1 = *reinterpret_cast<const uint4*>(q + q8_off(b, 1, r));
-        av[0] = w0.x; av[1] = w0.y; av[2] = w0.z; av[3] = w0.w;
-        av[4] = w1.x; av[5] = w1.y; av[6] = w1.z; av[7] = w1.w;
+        uint4 w[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          w[2 * j] = *reinterpret_cast<const uint4*>(q + q8_off(4 * h + j, 0, r));
+          w[2 * j + 1] = *reinterpret_cast<const uint4*>(q + q8_off(4 * h + j, 1, r));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          av[4 * j] = w[j].x; av[4 * j + 1] = w[j].y; av[4 * j + 2] = w[j].z; av[4 * j + 3] = w[j].w;
+        }
       }
-      tmem_st8(ta + 8 * b, av);
+      tmem_st32(ta + 32 * h, av);
     }
     tmem_st_wait();
     tc_fence_before();
@@ -496,34 +598,47 @@ QHL_DEV bool unpack_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
 }
 
 // MMA issuer (one thread): per item and block one M = 128, N = 8 per token,
-// K = 32 integer MMA into a D buffer.  Returns false on a timeout.
+// K = 32 integer MMA into a D buffer.  With C::kMmaThreads = 2 two threads
+// take alternate items (`sel` = 0 / 1: even / odd running count), so that one
+// thread's barrier checks and bookkeeping overlap the other's MMAs.  Returns
+// false on a timeout.
 template <class C>
-QHL_DEV bool mma_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int n, uint32_t K0) {
+QHL_DEV bool mma_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int n, uint32_t K0, int sel) {
   constexpr int QT = C::kQT;
   constexpr uint32_t idesc = idesc_i8(QT == kQ8_0, kTileRows, C::kN);
   for (int k = 0; k < n; ++k) {
     const uint32_t K = K0 + k;
+    if (C::kMmaThreads == 2 && (int)(K & 1u) != sel) continue;
     const int ab = K % C::kNA, sx = K % C::kSX;
-    if (!mbar_wait(smem_u32(&S.afull[ab]), (K / C::kNA) & 1u, a.err, a.wait_limit) ||
-        !mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit))
+    // fast path: the A buffer, the x slot and the first D buffer all ready
+    int db0;
+    uint32_t use0;
+    d_slot<C>(K, 0, db0, use0);
+    // (use0 = 0: parity 1 names the phase before the fresh barrier's first)
+    const bool ready = mbar_test3(smem_u32(&S.afull[ab]), (K / C::kNA) & 1u, smem_u32(&S.xfull[sx]),
+                                  (K / C::kSX) & 1u, smem_u32(&S.dfree[db0]), (use0 - 1) & 1u);
+    if (!ready && (!mbar_wait(smem_u32(&S.afull[ab]), (K / C::kNA) & 1u, a.err, a.wait_limit) ||
+                   !mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit)))
       return false;
     tc_fence_after();
     const uint32_t xs = smem_u32(S.xring + sx * C::kXS + QLayout<QT>::kScaleBytes);
+    const uint64_t desc0 = smem_desc_kmajor(xs, 128, kQChunkBytes);   // block b: start address + b * 256 / 16
     for (int g = 0; g < C::kNG; ++g) {
-      const uint32_t gc = K * C::kNG + g;
-      const int db = gc % C::kND;
-      if (gc >= C::kND && !mbar_wait(smem_u32(&S.dfree[db]), ((gc / C::kND) - 1) & 1u, a.err, a.wait_limit))
+      int db;
+      uint32_t use;
+      d_slot<C>(K, g, db, use);
+      if (!(ready && g == 0) && use >= 1 && !mbar_wait(smem_u32(&S.dfree[db]), (use - 1) & 1u, a.err, a.wait_limit))
         return false;
       tc_fence_after();
 #pragma unroll
       for (int j = 0; j < C::kGB; ++j) {
         const int b = g * C::kGB + j;
-        const uint64_t desc = smem_desc_kmajor(xs + b * kQBlockBytes, 128, kQChunkBytes);
+        const uint64_t desc = desc0 + (uint64_t)(b * (kQBlockBytes >> 4));
         mma_i8_ts(tmem + C::kDOff + db * C::kDCols + j * C::kN, tmem + ab * C::kACols + 8 * b, desc, idesc, false);
       }
       tc_commit(&S.dfull[db]);
     }
-    tc_commit(&S.afree[ab]);
+    if constexpr (!C::kOneCommit) tc_commit(&S.afree[ab]);
   }
   return true;
 }
@@ -558,15 +673,18 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
     const uint8_t* xsl = S.xring + sx * C::kXS;
     uint4 sc4 = make_uint4(0, 0, 0, 0);
     for (int g = 0; g < C::kNG; ++g) {
-      const uint32_t gc = K * C::kNG + g;
-      const int db = gc % C::kND;
+      int db;
+      uint32_t use;
+      d_slot<C>(K, g, db, use);
       // (the first group also waits for the x slot itself: its scales and
       // block metadata are read here, not only by the MMA).  After a timeout
       // this warp waits for nothing more; the four warps agree on stopping at
       // the next tile boundary, before any named barrier they share.
-      if (!timed_out)
-        timed_out = !(mbar_wait(smem_u32(&S.dfull[db]), (gc / C::kND) & 1u, a.err, a.wait_limit) &&
-                      (g > 0 || mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit)));
+      if (!timed_out && !(g == 0 && mbar_test3(smem_u32(&S.dfull[db]), use & 1u, smem_u32(&S.xfull[sx]),
+                                                (K / C::kSX) & 1u, smem_u32(&S.sfull[sx]), (K / C::kSX) & 1u)))
+        timed_out = !(mbar_wait(smem_u32(&S.dfull[db]), use & 1u, a.err, a.wait_limit) &&
+                      (g > 0 || (mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit) &&
+                                 mbar_wait(smem_u32(&S.sfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit))));
       if (timed_out) continue;
       tc_fence_after();
       if (g == 0) sc4 = *reinterpret_cast<const uint4*>(xsl + r * 16);   // the row's 8 block scales
@@ -615,7 +733,7 @@ QHL_DEV void load_rstd(const GemvArgs& a, const GemvSmem<C>& S, int quarter, int
 }
 
 template <int QT, int NT, int EPI>
-__global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kMinBlocks) qgemv_kernel(const GemvArgs a) {
   using C = GemvCfg<QT, NT>;
   extern __shared__ __align__(16) uint8_t gsmem[];
   const GemvSmem<C> S(gsmem);
@@ -634,21 +752,22 @@ __global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) 
   tc_fence_after();
   const uint32_t tmem = *S.tslot;
 
-  if (warp == kProducerWarp) {
-    if (lane == 0 && !produce_items<C>(a, S, cta, i0, n)) drain_inflight_copies();   // error path
-    return;   // the producer takes no part in the tensor-memory teardown
+  if (warp == kProducerWarp || warp == C::kXWarp) {
+    if (lane == 0 && !(warp == kProducerWarp ? produce_weights<C>(a, S, cta, i0, n) : produce_x<C>(a, S, i0, n)))
+      drain_inflight_copies();   // error path
+    return;   // the producers take no part in the tensor-memory teardown
   }
   bool ok = true;
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp || warp == C::kMma2Warp) {
     if (lane == 0) {
-      ok = mma_items<C>(a, S, tmem, n, 0);
+      ok = mma_items<C>(a, S, tmem, n, 0, warp == kMmaWarp ? 0 : 1);
       // every MMA this thread issued has completed before tensor memory goes
       tc_commit(S.drain);
       if (!mbar_wait(smem_u32(S.drain), 0, a.err, a.wait_limit)) ok = false;
     }
     __syncwarp();
-  } else if (warp < kUpdateWarp0) {
-    ok = unpack_items<C>(a, S, tmem, n, 0, warp & 3, lane);
+  } else if (warp < C::kUpdateWarp0) {
+    ok = unpack_items<C>(a, S, tmem, n, 0, warp & 3, (warp - kUnpackWarp0) >> 2, lane);
   } else {
     pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
     load_rstd<C>(a, S, warp & 3, lane);
@@ -656,7 +775,7 @@ __global__ void __launch_bounds__(kGemvCtaThreads, GemvCfg<QT, NT>::kMinBlocks) 
   }
   // ---------------- teardown: tensor memory back, after every MMA and load --
   tc_fence_before();
-  named_sync(kBarTmem, kGemvCtaThreads - 32);
+  named_sync(kBarTmem, C::kThreads - 64);
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);

@@ -317,17 +317,28 @@ bool gemv_fits(const stage* st, const GemvArgs& a, size_t packed, int out_cap) {
 // Whether an n-token forward can run as the one persistent kernel: n within
 // the instantiated range, one CTA per SM resident, and every mixer unit's
 // scratch within the kernel's.
-bool pass_eligible(const stage* st, int n) {
-  if (n > kPassMaxTok || !st->pass_layers) return false;
+// The reason a pass is not eligible is left in last_error (for diagnosis).
+bool pass_eligible(stage* st, int n) {
+  if (n > kPassMaxTok || !st->pass_layers) {
+    st->last_error = "persistent pass: n_tok above " + std::to_string(kPassMaxTok);
+    return false;
+  }
   int blocks = 0;
-  if (pass_occupancy(st->cfg.qtype, n, &blocks) != cudaSuccess || blocks < 1) {
+  const cudaError_t e = pass_occupancy(st->cfg.qtype, n, &blocks);
+  if (e != cudaSuccess || blocks < 1) {
     (void)cudaGetLastError();
+    st->last_error = "persistent pass: " + (e != cudaSuccess ? cuda_msg("occupancy query", e)
+                                                             : std::string("no CTA fits on an SM"));
     return false;
   }
   const int rep = st->cfg.att_q_heads / st->cfg.att_kv_heads;
   const int need = std::max({dn_smem_floats(n) * 4, st->nchunk * 3 * 4,
                              st->nchunk ? attn_smem_bytes(std::min(n, kAttGroup), rep) : 0});
-  return need <= kPassMixBytes;
+  if (need > kPassMixBytes) {
+    st->last_error = "persistent pass: mixer scratch " + std::to_string(need) + " bytes";
+    return false;
+  }
+  return true;
 }
 
 // One persistent kernel for the whole pass, after zeroing its phase counter.

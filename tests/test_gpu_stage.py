@@ -344,9 +344,18 @@ def test_f16_boundary_matches_the_oracle(q, stage3):
     st.rollback()
     ref = orc.forward(h16.astype(np.float64), pos)
     orc.rollback()
-    assert np.isfinite(got).all()
-    assert max(rel_err_rows(got, ref.astype(np.float16).astype(np.float64))) <= TOL
-    assert max(rel_err_rows(got, ref)) <= TOL
+    # untrained weights grow the hidden state past the binary16 range: an
+    # element whose true value is clearly beyond 65504 must come back as an
+    # infinity of its sign, every other element within the tolerance of the
+    # oracle, relative to the row's largest such element
+    over = np.abs(ref) > 65504.0 * (1 + TOL)
+    inside = np.abs(ref) < 65504.0 * (1 - TOL)
+    assert np.all(np.isinf(got[over]) & (np.sign(got[over]) == np.sign(ref[over])))
+    assert inside.any()
+    for g, r, m in zip(got, ref, inside):
+        if m.any():
+            assert np.isfinite(g[m]).all()
+            assert np.max(np.abs(g[m] - r[m])) / np.max(np.abs(r[m])) <= TOL
     assert st.committed_len == pos
 
 
@@ -477,7 +486,7 @@ def test_persistent_pass_equals_kernel_chain(q, qtype, ns):
             res = {}
             for mode in (q.PASS_PERSISTENT, q.PASS_KERNELS):
                 st.set_pass_mode(mode)
-                assert st.pass_persistent(n) == (mode == q.PASS_PERSISTENT), (n, mode)
+                assert st.pass_persistent(n) == (mode == q.PASS_PERSISTENT), (n, mode, st.last_error)
                 out = run(st, h, CTX)
                 st.commit(n)
                 res[mode] = (out, _states(st, 0, 4), {l: st.get_kv(l) for l in attn_layers(0, 4)})
