@@ -68,19 +68,21 @@ struct PassArgs {
 // to 6 query heads per KV head, the combine's chunk statistics, the DeltaNet
 // unit, the stage input.
 constexpr int kPassMixBytes = 40 * 1024;
-constexpr int kPassXQueueBytes = 32 * 16;   // the producer's x-job queue, after the mixer scratch
 constexpr int kPassMaxTok = 4;
 
 constexpr int kPassMixWarps = 8;      // warps 0..7; 0..3 are also the update warps
-constexpr int kPassProducerWarp = 8;
+constexpr int kPassProducerWarp = 8;  // weights
 constexpr int kPassMmaWarp = 9;
 constexpr int kPassUnpackWarp0 = 10;
-constexpr int kPassThreads = 14 * 32;
+constexpr int kPassXWarp = 14;
+constexpr int kPassMma2Warp = 15;
+constexpr int kPassThreads = 16 * 32;
 
 template <int QT, int NT>
-struct PassCfg : GemvGeom<QT, NT, 221 * 1024, 8, 4, 4, 12, kPassMixBytes + kPassXQueueBytes> {
+struct PassCfg : GemvGeom<QT, NT, 221 * 1024, 8, 4, 4, 12, kPassMixBytes> {
   static constexpr int kUnpackWarps = 4;
-  static constexpr int kMmaThreads = 1;
+  static constexpr int kMmaThreads = 2;
+  static_assert(PassCfg::kNA % 2 == 0 && PassCfg::kND % 2 == 0 && PassCfg::kSX % 2 == 0, "slots per MMA thread");
 };
 
 template <int QT, int NT>
@@ -138,95 +140,109 @@ QHL_DEV void group_arrive(const PassArgs& p, int bar_id, int nthreads, bool lead
   if (leader) red_release_gpu(p.bar);
 }
 
-// Producer (one thread): every projection item of this CTA in pass order.
-// The quants go as soon as a weight slot is free; the scales and x columns of
-// an item wait in a small queue until its phase may start and an x slot is
-// free.  The queue is serviced whenever the thread would otherwise wait.
-// An x part waiting in the producer's queue (shared memory).
-struct XJob {
-  int gemv;            // layer * 4 + projection
-  int item, chunk, phase;
-};
-constexpr int kPassXQueue = 32;
-
-template <class C>
-QHL_DEV bool pass_produce(const PassArgs& p, const GemvSmem<C>& S, int cta, XJob* q) {
-  constexpr int SW = C::kSW, SX = C::kSX;
-  constexpr int kQ = kPassXQueue;   // x jobs whose quants are issued, oldest first
-  int qh = 0, qn = 0;
-  uint32_t KX = 0;        // x parts issued so far
-  unsigned ready = 0;     // phases known to have started
-  // The counter is polled with relaxed loads whose value is read at the next
-  // call, so a poll never stalls the weight copies issued in between; once the
-  // target is seen, one acquiring load orders the phase's data before the x
-  // copies.
-  unsigned polled = 0;
-  bool poll_out = false;
-  uint32_t polls = 0;
-  const uint64_t pol = policy_evict_first();
-  const uint32_t limit = wait_limit(p.wait_limit);
-  // issue the ready head of the queue; false only on an error seen
-  auto service = [&]() -> bool {
-    while (qn > 0) {
-      const XJob& j = q[qh];
-      if ((unsigned)j.phase > ready) {
-        const unsigned target = (unsigned)j.phase * (unsigned)p.grid;
-        if (!poll_out) {
-          polled = ld_relaxed_gpu(p.bar);
-          poll_out = true;
-          return true;
-        }
-        poll_out = false;
-        if (polled < target) return (++polls & 63u) != 0 || ld_relaxed_gpu(p.err) == 0;
-        (void)ld_acquire_gpu(p.bar);
-        ready = (unsigned)j.phase;
-        fence_proxy_async_global();
-      }
-      if (KX >= (uint32_t)SX && !mbar_test(smem_u32(&S.xempty[KX % SX]), ((KX / SX) - 1) & 1u)) return true;
-      const GemvArgs& a = p.layers[j.gemv >> 2].g[j.gemv & 3];
-      issue_scales<C>(a, S, j.item, KX, pol);
-      issue_x<C>(a, S, j.chunk, KX);
-      ++KX;
-      qh = qh + 1 == kQ ? 0 : qh + 1;
-      --qn;
+// This CTA's projection items in pass order: layer, projection, item and its
+// chunk, stepped one item at a time.
+struct PassItems {
+  int l = 0, gi = -1, it = 0, i1 = 0, c = 0;
+  // To the next item; false past the last.
+  QHL_DEV bool next(const PassArgs& p, int cta) {
+    if (gi >= 0 && ++it < i1) {
+      if (++c == p.layers[l].g[gi].chunks) c = 0;
+      return true;
     }
-    return true;
-  };
-  uint32_t K = 0;         // quants issued so far
-  for (int l = 0; l < p.n_layers; ++l) {
-    const PassLayer& L = p.layers[l];
-    const int ph_out = L.phase_in + (L.attn ? 3 : 2);
-    const int phases[4] = {L.phase_in, ph_out, ph_out + 1, ph_out + 2};
-    for (int gi = 0; gi < 4; ++gi) {
-      const GemvArgs& a = L.g[gi];
+    for (;;) {
+      if (++gi == 4) {
+        gi = 0;
+        if (++l >= p.n_layers) return false;
+      }
+      const GemvArgs& a = p.layers[l].g[gi];
       if (cta >= a.workers) continue;
       const StreamK sk(a.tiles * a.chunks, a.workers);
-      const int i0 = sk.begin(cta), i1 = sk.begin(cta + 1);
-      int c = i0 % a.chunks;
-      for (int it = i0; it < i1; ++it, ++K) {
-        // a free weight slot and room in the queue; service the queue meanwhile
-        for (uint32_t spins = 0;; ++spins) {
-          const bool wfree = K < (uint32_t)SW || mbar_test(smem_u32(&S.wempty[K % SW]), ((K / SW) - 1) & 1u);
-          if (wfree && qn < kQ) break;
-          if (!service()) return false;
-          if (spins >= limit) {
-            atomicOr(p.err, ERR_WAIT_TIMEOUT);
-            return false;
-          }
-          __nanosleep(32);
-        }
-        issue_weights<C>(a, S, it, K, pol);
-        int qt = qh + qn;
-        if (qt >= kQ) qt -= kQ;
-        q[qt] = XJob{l * 4 + gi, it, c, phases[gi]};
-        ++qn;
-        if (++c == a.chunks) c = 0;
-        if (!service()) return false;
+      it = sk.begin(cta);
+      i1 = sk.begin(cta + 1);
+      if (it < i1) {
+        c = it % a.chunks;
+        return true;
       }
     }
   }
-  for (uint32_t spins = 0; qn > 0; ++spins) {
-    if (!service()) return false;
+  QHL_DEV const GemvArgs& args(const PassArgs& p) const { return p.layers[l].g[gi]; }
+  // The phase in which the item's x columns are written (and may be read).
+  QHL_DEV int phase(const PassArgs& p) const {
+    const PassLayer& L = p.layers[l];
+    return gi == 0 ? L.phase_in : L.phase_in + (L.attn ? 3 : 2) + gi - 1;
+  }
+};
+
+// Weight producer (one thread): every projection item's quants in pass order,
+// each as soon as its ring slot is released.  The weights never depend on the
+// pass, so the stream runs across phase boundaries.
+template <class C>
+QHL_DEV bool pass_produce_weights(const PassArgs& p, const GemvSmem<C>& S, int cta) {
+  constexpr int SW = C::kSW;
+  const uint64_t pol = policy_evict_first();
+  PassItems w;
+  for (uint32_t K = 0; w.next(p, cta); ++K) {
+    if (K >= (uint32_t)SW && !mbar_wait(smem_u32(&S.wempty[K % SW]), ((K / SW) - 1) & 1u, p.err, p.wait_limit))
+      return false;
+    issue_weights<C>(w.args(p), S, w.it, K, pol);
+  }
+  return true;
+}
+
+// x producer (one thread): every item's block scales and x columns.  Two
+// cursors run over the items: the scales go as soon as the item's x slot is
+// released (they are weights), the x columns once the phase that writes them
+// has completed on every CTA.  The phase counter is polled with relaxed loads
+// whose value is read at the next turn, so a poll never stalls the scale
+// copies; once the target is seen, one acquiring load and a proxy fence order
+// the phase's data before the bulk copies that read it.
+template <class C>
+QHL_DEV bool pass_produce_x(const PassArgs& p, const GemvSmem<C>& S, int cta) {
+  constexpr int SX = C::kSX;
+  const uint64_t pol = policy_evict_first();
+  const uint32_t limit = wait_limit(p.wait_limit);
+  PassItems sc, xc;
+  bool s_ok = sc.next(p, cta), x_ok = xc.next(p, cta);
+  uint32_t KS = 0, KX = 0;   // items whose scales / x columns are requested
+  int ready = 0;             // phases known to have completed before
+  unsigned polled = 0;
+  bool poll_out = false;
+  for (uint32_t spins = 0; x_ok;) {
+    bool did = false;
+    if (s_ok && (KS < (uint32_t)SX || mbar_test(smem_u32(&S.xempty[KS % SX]), ((KS / SX) - 1) & 1u))) {
+      issue_scales<C>(sc.args(p), S, sc.it, KS, pol);
+      ++KS;
+      s_ok = sc.next(p, cta);
+      did = true;
+    }
+    if (KX < KS) {
+      const int ph = xc.phase(p);
+      if (ph > ready) {
+        if (!poll_out) {
+          polled = ld_relaxed_gpu(p.bar);
+          poll_out = true;
+        } else {
+          poll_out = false;
+          if (polled >= (unsigned)ph * (unsigned)p.grid) {
+            (void)ld_acquire_gpu(p.bar);
+            fence_proxy_async_global();
+            ready = ph;
+          }
+        }
+      }
+      if (ph <= ready) {
+        issue_x<C>(xc.args(p), S, xc.c, KX);
+        ++KX;
+        x_ok = xc.next(p, cta);
+        did = true;
+      }
+    }
+    if (did) {
+      spins = 0;
+      continue;
+    }
+    if ((++spins & 63u) == 0 && ld_relaxed_gpu(p.err)) return false;
     if (spins >= limit) {
       atomicOr(p.err, ERR_WAIT_TIMEOUT);
       return false;
@@ -245,7 +261,7 @@ __global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
   const int cta = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  if (tid == 0) S.init();
+  if (warp == kPassProducerWarp) S.init(lane);
   if (warp == kPassMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -254,9 +270,12 @@ __global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
   bool ok = true;
 
   if (warp == kPassProducerWarp) {
-    if (lane == 0 && !pass_produce<C>(p, S, cta, reinterpret_cast<XJob*>(mix + kPassMixBytes)))
-      drain_inflight_copies();   // error path
-    return;   // the producer takes no part in the tensor-memory teardown
+    if (lane == 0 && !pass_produce_weights<C>(p, S, cta)) drain_inflight_copies();   // error path
+    return;   // the producers take no part in the tensor-memory teardown
+  }
+  if (warp == kPassXWarp) {
+    if (lane == 0 && !pass_produce_x<C>(p, S, cta)) drain_inflight_copies();   // error path
+    return;
   }
   uint32_t K = 0;   // this CTA's items so far, over every projection of the pass
   if (warp < kPassMixWarps) {
@@ -334,7 +353,7 @@ __global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
       if (!ok && lane == 0) drain_inflight_copies();
       return;   // warps 4..7 take no part in the tensor-memory teardown
     }
-  } else if (warp == kPassMmaWarp) {
+  } else if (warp == kPassMmaWarp || warp == kPassMma2Warp) {
     if (lane == 0) {
       for (int l = 0; l < p.n_layers && ok; ++l)
         for (int gi = 0; gi < 4 && ok; ++gi) {
@@ -342,7 +361,7 @@ __global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
           if (cta >= a.workers) continue;
           const StreamK sk(a.tiles * a.chunks, a.workers);
           const int n = sk.begin(cta + 1) - sk.begin(cta);
-          ok = mma_items<C>(a, S, tmem, n, K, 0);
+          ok = mma_items<C>(a, S, tmem, n, K, warp == kPassMmaWarp ? 0 : 1);
           K += n;
         }
       // every MMA this thread issued has completed before tensor memory goes
@@ -363,7 +382,7 @@ __global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
   }
   // ---------------- teardown: tensor memory back, after every MMA and load --
   tc_fence_before();
-  named_sync(kBarTmem, 9 * 32);
+  named_sync(kBarTmem, 10 * 32);   // update 0..3, the two MMA warps, unpack 10..13
   if (warp == kPassMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);

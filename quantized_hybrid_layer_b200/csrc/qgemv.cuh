@@ -394,26 +394,26 @@ struct GemvSmem {
     dfree = dfull + C::kND;
     drain = dfree + C::kND;
   }
-  // barrier set-up by one thread
-  QHL_DEV void init() const {
-    for (int s = 0; s < C::kSW; ++s) {
+  // barrier set-up by the 32 lanes of one warp
+  QHL_DEV void init(int lane) const {
+    for (int s = lane; s < C::kSW; s += 32) {
       mbar_init(smem_u32(&wfull[s]), 1);
       mbar_init(smem_u32(&wempty[s]), C::kUnpackWarps);
     }
-    for (int s = 0; s < C::kSX; ++s) {
+    for (int s = lane; s < C::kSX; s += 32) {
       mbar_init(smem_u32(&xfull[s]), 1);
       mbar_init(smem_u32(&sfull[s]), 1);
       mbar_init(smem_u32(&xempty[s]), 4);
     }
-    for (int b = 0; b < C::kNA; ++b) {
+    for (int b = lane; b < C::kNA; b += 32) {
       mbar_init(smem_u32(&afull[b]), C::kUnpackWarps);
       mbar_init(smem_u32(&afree[b]), 1);
     }
-    for (int b = 0; b < C::kND; ++b) {
+    for (int b = lane; b < C::kND; b += 32) {
       mbar_init(smem_u32(&dfull[b]), 1);
       mbar_init(smem_u32(&dfree[b]), 4);
     }
-    mbar_init(smem_u32(drain), C::kMmaThreads);
+    if (lane == 0) mbar_init(smem_u32(drain), C::kMmaThreads);
     fence_mbar_init();
   }
 };
@@ -499,14 +499,54 @@ QHL_DEV bool produce_weights(const GemvArgs& a, const GemvSmem<C>& S, int cta, i
   }
   return true;
 }
+// The x producer is a whole warp.  Its lane 0 bulk-copies each item's block
+// scales and x columns into the x ring as slots are released.  Bulk copies of
+// one SM are served in order, so at the start of a projection the first x
+// columns (a few KB from L2) would queue behind the ring of weight copies just
+// requested; up to two tokens the whole warp moves the first kHead items' x
+// columns through the load/store path instead (each lane loads its 16-byte
+// pieces, stores them and fences them for the tensor core's async proxy).
 template <class C>
-QHL_DEV bool produce_x(const GemvArgs& a, const GemvSmem<C>& S, int i0, int n) {
-  constexpr int SX = C::kSX;
+QHL_DEV bool produce_x(const GemvArgs& a, const GemvSmem<C>& S, int i0, int n, int lane) {
+  constexpr int QT = C::kQT, NT = C::kNT, SX = C::kSX;
+  constexpr int kPer = kQChunkBytes / 16 / 32;      // 16-byte pieces per lane and token
+  constexpr int kHead = NT <= 2 ? 4 / NT : 0;       // items through the load/store path (16 pieces a lane)
+  static_assert(kHead <= SX, "head items take distinct x slots");
   const uint64_t pol = policy_evict_first();
-  int c = i0 % a.chunks;   // chunk of the current item, stepped without division
-  for (int k = 0; k < n && k < SX; ++k) issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
+  if (lane == 0)
+    for (int k = 0; k < n && k < SX; ++k) issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
   pdl_wait();
-  for (int k = 0; k < n; ++k) {
+  int c = i0 % a.chunks;   // chunk of the next item, stepped without division
+  const int nh = min(kHead, n);
+  if constexpr (kHead > 0) {
+    uint4 v[kHead > 0 ? kHead : 1][NT * kPer];
+    int cc = c;
+#pragma unroll
+    for (int j = 0; j < kHead; ++j) {
+      if (j < nh)
+#pragma unroll
+        for (int i = 0; i < NT * kPer; ++i)
+          v[j][i] = ld_cg_once(reinterpret_cast<const uint4*>(a.qx + (size_t)(i / kPer) * a.qx_stride +
+                                                              (size_t)cc * kQChunkBytes) +
+                               (i % kPer) * 32 + lane);
+      if (++cc == a.chunks) cc = 0;
+    }
+#pragma unroll
+    for (int j = 0; j < kHead; ++j)
+      if (j < nh) {
+        uint8_t* slot = S.xring + j * C::kXS + QLayout<QT>::kScaleBytes;
+#pragma unroll
+        for (int i = 0; i < NT * kPer; ++i)
+          *reinterpret_cast<uint4*>(slot + (i / kPer) * kQChunkBytes + ((i % kPer) * 32 + lane) * 16) = v[j][i];
+      }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0)
+      for (int j = 0; j < nh; ++j) mbar_arrive(smem_u32(&S.xfull[j]));
+    c = cc;
+  }
+  if (lane != 0) return true;
+  for (int k = nh; k < n; ++k) {
     if (k >= SX) {
       if (!mbar_wait(smem_u32(&S.xempty[k % SX]), ((k / SX) - 1) & 1u, a.err, a.wait_limit)) return false;
       issue_scales<C>(a, S, i0 + k, (uint32_t)k, pol);
@@ -659,16 +699,18 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t] = 0.f;
   int tile = i0 / a.chunks;
+  int ci = i0 - tile * a.chunks;   // chunk of item k within its tile
   bool timed_out = false;
-  for (int k = 0; k < n; ++k) {
+  for (int k = 0; k < n; ++k, ++ci) {
     const uint32_t K = K0 + k;
-    const int item = i0 + k, sx = K % C::kSX;
-    if (item / a.chunks != tile) {
+    const int sx = K % C::kSX;
+    if (ci == a.chunks) {   // item k starts the next tile: finish this one
       if (!bar_and(kBarUpdate, 128, !timed_out)) return false;
       gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane);
 #pragma unroll
       for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-      tile = item / a.chunks;
+      ++tile;
+      ci = 0;
     }
     const uint8_t* xsl = S.xring + sx * C::kXS;
     uint4 sc4 = make_uint4(0, 0, 0, 0);
@@ -745,17 +787,20 @@ __global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kM
   const int i0 = sk.begin(cta), n = sk.begin(cta + 1) - i0;
   if (n == 0) return;
 
-  if (tid == 0) S.init();
+  if (warp == kProducerWarp) S.init(lane);
   if (warp == kMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *S.tslot;
 
-  if (warp == kProducerWarp || warp == C::kXWarp) {
-    if (lane == 0 && !(warp == kProducerWarp ? produce_weights<C>(a, S, cta, i0, n) : produce_x<C>(a, S, i0, n)))
-      drain_inflight_copies();   // error path
+  if (warp == kProducerWarp) {
+    if (lane == 0 && !produce_weights<C>(a, S, cta, i0, n)) drain_inflight_copies();   // error path
     return;   // the producers take no part in the tensor-memory teardown
+  }
+  if (warp == C::kXWarp) {
+    if (!produce_x<C>(a, S, i0, n, lane) && lane == 0) drain_inflight_copies();   // error path
+    return;
   }
   bool ok = true;
   if (warp == kMmaWarp || warp == C::kMma2Warp) {
