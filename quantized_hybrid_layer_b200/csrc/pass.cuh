@@ -81,6 +81,7 @@ constexpr int kPassThreads = 16 * 32;
 template <int QT, int NT>
 struct PassCfg : GemvGeom<QT, NT, 221 * 1024, 8, 4, 4, 12, kPassMixBytes> {
   static constexpr int kUnpackWarps = 4;
+  static constexpr int kUpdateWarps = 4;
   static constexpr int kMmaThreads = 2;
   static_assert(PassCfg::kNA % 2 == 0 && PassCfg::kND % 2 == 0 && PassCfg::kSX % 2 == 0, "slots per MMA thread");
 };

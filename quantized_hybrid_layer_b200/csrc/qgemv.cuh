@@ -103,9 +103,12 @@ struct StreamK {
 constexpr int kProducerWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kUnpackWarp0 = 2;
-// Named barriers: 1 = the four update warps, 2 = every warp that touches tensor memory.
+// Named barriers: 1 = the (first) four update warps, 2 = every warp that
+// touches tensor memory, 3 = the second four update warps, 4 = all eight.
 constexpr int kBarUpdate = 1;
 constexpr int kBarTmem = 2;
+constexpr int kBarUpdate2 = 3;
+constexpr int kBarUpdateAll = 4;
 
 // Geometry and shared-memory layout of one GEMV configuration: weight type,
 // token count, shared-memory budget, x-ring depth SX, tensor-memory A and D
@@ -155,20 +158,42 @@ struct GemvGeom {
 // four A and four D buffers in tensor memory, so the unpack warps, the MMA
 // thread and the update warps each run up to four items apart instead of
 // waiting on one another's latencies.
+// x-ring depth: up to 140 KB of x slots, leaving at least three weight slots
+// (two of Q8_0's 32 KB beyond eight tokens), an even count from 2 to 16 (a
+// slot holds the block scales and 2 KB per 8-row MMA group).  With many
+// tokens an item's x columns outweigh its quants, and they are requested only
+// when the update warps release a slot, so the ring must cover their latency.
+constexpr int gemv_sx(int qt, int nt) {
+  const int xs = 2048 + (nt == 1 ? 1 : 2 * ((nt + 1) / 2)) * 2048;
+  const int keep = qt == kQ4_0 ? 3 * 16384 : (nt > 8 ? 2 : 3) * 32768;
+  const int room = 213 * 1024 - keep;
+  const int sx = ((room < 140 * 1024 ? room : 140 * 1024) / xs) & ~1;
+  return sx < 2 ? 2 : (sx > 16 ? 16 : sx);
+}
+// Tensor-memory buffers: four A and four D buffers up to eight tokens; beyond,
+// where one D group is 128 columns, two A and three D buffers.
 template <int QT, int NT>
-struct GemvCfg : GemvGeom<QT, NT, 200 * 1024, NT <= 2 ? 16 : (NT <= 8 ? 4 : 2), 4, NT <= 8 ? 4 : 2, 12, 0> {
+struct GemvCfg : GemvGeom<QT, NT, 225 * 1024, gemv_sx(QT, NT), NT <= 8 ? 4 : 2, NT <= 8 ? 4 : 3, 12, 0> {
   static constexpr int kMinBlocks = 1;
-  // Sixteen warps leave 128 registers a thread (four warps per SM
-  // sub-partition), enough up to eight tokens; beyond, twelve warps.
+  // Sixteen warps, 128 registers a thread (four warps per SM sub-partition).
+  // Up to eight tokens: eight unpack warps (half an item each) and four update
+  // warps; beyond, where the f32 updates dominate, four unpack warps and two
+  // sets of four update warps, each set owning half of the tokens.
   static constexpr int kUnpackWarps = NT <= 8 ? 8 : 4;
+  static constexpr int kUpdateWarps = NT <= 8 ? 4 : 8;
+  static constexpr int kNTA = kUpdateWarps == 8 ? (NT + 1) / 2 : NT;   // tokens of the first set
   static constexpr int kUpdateWarp0 = kUnpackWarp0 + kUnpackWarps;
-  static constexpr int kXWarp = kUpdateWarp0 + 4;
+  static constexpr int kXWarp = kUpdateWarp0 + kUpdateWarps;
   static constexpr int kMma2Warp = kXWarp + 1;
-  static constexpr int kMmaThreads = 2;
+  // Two MMA threads where an item is one or two D groups (their barrier
+  // checks and bookkeeping then cost as much as the MMAs); beyond, one thread
+  // that keeps every D buffer in play (the second MMA warp idles).
+  static constexpr int kMmaThreads = NT <= 2 ? 2 : 1;
   static constexpr int kThreads = (kMma2Warp + 1) * 32;
   // each MMA thread waits on its own half of the A, D and x slots (item K
   // uses A slot K % NA and x slot K % SX, both even counts)
-  static_assert(GemvCfg::kNA % 2 == 0 && GemvCfg::kND % 2 == 0 && GemvCfg::kSX % 2 == 0, "slots per MMA thread");
+  static_assert(kMmaThreads == 1 || (GemvCfg::kNA % 2 == 0 && GemvCfg::kND % 2 == 0 && GemvCfg::kSX % 2 == 0),
+                "slots per MMA thread");
 };
 
 template <int QT, int NT>
@@ -260,108 +285,119 @@ QHL_DEV float tile_sumsq(float v, float* red, int quarter, int lane, int bar_id)
   return s;
 }
 
-// Epilogue of one finished tile by the four update warps, thread = tile row r
-// (quarter q = r / 32); v[t] = the tile's final sums for row r.
-template <int EPI, int NT>
-QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, const float (&v)[NT], const float* rstd, float* ex, int quarter,
-                           int lane) {
+// The tokens one set of four update warps owns: [T0, T0 + NTL) of the
+// pass's tokens, with its own named barrier `barq` (128 threads) and the
+// barrier `barall` over every update warp (`nall` threads; the same barrier
+// when one set owns every token).
+struct UpdSlice {
+  int barq, barall, nall;
+};
+
+// Epilogue of one finished tile by a set of four update warps, thread = tile
+// row r (quarter q = r / 32); v[t] = the tile's final sums for row r and
+// token T0 + t.
+template <int EPI, int T0, int NTL>
+QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, const float (&v)[NTL], const float* rstd, float* ex,
+                           int quarter, int lane, const UpdSlice& us) {
   const int r = quarter * 32 + lane;
   if constexpr (EPI == EPI_STORE) {
     const int gr = tile * kTileRows + r;
     if (gr < a.out_valid)
 #pragma unroll
-      for (int t = 0; t < NT; ++t) a.y[(size_t)t * a.y_stride + gr] = __fmul_rn(v[t], rstd[t]);
+      for (int t = 0; t < NTL; ++t) a.y[(size_t)(T0 + t) * a.y_stride + gr] = __fmul_rn(v[t], rstd[T0 + t]);
   } else if constexpr (EPI == EPI_SWIGLU) {
     // rows 0..63: gate rows of features 64 tile + r; rows 64..127 the matching up rows
     if (r >= 64)
 #pragma unroll
-      for (int t = 0; t < NT; ++t) ex[t * kTileRows + r - 64] = __fmul_rn(v[t], rstd[t]);
-    named_sync(kBarUpdate, 128);
+      for (int t = 0; t < NTL; ++t) ex[(T0 + t) * kTileRows + r - 64] = __fmul_rn(v[t], rstd[T0 + t]);
+    named_sync(us.barq, 128);
     if (r < 64) {
       const int f = tile * 64 + r;
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
+      for (int t = 0; t < NTL; ++t) {
         float u = 0.f;
         if (f < a.out_valid) {
-          const float g = __fmul_rn(v[t], rstd[t]);
-          const float up = ex[t * kTileRows + r];
+          const float g = __fmul_rn(v[t], rstd[T0 + t]);
+          const float up = ex[(T0 + t) * kTileRows + r];
           u = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), up);   // silu(g) * up
         }
-        qact_store_block(u, a.qout + (size_t)t * a.qout_stride, tile * 2 + quarter, lane);
+        qact_store_block(u, a.qout + (size_t)(T0 + t) * a.qout_stride, tile * 2 + quarter, lane);
       }
     }
-    named_sync(kBarUpdate, 128);
+    named_sync(us.barq, 128);
   } else {
     const int gr = tile * kTileRows + r;
     const bool valid = gr < a.out_valid;
     const float gam = a.qout && valid ? __ldg(a.gamma_next + gr) : 0.f;
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
+    for (int t = 0; t < NTL; ++t) {
+      const int tg = T0 + t;
       float hn = 0.f;
       if (valid) {
-        hn = __fadd_rn(__ldcg(a.y + (size_t)t * a.y_stride + gr), v[t]);
-        a.y[(size_t)t * a.y_stride + gr] = hn;
+        hn = __fadd_rn(__ldcg(a.y + (size_t)tg * a.y_stride + gr), v[t]);
+        a.y[(size_t)tg * a.y_stride + gr] = hn;
       }
-      if (a.qout) qact_store_block(__fmul_rn(hn, gam), a.qout + (size_t)t * a.qout_stride, tile * 4 + quarter, lane);
+      if (a.qout) qact_store_block(__fmul_rn(hn, gam), a.qout + (size_t)tg * a.qout_stride, tile * 4 + quarter, lane);
       if (a.ss_out) {
-        const float s = tile_sumsq(hn, ex + 4 * t, quarter, lane, kBarUpdate);
-        if (r == 0) a.ss_out[(size_t)t * a.ss_out_stride + tile] = s;
+        const float s = tile_sumsq(hn, ex + 4 * tg, quarter, lane, us.barq);
+        if (r == 0) a.ss_out[(size_t)tg * a.ss_out_stride + tile] = s;
       }
     }
   }
 }
 
-// Update warps: finish tile `tl` given this CTA's partial v (stream-K fix-up
-// if the tile is shared, then the epilogue).
-template <int EPI, int NT>
-QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int i0, int i1, int tl, float (&v)[NT],
-                              const float* rstd, float* ex, int* flag, int quarter, int lane) {
+// Update warps: finish tile `tl` given this CTA's partial v for tokens
+// [T0, T0 + NTL) (stream-K fix-up if the tile is shared, then the epilogue).
+// Every update warp of the CTA takes part: one decision per tile.
+template <int EPI, int NT, int T0, int NTL>
+QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int i0, int i1, int tl, float (&v)[NTL],
+                              const float* rstd, float* ex, int* flag, int quarter, int lane, const UpdSlice& us) {
   const int r = quarter * 32 + lane;
   const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
   if (t_lo >= i0 && t_hi <= i1) {
-    gemv_epilogue<EPI, NT>(a, tl, v, rstd, ex, quarter, lane);
+    gemv_epilogue<EPI, T0, NTL>(a, tl, v, rstd, ex, quarter, lane, us);
     return;
   }
   // publish this CTA's partial (slot 0: its first tile, slot 1: its last)
   const int first_tile = i0 / a.chunks;
   float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * kTileRows;
 #pragma unroll
-  for (int t = 0; t < NT; ++t) mine[t * kTileRows + r] = v[t];
+  for (int t = 0; t < NTL; ++t) mine[(T0 + t) * kTileRows + r] = v[t];
   __threadfence();
-  named_sync(kBarUpdate, 128);
+  named_sync(us.barall, us.nall);
   const int cf = sk.owner(t_lo), cl = sk.owner(t_hi - 1);
-  if (r == 0) *flag = counter_add_acq_rel(&a.counters[tl]) == cl - cf ? 1 : 0;
-  named_sync(kBarUpdate, 128);
+  if (T0 == 0 && r == 0) *flag = counter_add_acq_rel(&a.counters[tl]) == cl - cf ? 1 : 0;
+  named_sync(us.barall, us.nall);
   const int last = *flag;
-  named_sync(kBarUpdate, 128);
+  named_sync(us.barall, us.nall);
   if (!last) return;
   __threadfence();   // every thread orders its partial loads after the acquire above
   // combine every contributor's partial in CTA order; tile tl is the first
   // tile of every contributor after cf, and of cf exactly when cf's range
   // starts at the tile's first item
   const int cf_slot = sk.begin(cf) == t_lo ? 0 : 1;
-  float acc[NT];
+  float acc[NTL];
   constexpr int CB = 4;
   for (int c0 = cf; c0 <= cl; c0 += CB) {
-    float pv[CB][NT];
+    float pv[CB][NTL];
 #pragma unroll
     for (int k = 0; k < CB; ++k) {
       const int c = c0 + k;
       if (c <= cl) {
         const float* pc = a.partials + (size_t)(2 * c + (c == cf ? cf_slot : 0)) * NT * kTileRows;
 #pragma unroll
-        for (int t = 0; t < NT; ++t) pv[k][t] = c == cta ? v[t] : ld_cg_once(pc + t * kTileRows + r);
+        for (int t = 0; t < NTL; ++t) pv[k][t] = c == cta ? v[t] : ld_cg_once(pc + (T0 + t) * kTileRows + r);
       }
     }
 #pragma unroll
     for (int k = 0; k < CB; ++k)
       if (c0 + k <= cl) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = (c0 + k == cf) ? pv[k][t] : __fadd_rn(acc[t], pv[k][t]);
+        for (int t = 0; t < NTL; ++t) acc[t] = (c0 + k == cf) ? pv[k][t] : __fadd_rn(acc[t], pv[k][t]);
       }
   }
-  gemv_epilogue<EPI, NT>(a, tl, acc, rstd, ex, quarter, lane);
-  if (r == 0) a.counters[tl] = 0;
+  gemv_epilogue<EPI, T0, NTL>(a, tl, acc, rstd, ex, quarter, lane, us);
+  if (T0 == 0 && r == 0) a.counters[tl] = 0;
 }
 
 // Pointers of one CTA's GEMV machinery in shared memory (layout of config C).
@@ -403,7 +439,7 @@ struct GemvSmem {
     for (int s = lane; s < C::kSX; s += 32) {
       mbar_init(smem_u32(&xfull[s]), 1);
       mbar_init(smem_u32(&sfull[s]), 1);
-      mbar_init(smem_u32(&xempty[s]), 4);
+      mbar_init(smem_u32(&xempty[s]), C::kUpdateWarps);
     }
     for (int b = lane; b < C::kNA; b += 32) {
       mbar_init(smem_u32(&afull[b]), C::kUnpackWarps);
@@ -411,7 +447,7 @@ struct GemvSmem {
     }
     for (int b = lane; b < C::kND; b += 32) {
       mbar_init(smem_u32(&dfull[b]), 1);
-      mbar_init(smem_u32(&dfree[b]), 4);
+      mbar_init(smem_u32(&dfree[b]), C::kUpdateWarps);
     }
     if (lane == 0) mbar_init(smem_u32(drain), C::kMmaThreads);
     fence_mbar_init();
@@ -683,21 +719,22 @@ QHL_DEV bool mma_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, i
   return true;
 }
 
-// Update warps (thread = row r of quarter `quarter`, the four warps of
-// kBarUpdate): f32 block updates of every item in order, then the tile finish
-// at each tile boundary.  rstd[] must hold the input's RMS scale.  The four
-// warps take every decision together.  Returns false on a timeout.
-template <class C, int EPI>
+// Update warps (thread = row r of quarter `quarter`; one set of four warps per
+// token slice [T0, T0 + NTL)): f32 block updates of every item in order, then
+// the tile finish at each tile boundary.  rstd[] must hold the input's RMS
+// scale.  The update warps take every decision together.  Returns false on a
+// timeout.
+template <class C, int EPI, int T0, int NTL>
 QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int cta, int i0, int n,
-                          uint32_t K0, int quarter, int lane) {
+                          uint32_t K0, int quarter, int lane, const UpdSlice& us) {
   constexpr int QT = C::kQT, NT = C::kNT;
   const int r = quarter * 32 + lane;
   const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
   const StreamK sk(a.tiles * a.chunks, a.workers);
   const int i1 = i0 + n;
-  float acc[NT];
+  float acc[NTL];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+  for (int t = 0; t < NTL; ++t) acc[t] = 0.f;
   int tile = i0 / a.chunks;
   int ci = i0 - tile * a.chunks;   // chunk of item k within its tile
   bool timed_out = false;
@@ -705,10 +742,10 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
     const uint32_t K = K0 + k;
     const int sx = K % C::kSX;
     if (ci == a.chunks) {   // item k starts the next tile: finish this one
-      if (!bar_and(kBarUpdate, 128, !timed_out)) return false;
-      gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane);
+      if (!bar_and(us.barall, us.nall, !timed_out)) return false;
+      gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane, us);
 #pragma unroll
-      for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+      for (int t = 0; t < NTL; ++t) acc[t] = 0.f;
       ++tile;
       ci = 0;
     }
@@ -720,8 +757,8 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
       d_slot<C>(K, g, db, use);
       // (the first group also waits for the x slot itself: its scales and
       // block metadata are read here, not only by the MMA).  After a timeout
-      // this warp waits for nothing more; the four warps agree on stopping at
-      // the next tile boundary, before any named barrier they share.
+      // this warp waits for nothing more; the update warps agree on stopping
+      // at the next tile boundary, before any named barrier they share.
       if (!timed_out && !(g == 0 && mbar_test3(smem_u32(&S.dfull[db]), use & 1u, smem_u32(&S.xfull[sx]),
                                                 (K / C::kSX) & 1u, smem_u32(&S.sfull[sx]), (K / C::kSX) & 1u)))
         timed_out = !(mbar_wait(smem_u32(&S.dfull[db]), use & 1u, a.err, a.wait_limit) &&
@@ -730,12 +767,12 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
       if (timed_out) continue;
       tc_fence_after();
       if (g == 0) sc4 = *reinterpret_cast<const uint4*>(xsl + r * 16);   // the row's 8 block scales
-      int dv[C::kGB][NT][4];
+      int dv[C::kGB][NTL][4];
 #pragma unroll
       for (int j = 0; j < C::kGB; ++j)
 #pragma unroll
-        for (int t = 0; t < NT; ++t)
-          tmem_ld4(tmem + lane_base + C::kDOff + db * C::kDCols + j * C::kN + t * 8, dv[j][t]);
+        for (int t = 0; t < NTL; ++t)
+          tmem_ld4(tmem + lane_base + C::kDOff + db * C::kDCols + j * C::kN + (T0 + t) * 8, dv[j][t]);
       tmem_ld_wait();
       const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
@@ -744,8 +781,8 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
         const uint32_t w = scw[b >> 1];
         const float d = __half2float(__ushort_as_half(static_cast<unsigned short>((b & 1) ? (w >> 16) : (w & 0xFFFFu))));
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const int4 m = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + t * kQChunkBytes +
+        for (int t = 0; t < NTL; ++t) {
+          const int4 m = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + (T0 + t) * kQChunkBytes +
                                                         b * kQBlockBytes + kQMetaOff);
           acc[t] = block_update<QT>(acc[t], d, __int_as_float(m.x), dv[j][t][0], dv[j][t][1], dv[j][t][2], m.y, m.z);
         }
@@ -757,21 +794,29 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
     __syncwarp();
     if (!timed_out && lane == 0) mbar_arrive(smem_u32(&S.xempty[sx]));
   }
-  if (!bar_and(kBarUpdate, 128, !timed_out)) return false;
-  gemv_finish_tile<EPI, NT>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane);
+  if (!bar_and(us.barall, us.nall, !timed_out)) return false;
+  gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane, us);
   return true;
 }
+// One set of four update warps owning every token.
+template <class C, int EPI>
+QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem, int cta, int i0, int n,
+                          uint32_t K0, int quarter, int lane) {
+  return update_items<C, EPI, 0, C::kNT>(a, S, tmem, cta, i0, n, K0, quarter, lane,
+                                         UpdSlice{kBarUpdate, kBarUpdate, 128});
+}
 
-// The input's RMS scale per token into S.rstd (update warps; after the
-// dependency on the kernel that wrote ss_in is resolved).
+// The input's RMS scale of tokens [t0, t0 + nt) into S.rstd (one set of
+// four update warps, barrier `bar`; after the dependency on the kernel that
+// wrote ss_in is resolved).
 template <class C>
-QHL_DEV void load_rstd(const GemvArgs& a, const GemvSmem<C>& S, int quarter, int lane) {
-  constexpr int NT = C::kNT;
-  for (int t = quarter; t < NT; t += 4) {
+QHL_DEV void load_rstd(const GemvArgs& a, const GemvSmem<C>& S, int quarter, int lane, int t0 = 0, int nt = C::kNT,
+                       int bar = kBarUpdate) {
+  for (int t = t0 + quarter; t < t0 + nt; t += 4) {
     const float rs = a.ss_in ? rstd_warp(a.ss_in + (size_t)t * a.ss_stride, a.ss_tiles, a.inv_dim, a.eps, lane) : 1.f;
     if (lane == 0) S.rstd[t] = rs;
   }
-  named_sync(kBarUpdate, 128);
+  named_sync(bar, 128);
 }
 
 template <int QT, int NT, int EPI>
@@ -804,7 +849,7 @@ __global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kM
   }
   bool ok = true;
   if (warp == kMmaWarp || warp == C::kMma2Warp) {
-    if (lane == 0) {
+    if (lane == 0 && (warp == kMmaWarp || C::kMmaThreads == 2)) {
       ok = mma_items<C>(a, S, tmem, n, 0, warp == kMmaWarp ? 0 : 1);
       // every MMA this thread issued has completed before tensor memory goes
       tc_commit(S.drain);
@@ -815,8 +860,21 @@ __global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kM
     ok = unpack_items<C>(a, S, tmem, n, 0, warp & 3, (warp - kUnpackWarp0) >> 2, lane);
   } else {
     pdl_wait();   // ss_in, the residual stream and the scratch come from earlier kernels
-    load_rstd<C>(a, S, warp & 3, lane);
-    ok = update_items<C, EPI>(a, S, tmem, cta, i0, n, 0, warp & 3, lane);
+    if constexpr (C::kUpdateWarps == 4) {
+      load_rstd<C>(a, S, warp & 3, lane);
+      ok = update_items<C, EPI>(a, S, tmem, cta, i0, n, 0, warp & 3, lane);
+    } else {
+      constexpr int NA = C::kNTA;
+      if (warp < C::kUpdateWarp0 + 4) {
+        load_rstd<C>(a, S, warp & 3, lane, 0, NA, kBarUpdate);
+        ok = update_items<C, EPI, 0, NA>(a, S, tmem, cta, i0, n, 0, warp & 3, lane,
+                                         UpdSlice{kBarUpdate, kBarUpdateAll, 256});
+      } else {
+        load_rstd<C>(a, S, warp & 3, lane, NA, NT - NA, kBarUpdate2);
+        ok = update_items<C, EPI, NA, NT - NA>(a, S, tmem, cta, i0, n, 0, warp & 3, lane,
+                                               UpdSlice{kBarUpdate2, kBarUpdateAll, 256});
+      }
+    }
   }
   // ---------------- teardown: tensor memory back, after every MMA and load --
   tc_fence_before();
