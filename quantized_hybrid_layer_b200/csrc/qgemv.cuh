@@ -232,6 +232,21 @@ QHL_DEV bool mbar_test2(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1) {
       : "memory");
   return ok != 0;
 }
+// The two phases' states as bits 0 and 1, in one round trip.
+QHL_DEV uint32_t mbar_test2m(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1) {
+  uint32_t m;
+  asm volatile(
+      "{\n\t.reg .pred q0, q1;\n\t.reg .b32 r0, r1;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
+      "selp.u32 r0, 1, 0, q0;\n\t"
+      "selp.u32 r1, 2, 0, q1;\n\t"
+      "or.b32 %0, r0, r1;\n\t}"
+      : "=r"(m)
+      : "r"(b0), "r"(p0), "r"(b1), "r"(p1)
+      : "memory");
+  return m;
+}
 QHL_DEV bool mbar_test3(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1, uint32_t b2, uint32_t p2) {
   uint32_t ok;
   asm volatile(
@@ -751,16 +766,31 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
     }
     const uint8_t* xsl = S.xring + sx * C::kXS;
     uint4 sc4 = make_uint4(0, 0, 0, 0);
+    uint32_t known = 0;   // groups of this item whose D is known to be complete
     for (int g = 0; g < C::kNG; ++g) {
       int db;
       uint32_t use;
       d_slot<C>(K, g, db, use);
       // (the first group also waits for the x slot itself: its scales and
-      // block metadata are read here, not only by the MMA).  After a timeout
-      // this warp waits for nothing more; the update warps agree on stopping
-      // at the next tile boundary, before any named barrier they share.
-      if (!timed_out && !(g == 0 && mbar_test3(smem_u32(&S.dfull[db]), use & 1u, smem_u32(&S.xfull[sx]),
-                                                (K / C::kSX) & 1u, smem_u32(&S.sfull[sx]), (K / C::kSX) & 1u)))
+      // block metadata are read here, not only by the MMA; later groups test
+      // the next group's D in the same round trip).  After a timeout this
+      // warp waits for nothing more; the update warps agree on stopping at the
+      // next tile boundary, before any named barrier they share.
+      bool ready = (known >> g) & 1u;
+      if (!timed_out && !ready && g > 0) {
+        if (g + 1 < C::kNG) {
+          int db1;
+          uint32_t use1;
+          d_slot<C>(K, g + 1, db1, use1);
+          const uint32_t m = mbar_test2m(smem_u32(&S.dfull[db]), use & 1u, smem_u32(&S.dfull[db1]), use1 & 1u);
+          ready = m & 1u;
+          if (m == 3u) known |= 1u << (g + 1);
+        } else {
+          ready = mbar_test(smem_u32(&S.dfull[db]), use & 1u);
+        }
+      }
+      if (!timed_out && !ready && !(g == 0 && mbar_test3(smem_u32(&S.dfull[db]), use & 1u, smem_u32(&S.xfull[sx]),
+                                                         (K / C::kSX) & 1u, smem_u32(&S.sfull[sx]), (K / C::kSX) & 1u)))
         timed_out = !(mbar_wait(smem_u32(&S.dfull[db]), use & 1u, a.err, a.wait_limit) &&
                       (g > 0 || (mbar_wait(smem_u32(&S.xfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit) &&
                                  mbar_wait(smem_u32(&S.sfull[sx]), (K / C::kSX) & 1u, a.err, a.wait_limit))));
