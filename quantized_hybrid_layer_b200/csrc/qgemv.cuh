@@ -361,35 +361,72 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, const float (&v)[NTL], c
   }
 }
 
-// Update warps: finish tile `tl` given this CTA's partial v for tokens
-// [T0, T0 + NTL) (stream-K fix-up if the tile is shared, then the epilogue).
-// Every update warp of the CTA takes part: one decision per tile.
+// bar.red.or over the `nthreads` threads of named barrier `id`.
+QHL_DEV bool bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+// A shared tile whose partial this CTA has published: its counter's old value
+// (held by the thread that added to it) and the count that makes this CTA the
+// tile's last contributor.
+struct TilePend {
+  int tile = -1, old = 0, need = 0;
+};
+
+// Update warps, stream-K: finish tile `tl` given this CTA's partial v for
+// tokens [T0, T0 + NTL).  A tile the CTA owns whole goes straight to the
+// epilogue.  Otherwise the partial is published (slot 0: the CTA's first
+// tile, slot 1: its last) and counted, and the count's answer is left
+// pending, to be read by tile_resolve at the end of the CTA's range, so that
+// the memory round trip never stalls the update warps mid-stream.  Every
+// update warp of the CTA takes part.
 template <int EPI, int NT, int T0, int NTL>
 QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int i0, int i1, int tl, float (&v)[NTL],
-                              const float* rstd, float* ex, int* flag, int quarter, int lane, const UpdSlice& us) {
+                              const float* rstd, float* ex, TilePend& pend, int quarter, int lane,
+                              const UpdSlice& us) {
   const int r = quarter * 32 + lane;
   const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
   if (t_lo >= i0 && t_hi <= i1) {
     gemv_epilogue<EPI, T0, NTL>(a, tl, v, rstd, ex, quarter, lane, us);
     return;
   }
-  // publish this CTA's partial (slot 0: its first tile, slot 1: its last)
   const int first_tile = i0 / a.chunks;
   float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * kTileRows;
 #pragma unroll
   for (int t = 0; t < NTL; ++t) mine[(T0 + t) * kTileRows + r] = v[t];
-  __threadfence();
-  named_sync(us.barall, us.nall);
-  const int cf = sk.owner(t_lo), cl = sk.owner(t_hi - 1);
-  if (T0 == 0 && r == 0) *flag = counter_add_acq_rel(&a.counters[tl]) == cl - cf ? 1 : 0;
-  named_sync(us.barall, us.nall);
-  const int last = *flag;
-  named_sync(us.barall, us.nall);
+  named_sync(us.barall, us.nall);   // every update thread's partial stores come before the release below
+  pend.tile = tl;
+  pend.need = sk.owner(t_hi - 1) - sk.owner(t_lo);
+  if (T0 == 0 && r == 0) {
+    __threadfence();
+    pend.old = atomicAdd(&a.counters[tl], 1);   // read in tile_resolve
+  }
+}
+
+// Read a pending tile's count: if this CTA was the tile's last contributor,
+// sum every contributor's partial in CTA order (tile tl is the first tile of
+// every contributor after cf, and of cf exactly when cf's range starts at the
+// tile's first item) and run the epilogue.
+template <int EPI, int NT, int T0, int NTL>
+QHL_DEV void tile_resolve(const GemvArgs& a, const StreamK& sk, TilePend& pend, const float* rstd, float* ex,
+                          int quarter, int lane, const UpdSlice& us) {
+  const int r = quarter * 32 + lane;
+  const int tl = pend.tile;
+  const bool last = bar_or(us.barall, us.nall, T0 == 0 && r == 0 && pend.old == pend.need);
+  pend.tile = -1;
   if (!last) return;
-  __threadfence();   // every thread orders its partial loads after the acquire above
-  // combine every contributor's partial in CTA order; tile tl is the first
-  // tile of every contributor after cf, and of cf exactly when cf's range
-  // starts at the tile's first item
+  __threadfence();   // every thread orders its partial loads after the count
+  const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
+  const int cf = sk.owner(t_lo), cl = sk.owner(t_hi - 1);
   const int cf_slot = sk.begin(cf) == t_lo ? 0 : 1;
   float acc[NTL];
   constexpr int CB = 4;
@@ -401,7 +438,7 @@ QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int
       if (c <= cl) {
         const float* pc = a.partials + (size_t)(2 * c + (c == cf ? cf_slot : 0)) * NT * kTileRows;
 #pragma unroll
-        for (int t = 0; t < NTL; ++t) pv[k][t] = c == cta ? v[t] : ld_cg_once(pc + (T0 + t) * kTileRows + r);
+        for (int t = 0; t < NTL; ++t) pv[k][t] = ld_cg_once(pc + (T0 + t) * kTileRows + r);
       }
     }
 #pragma unroll
@@ -753,12 +790,15 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
   int tile = i0 / a.chunks;
   int ci = i0 - tile * a.chunks;   // chunk of item k within its tile
   bool timed_out = false;
+  TilePend pend[2];                // a CTA shares at most two tiles: its first and its last
+  int np = 0;
   for (int k = 0; k < n; ++k, ++ci) {
     const uint32_t K = K0 + k;
     const int sx = K % C::kSX;
     if (ci == a.chunks) {   // item k starts the next tile: finish this one
       if (!bar_and(us.barall, us.nall, !timed_out)) return false;
-      gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane, us);
+      gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, pend[np], quarter, lane, us);
+      if (pend[np].tile >= 0) ++np;
 #pragma unroll
       for (int t = 0; t < NTL; ++t) acc[t] = 0.f;
       ++tile;
@@ -825,7 +865,9 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
     if (!timed_out && lane == 0) mbar_arrive(smem_u32(&S.xempty[sx]));
   }
   if (!bar_and(us.barall, us.nall, !timed_out)) return false;
-  gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, S.flag, quarter, lane, us);
+  gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, pend[np], quarter, lane, us);
+  if (pend[np].tile >= 0) ++np;
+  for (int j = 0; j < np; ++j) tile_resolve<EPI, NT, T0, NTL>(a, sk, pend[j], S.rstd, S.ex, quarter, lane, us);
   return true;
 }
 // One set of four update warps owning every token.
