@@ -313,7 +313,7 @@ struct UpdSlice {
 // token T0 + t.
 template <int EPI, int T0, int NTL>
 QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, const float (&v)[NTL], const float* rstd, float* ex,
-                           int quarter, int lane, const UpdSlice& us) {
+                           int quarter, int lane, const UpdSlice& us, const float (&yres)[NTL]) {
   const int r = quarter * 32 + lane;
   if constexpr (EPI == EPI_STORE) {
     const int gr = tile * kTileRows + r;
@@ -349,7 +349,7 @@ QHL_DEV void gemv_epilogue(const GemvArgs& a, int tile, const float (&v)[NTL], c
       const int tg = T0 + t;
       float hn = 0.f;
       if (valid) {
-        hn = __fadd_rn(__ldcg(a.y + (size_t)tg * a.y_stride + gr), v[t]);
+        hn = __fadd_rn(yres[t], v[t]);
         a.y[(size_t)tg * a.y_stride + gr] = hn;
       }
       if (a.qout) qact_store_block(__fmul_rn(hn, gam), a.qout + (size_t)tg * a.qout_stride, tile * 4 + quarter, lane);
@@ -375,11 +375,28 @@ QHL_DEV bool bar_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
+// The residual stream of tile `tile`'s rows for tokens [T0, T0 + NTL), read
+// when the CTA starts on the tile so that the epilogue does not wait for it
+// (residual epilogue only; the rows are written only by the tile's epilogue).
+template <int EPI, int T0, int NTL>
+QHL_DEV void load_residual(const GemvArgs& a, int tile, int r, float (&yres)[NTL]) {
+#pragma unroll
+  for (int t = 0; t < NTL; ++t) yres[t] = 0.f;
+  if constexpr (EPI == EPI_RESID) {
+    const int gr = tile * kTileRows + r;
+    if (gr < a.out_valid)
+#pragma unroll
+      for (int t = 0; t < NTL; ++t) yres[t] = __ldcg(a.y + (size_t)(T0 + t) * a.y_stride + gr);
+  }
+}
+
 // A shared tile whose partial this CTA has published: its counter's old value
 // (held by the thread that added to it) and the count that makes this CTA the
 // tile's last contributor.
+template <int NTL>
 struct TilePend {
   int tile = -1, old = 0, need = 0;
+  float yres[NTL];   // the tile's residual rows, read at its start
 };
 
 // Update warps, stream-K: finish tile `tl` given this CTA's partial v for
@@ -391,14 +408,16 @@ struct TilePend {
 // update warp of the CTA takes part.
 template <int EPI, int NT, int T0, int NTL>
 QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int i0, int i1, int tl, float (&v)[NTL],
-                              const float* rstd, float* ex, TilePend& pend, int quarter, int lane,
-                              const UpdSlice& us) {
+                              const float (&yres)[NTL], const float* rstd, float* ex, TilePend<NTL>& pend,
+                              int quarter, int lane, const UpdSlice& us) {
   const int r = quarter * 32 + lane;
   const int t_lo = tl * a.chunks, t_hi = t_lo + a.chunks;
   if (t_lo >= i0 && t_hi <= i1) {
-    gemv_epilogue<EPI, T0, NTL>(a, tl, v, rstd, ex, quarter, lane, us);
+    gemv_epilogue<EPI, T0, NTL>(a, tl, v, rstd, ex, quarter, lane, us, yres);
     return;
   }
+#pragma unroll
+  for (int t = 0; t < NTL; ++t) pend.yres[t] = yres[t];
   const int first_tile = i0 / a.chunks;
   float* mine = a.partials + (size_t)(2 * cta + (tl == first_tile ? 0 : 1)) * NT * kTileRows;
 #pragma unroll
@@ -417,7 +436,7 @@ QHL_DEV void gemv_finish_tile(const GemvArgs& a, int cta, const StreamK& sk, int
 // every contributor after cf, and of cf exactly when cf's range starts at the
 // tile's first item) and run the epilogue.
 template <int EPI, int NT, int T0, int NTL>
-QHL_DEV void tile_resolve(const GemvArgs& a, const StreamK& sk, TilePend& pend, const float* rstd, float* ex,
+QHL_DEV void tile_resolve(const GemvArgs& a, const StreamK& sk, TilePend<NTL>& pend, const float* rstd, float* ex,
                           int quarter, int lane, const UpdSlice& us) {
   const int r = quarter * 32 + lane;
   const int tl = pend.tile;
@@ -448,7 +467,7 @@ QHL_DEV void tile_resolve(const GemvArgs& a, const StreamK& sk, TilePend& pend, 
         for (int t = 0; t < NTL; ++t) acc[t] = (c0 + k == cf) ? pv[k][t] : __fadd_rn(acc[t], pv[k][t]);
       }
   }
-  gemv_epilogue<EPI, T0, NTL>(a, tl, acc, rstd, ex, quarter, lane, us);
+  gemv_epilogue<EPI, T0, NTL>(a, tl, acc, rstd, ex, quarter, lane, us, pend.yres);
   if (T0 == 0 && r == 0) a.counters[tl] = 0;
 }
 
@@ -561,9 +580,10 @@ QHL_DEV void issue_x(const GemvArgs& a, const GemvSmem<C>& S, int chunk, uint32_
 
 // Producers of one stand-alone projection (K0 = 0), two threads in two warps
 // so that neither ring waits for the other's slots.  The weight thread keeps
-// the weight ring full: it requests the first SW items at once (the weights
-// never depend on earlier kernels) and then each item as soon as its slot is
-// released, sleeping in the barrier wait in between.  The x thread does the
+// the weight ring full: it requests the first two items, the rest of the
+// first ring once item 0 has landed (the weights never depend on earlier
+// kernels), and then each item as soon as its slot is released, sleeping in
+// the barrier wait in between.  The x thread does the
 // same for the x ring (an item's block scales and x columns); the x columns
 // are written by the previous kernel, so they are requested only once
 // griddepcontrol.wait has returned.  Each returns false on a timeout.
@@ -574,6 +594,11 @@ QHL_DEV bool produce_weights(const GemvArgs& a, const GemvSmem<C>& S, int cta, i
   const uint64_t pol = policy_evict_first();
   for (int k = 0; k < n; ++k) {
     if (k >= SW && !mbar_wait(smem_u32(&S.wempty[k % SW]), ((k / SW) - 1) & 1u, a.err, a.wait_limit)) return false;
+    // the rest of the first ring only once the first item is in: the copies
+    // in flight share the SM's bandwidth, and the pipeline starts on item 0
+    if (k == 2 && n > 2 && !(cta == 0 && a.fault_item == 0) &&
+        !mbar_wait(smem_u32(&S.wfull[0]), 0u, a.err, a.wait_limit))
+      return false;
     if (cta == 0 && k == a.fault_item) continue;   // injected failure: this slot never fills
     issue_weights<C>(a, S, i0 + k, (uint32_t)k, pol);
   }
@@ -790,19 +815,23 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
   int tile = i0 / a.chunks;
   int ci = i0 - tile * a.chunks;   // chunk of item k within its tile
   bool timed_out = false;
-  TilePend pend[2];                // a CTA shares at most two tiles: its first and its last
+  TilePend<NTL> pend[2];           // a CTA shares at most two tiles: its first and its last
   int np = 0;
+  float yres[NTL];
+  load_residual<EPI, T0, NTL>(a, tile, r, yres);
   for (int k = 0; k < n; ++k, ++ci) {
     const uint32_t K = K0 + k;
     const int sx = K % C::kSX;
     if (ci == a.chunks) {   // item k starts the next tile: finish this one
       if (!bar_and(us.barall, us.nall, !timed_out)) return false;
-      gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, pend[np], quarter, lane, us);
+      gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, yres, S.rstd, S.ex, pend[np], quarter, lane,
+                                         us);
       if (pend[np].tile >= 0) ++np;
 #pragma unroll
       for (int t = 0; t < NTL; ++t) acc[t] = 0.f;
       ++tile;
       ci = 0;
+      load_residual<EPI, T0, NTL>(a, tile, r, yres);
     }
     const uint8_t* xsl = S.xring + sx * C::kXS;
     uint4 sc4 = make_uint4(0, 0, 0, 0);
@@ -865,7 +894,7 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
     if (!timed_out && lane == 0) mbar_arrive(smem_u32(&S.xempty[sx]));
   }
   if (!bar_and(us.barall, us.nall, !timed_out)) return false;
-  gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, S.rstd, S.ex, pend[np], quarter, lane, us);
+  gemv_finish_tile<EPI, NT, T0, NTL>(a, cta, sk, i0, i1, tile, acc, yres, S.rstd, S.ex, pend[np], quarter, lane, us);
   if (pend[np].tile >= 0) ++np;
   for (int j = 0; j < np; ++j) tile_resolve<EPI, NT, T0, NTL>(a, sk, pend[j], S.rstd, S.ex, quarter, lane, us);
   return true;
