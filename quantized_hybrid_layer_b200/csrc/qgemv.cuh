@@ -285,6 +285,23 @@ QHL_DEV float block_update(float acc, float d, float s, int H, int M, int L, int
   return __fmaf_rn(__fmul_rn(d, s), v, acc);
 }
 
+// The same update for two tokens at once on packed f32 pairs: each lane is
+// rounded exactly as block_update rounds it, so the results are the same bits.
+template <int QT>
+QHL_DEV float2 block_update2(float2 acc, float d, float2 s, int H0, int M0, int L0, int H1, int M1, int L1, int2 Sh,
+                             int2 Sml) {
+  int Hx0 = H0, MLx0 = M0 * 256 + L0, Hx1 = H1, MLx1 = M1 * 256 + L1;
+  if constexpr (QT == kQ4_0) {   // weights are nibble - 8
+    Hx0 -= 8 * Sh.x;
+    MLx0 -= 8 * Sml.x;
+    Hx1 -= 8 * Sh.y;
+    MLx1 -= 8 * Sml.y;
+  }
+  const float2 v = __ffma2_rn(make_float2(__int2float_rn(Hx0), __int2float_rn(Hx1)), make_float2(65536.f, 65536.f),
+                              make_float2(__int2float_rn(MLx0), __int2float_rn(MLx1)));
+  return __ffma2_rn(__fmul2_rn(make_float2(d, d), s), v, acc);
+}
+
 // Sum of squares of a 128-row tile held one row per thread by four warps
 // (quarter q = rows 32q .. 32q + 31): xor-butterfly per warp, then the four
 // warps in order.  The one definition used for the per-tile RMSNorm partials
@@ -880,7 +897,20 @@ QHL_DEV bool update_items(const GemvArgs& a, const GemvSmem<C>& S, uint32_t tmem
         const uint32_t w = scw[b >> 1];
         const float d = __half2float(__ushort_as_half(static_cast<unsigned short>((b & 1) ? (w >> 16) : (w & 0xFFFFu))));
 #pragma unroll
-        for (int t = 0; t < NTL; ++t) {
+        for (int t = 0; t + 1 < NTL; t += 2) {   // token pairs on packed f32 lanes
+          const int4 m0 = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + (T0 + t) * kQChunkBytes +
+                                                         b * kQBlockBytes + kQMetaOff);
+          const int4 m1 = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + (T0 + t + 1) * kQChunkBytes +
+                                                         b * kQBlockBytes + kQMetaOff);
+          const float2 r2 = block_update2<QT>(make_float2(acc[t], acc[t + 1]), d,
+                                              make_float2(__int_as_float(m0.x), __int_as_float(m1.x)), dv[j][t][0],
+                                              dv[j][t][1], dv[j][t][2], dv[j][t + 1][0], dv[j][t + 1][1],
+                                              dv[j][t + 1][2], make_int2(m0.y, m1.y), make_int2(m0.z, m1.z));
+          acc[t] = r2.x;
+          acc[t + 1] = r2.y;
+        }
+        if constexpr (NTL % 2 == 1) {
+          constexpr int t = NTL - 1;
           const int4 m = *reinterpret_cast<const int4*>(xsl + QLayout<QT>::kScaleBytes + (T0 + t) * kQChunkBytes +
                                                         b * kQBlockBytes + kQMetaOff);
           acc[t] = block_update<QT>(acc[t], d, __int_as_float(m.x), dv[j][t][0], dv[j][t][1], dv[j][t][2], m.y, m.z);
