@@ -172,8 +172,14 @@ constexpr int gemv_sx(int qt, int nt) {
 }
 // Tensor-memory buffers: four A and four D buffers up to eight tokens; beyond,
 // where one D group is 128 columns, two A and three D buffers.
+// Weight ring: four items for one token, twelve beyond.  When every CTA of a
+// launch starts at once, a shallow ring lands each CTA's first item sooner
+// (fewer requests queue ahead of it); four items on 148 SMs still hold about
+// 10 MB in flight, enough to keep HBM busy.  With more tokens the ring depth
+// makes no measurable difference.
 template <int QT, int NT>
-struct GemvCfg : GemvGeom<QT, NT, 225 * 1024, gemv_sx(QT, NT), NT <= 8 ? 4 : 2, NT <= 8 ? 4 : 3, 12, 0> {
+struct GemvCfg : GemvGeom<QT, NT, 225 * 1024, gemv_sx(QT, NT), NT <= 8 ? 4 : 2, NT <= 8 ? 4 : 3,
+                          NT == 1 ? 4 : 12, 0> {
   static constexpr int kMinBlocks = 1;
   // Sixteen warps, 128 registers a thread (four warps per SM sub-partition).
   // Up to eight tokens: eight unpack warps (half an item each) and four update
