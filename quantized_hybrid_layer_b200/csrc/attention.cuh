@@ -5,15 +5,25 @@
 //
 // Token t of a pass sits at absolute position pos + t and attends to cache rows
 // 0 .. pos + t.  The context is cut into fixed chunks of 64 rows at absolute
-// multiples of 64; one CTA handles one (chunk, KV head) for every token and
-// every query head of the group, so each K/V row is read from HBM once per pass.
-// A token's partial (max, sum, weighted V) over a chunk depends only on the
-// token and the chunk, and the combine walks chunks 0 .. in order, so a batched
-// pass gives the same bits as running the tokens one at a time.
+// multiples of 64; one CTA handles one (chunk, KV head) for a group of up to
+// four tokens and every query head of the KV head, so each K/V row is read
+// from HBM once per token group.  A token's partial (max, sum, weighted V) over
+// a chunk depends only on the token and the chunk, and the combine walks chunks
+// 0 .. in order, so a batched pass gives the same bits as running the tokens
+// one at a time.
 //
-// New rows: the CTA whose chunk holds position p = pos + t normalises and
-// rotates the token's k, rounds k and v to f16, writes them to the cache and
-// uses the rounded values, exactly what a later pass reads back.
+// New rows: every CTA whose chunk holds a position p = pos + t that its tokens
+// see normalises and rotates the token's k and rounds k and v to f16 itself
+// (the same operations in every CTA, so the same bits), and uses the rounded
+// values -- exactly what a later pass reads back.  Only the CTA of the token's
+// own group writes the row to the cache, and no CTA reads a row of this pass
+// from the cache, so the CTAs of one launch never depend on one another.
+//
+// The two contractions of a chunk, scores = q.k and out = p.v, run on the
+// warp-level tensor-core MMA (m16n8k16, f16 operands, f32 accumulation).  K and
+// V are f16 already; q and p are f32, and each is split into an f16 high part
+// and an f16 remainder, two MMAs per step, which keeps about 22 bits of each
+// (the products themselves are exact in f32).
 #pragma once
 
 #include "qact.cuh"
@@ -49,11 +59,16 @@ struct AttnArgs {
   int qout_stride;
 };
 
-// Shared memory of one attention unit: normalised, rotated queries
-// [jobs][256], scores / probabilities [jobs][64], a per-warp vector [8][256];
-// jobs = NT * (query heads per KV head).
+// Shared memory of one attention unit with jobs = tokens x query heads of the
+// KV head, in MT = ceil(jobs / 16) row tiles of 16 jobs:
+//   [0, MT * 16 KB): first the new K and V rows (16 x 512 B each), then the
+//     queries' f16 high and low parts ([MT*16][256] each), then the score
+//     partials of the two dimension halves ([2][MT*16][64] f32) followed by the
+//     probabilities' high and low parts ([2][MT*16][72] f16);
+//   [MT * 16 KB, + 8 KB): one 256-float vector per warp.
+__host__ __device__ constexpr int attn_mtiles(int nt, int rep) { return (nt * rep + 15) / 16; }
 __host__ __device__ constexpr int attn_smem_bytes(int nt, int rep) {
-  return nt * rep * kAttDim * 4 + nt * rep * kAttChunk * 4 + 8 * kAttDim * 4;
+  return attn_mtiles(nt, rep) * 16384 + 8 * kAttDim * 4;
 }
 template <int NT>
 constexpr int attn_smem_bytes(int rep) {
@@ -91,41 +106,107 @@ QHL_DEV void load8_cg(const float* p, float (&x)[8]) {
   x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 
-QHL_DEV void half8(uint4 w, float (&f)[8]) {
-  const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w4[i] & 0xFFFFu)));
-    f[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w4[i] >> 16)));
-  }
+// One m16n8k16 MMA, f16 operands, f32 accumulators: d += A(16x16) * B(16x8).
+// Fragments (g = lane / 4, t = lane % 4): a0 = A[g][2t..2t+1],
+// a1 = A[g+8][2t..], a2 = A[g][2t+8..], a3 = A[g+8][2t+8..];
+// b0 = B[2t..2t+1][g], b1 = B[2t+8..2t+9][g]; d = {D[g][2t], D[g][2t+1],
+// D[g+8][2t], D[g+8][2t+1]}.
+QHL_DEV void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                           uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// f32 pair -> f16 high parts and f16 remainders, each packed low | high << 16.
+QHL_DEV void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+  const __half l0 = __float2half_rn(__fsub_rn(x0, __half2float(h0)));
+  const __half l1 = __float2half_rn(__fsub_rn(x1, __half2float(h1)));
+  hi = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+  lo = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+}
+
+// The K and V fragments of one attention unit, held in registers.  Warp w
+// takes keys 16 (w % 4) .. +15 and dimensions 128 (w / 4) .. +127 for the
+// scores: k[i] (k[4 + i]) = the 8 dimensions 32 (4 (w / 4) + i) + 8t .. +7 of
+// key 16 (w % 4) + g (+ 8).  For the weighted sum it takes dimensions
+// 32w .. 32w + 31: v[(2 qq + ...)] = the dimension pair 16 (2w + qq) + 2g of keys
+// 16j + 2t + {0, 1, 8, 9}, at index (qq * 4 + j) * 4 + e.
+struct AttnRegs {
+  uint4 k[8];
+  uint32_t v[32];
+};
+
+// Fill the fragments from cache rows of earlier passes (rows < pos) and zero
+// the rows past the last key the unit's tokens see; rows pos .. come from
+// attn_compute.  Needs nothing written by this pass, so a kernel issues it
+// before waiting for the in-projection.
+QHL_DEV void attn_load_old(const AttnArgs& a, int c, int g, int pos, int ctx_end, AttnRegs& R) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gl = lane >> 2, tl = lane & 3;
+  const int k0 = c * kAttChunk;
+  const int n_old = min(kAttChunk, pos - k0);   // rows of earlier passes in the chunk (may be <= 0)
+  const size_t head_base = (size_t)g * a.max_ctx;
+  const int kq = warp & 3, dh = warp >> 2;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int key = 16 * kq + gl + 8 * r;
+    const uint4* row = reinterpret_cast<const uint4*>(a.K + (head_base + k0 + key) * kAttDim);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      R.k[4 * r + i] = key < n_old ? ld_cg_once(row + 4 * (4 * dh + i) + tl) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = 16 * j + 2 * tl + (e & 1) + 8 * (e >> 1);
+        R.v[(qq * 4 + j) * 4 + e] =
+            key < n_old ? ld_cg_once(reinterpret_cast<const uint32_t*>(a.V + (head_base + k0 + key) * kAttDim) +
+                                     8 * (2 * warp + qq) + gl)
+                        : 0u;
+      }
+  (void)ctx_end;
+}
+
+// Byte offset of the 8-byte unit u of query row r in a [rows][256] f16 plane:
+// units are XOR-swizzled with (r & 1) | (r & 2) << 2 so that the 16 lanes of a
+// half-warp reading B fragments hit 16 distinct bank pairs.
+QHL_DEV int q_unit_off(int r, int u) { return r * 512 + ((u ^ ((r & 1) | ((r & 2) << 2))) << 3); }
+
 // One attention unit: KV head g, context chunk c (rows 64c .. 64c+63), tokens
-// t0 .. t0 + min(kAttGroup, NT - t0) - 1 and the group's query heads.  Writes
-// per (token, head, chunk) the max score, the sum of exp and the exp-weighted
-// V sum.  The unit's tokens' own rows in the chunk are written first; then the
-// chunk's K and V rows are loaded into registers through L2.  All 256 threads
-// of the CTA take part; `pos` is the position of token 0.  A token's results
-// depend only on the token and the chunk, whatever its group.
+// t0 .. t0 + min(kAttGroup, NT - t0) - 1 and the group's query heads (jobs).
+// Writes per (token, head, chunk) the max score, the sum of exp and the
+// exp-weighted V sum.  All 256 threads of the CTA take part; `pos` is the
+// position of token 0.  A token's results depend only on the token and the
+// chunk, whatever its group and its row in the MMA tiles.  At most 7 query
+// heads per KV head (stage_load refuses more): up to 28 jobs, two row tiles of
+// 16 and four column tiles of 8.
 template <int NT>
-QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t* smem) {
+QHL_DEV void attn_compute(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t* smem, AttnRegs& R) {
   const int rep = a.Hq / a.Hkv;
   const int ntk = min(kAttGroup, NT - t0);
   const int njobs = ntk * rep;
-  float* qs = reinterpret_cast<float*>(smem);                 // [njobs][256]
-  float* sc = qs + njobs * kAttDim;                            // [njobs][64]
-  float* vec_all = sc + njobs * kAttChunk;                     // [8][256]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int MT = (njobs + 15) / 16, rows = 16 * MT;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, tl = lane & 3;
   const int k0 = c * kAttChunk;
   const int ctx_end = pos + t0 + ntk;                          // rows the unit's tokens see
   const int nkeys = min(kAttChunk, ctx_end - k0);             // > 0 by the caller
-  float* vec = vec_all + warp * kAttDim;
+  float* vec = reinterpret_cast<float*>(smem + MT * 16384) + warp * kAttDim;
   const int q_off = 0, k_off = 2 * a.Hq * kAttDim, v_off = k_off + a.Hkv * kAttDim;
   const size_t head_base = (size_t)g * a.max_ctx;
 
-  // this pass's own rows that fall in the chunk: QK-norm + RoPE k, round k and v to f16, store
-  const int p_lo = max(k0, pos + t0), p_hi = min(k0 + kAttChunk, ctx_end);
-  for (int p = p_lo + warp; p < p_hi; p += 8) {
+  // 1. this pass's rows in the chunk that the unit's tokens see: QK-norm +
+  //    RoPE k, round k and v to f16, keep them in shared memory; the rows of
+  //    the unit's own tokens also go to the cache
+  const int pn0 = max(k0, pos), p_hi = min(k0 + kAttChunk, ctx_end);
+  uint8_t* newk = smem;               // [16][256] f16
+  uint8_t* newv = smem + 16 * 512;    // [16][256] f16
+  for (int p = pn0 + warp; p < p_hi; p += 8) {
     const int t = p - pos;
     const float* yt = a.y + (size_t)t * a.y_stride;
     float x[8];
@@ -139,157 +220,211 @@ QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t
       kh[i] = __half_as_ushort(__float2half_rn(vec[8 * lane + i]));
       vh[i] = __half_as_ushort(__float2half_rn(vv[i]));
     }
-    reinterpret_cast<uint4*>(a.K + (head_base + p) * kAttDim)[lane] =
-        make_uint4(kh[0] | (kh[1] << 16), kh[2] | (kh[3] << 16), kh[4] | (kh[5] << 16), kh[6] | (kh[7] << 16));
-    reinterpret_cast<uint4*>(a.V + (head_base + p) * kAttDim)[lane] =
-        make_uint4(vh[0] | (vh[1] << 16), vh[2] | (vh[3] << 16), vh[4] | (vh[5] << 16), vh[6] | (vh[7] << 16));
+    const uint4 kr = make_uint4(kh[0] | (kh[1] << 16), kh[2] | (kh[3] << 16), kh[4] | (kh[5] << 16), kh[6] | (kh[7] << 16));
+    const uint4 vr = make_uint4(vh[0] | (vh[1] << 16), vh[2] | (vh[3] << 16), vh[4] | (vh[5] << 16), vh[6] | (vh[7] << 16));
+    reinterpret_cast<uint4*>(newk + (p - pn0) * 512)[lane] = kr;
+    reinterpret_cast<uint4*>(newv + (p - pn0) * 512)[lane] = vr;
+    if (p >= pos + t0) {
+      reinterpret_cast<uint4*>(a.K + (head_base + p) * kAttDim)[lane] = kr;
+      reinterpret_cast<uint4*>(a.V + (head_base + p) * kAttDim)[lane] = vr;
+    }
     __syncwarp();
   }
-  // queries of every token that sees this chunk
-  for (int job = warp; job < njobs; job += 8) {
-    const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
-    if (pos + t < k0) continue;
-    const float* yt = a.y + (size_t)t * a.y_stride;
-    float x[8];
-    load8_cg(yt + q_off + (g * rep + j) * kAttDim + 8 * lane, x);
-    norm_rope(x, a.gq, a.eps, a.rope + (size_t)(pos + t) * (kRopeDims / 2), vec, lane);
-    reinterpret_cast<float4*>(qs + job * kAttDim)[2 * lane] = reinterpret_cast<const float4*>(vec)[2 * lane];
-    reinterpret_cast<float4*>(qs + job * kAttDim)[2 * lane + 1] = reinterpret_cast<const float4*>(vec)[2 * lane + 1];
-    __syncwarp();
-  }
-  named_sync(kBarMix, 256);   // new cache rows and queries visible to all 256 threads
-
-  // K rows are loaded up front and V rows right after the scores (through L2,
-  // each in one round), so the unit pays the memory latency about twice.  Scores: lane quad (lane >> 2) of warp w owns key
-  // 8w + (lane >> 2); the quad's 4 lanes split its 256 dims into interleaved
-  // 8-dim groups (group 4i + r for lane r), so q is read from shared memory
-  // as conflict-free broadcasts and a score needs two shuffles.  PV: thread
-  // (pair p = tid & 127, half = tid >> 7) owns dims 2p, 2p+1 over keys
-  // 32 half .. 32 half + 31.
-  const int r4 = lane & 3, key = warp * 8 + (lane >> 2);
-  uint4 kw[8];
+  if (p_hi > pn0) {   // uniform over the CTA
+    named_sync(kBarMix, 256);
+    const int kq = warp & 3, dh = warp >> 2;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    kw[i] = key < nkeys ? ld_cg_once(reinterpret_cast<const uint4*>(a.K + (head_base + k0 + key) * kAttDim) + 4 * i + r4)
-                        : make_uint4(0u, 0u, 0u, 0u);
-
-  // scores q.k / 16 (1 / sqrt(256)); per (query, key): each lane's 64 dims in
-  // group order, then the quad butterfly -- the same operations for any NT
-  for (int j0 = 0; j0 < njobs; j0 += 8) {
-    float acc[8];
+    for (int r = 0; r < 2; ++r) {
+      const int p = k0 + 16 * kq + gl + 8 * r;
+      if (p >= pn0 && p < p_hi)
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) acc[jj] = 0.f;
+        for (int i = 0; i < 4; ++i) R.k[4 * r + i] = reinterpret_cast<const uint4*>(newk + (p - pn0) * 512)[4 * (4 * dh + i) + tl];
+    }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float kf[8];
-      half8(kw[i], kf);
+    for (int qq = 0; qq < 2; ++qq)
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        if (j0 + jj < njobs) {
-          const float4* qp = reinterpret_cast<const float4*>(qs + (j0 + jj) * kAttDim + 8 * (4 * i + r4));
-          const float4 qa = qp[0], qb = qp[1];
-          float s = acc[jj];
-          s = __fmaf_rn(qa.x, kf[0], s);
-          s = __fmaf_rn(qa.y, kf[1], s);
-          s = __fmaf_rn(qa.z, kf[2], s);
-          s = __fmaf_rn(qa.w, kf[3], s);
-          s = __fmaf_rn(qb.x, kf[4], s);
-          s = __fmaf_rn(qb.y, kf[5], s);
-          s = __fmaf_rn(qb.z, kf[6], s);
-          s = __fmaf_rn(qb.w, kf[7], s);
-          acc[jj] = s;
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int p = k0 + 16 * j + 2 * tl + (e & 1) + 8 * (e >> 1);
+          if (p >= pn0 && p < p_hi)
+            R.v[(qq * 4 + j) * 4 + e] = reinterpret_cast<const uint32_t*>(newv + (p - pn0) * 512)[8 * (2 * warp + qq) + gl];
         }
-      }
-    }
-#pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
-      float s = acc[jj];
-      s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 1));
-      s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 2));
-      if (j0 + jj < njobs && r4 == 0 && key < nkeys) sc[(j0 + jj) * kAttChunk + key] = __fmul_rn(s, 1.f / 16.f);
-    }
+    named_sync(kBarMix, 256);   // the new rows' space is reused below
   }
-  // V rows, issued before the softmax so their latency overlaps it (volatile
-  // loads: the compiler may neither repeat them later nor move them)
-  const int pair = tid & 127, half = tid >> 7;
-  uint32_t vr[32];
+
+  // 2. queries of every token that sees this chunk, normalised and rotated,
+  //    as f16 high and low planes; rows of other tokens and padding are zero
+  uint8_t* qhi = smem;
+  uint8_t* qlo = smem + rows * 512;
+  for (int job = warp; job < rows; job += 8) {
+    const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
+    uint32_t h[4] = {0u, 0u, 0u, 0u}, l[4] = {0u, 0u, 0u, 0u};
+    if (job < njobs && pos + t >= k0) {
+      const float* yt = a.y + (size_t)t * a.y_stride;
+      float x[8];
+      load8_cg(yt + q_off + (g * rep + j) * kAttDim + 8 * lane, x);
+      norm_rope(x, a.gq, a.eps, a.rope + (size_t)(pos + t) * (kRopeDims / 2), vec, lane);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int kk = half * 32 + i;
-    vr[i] = kk < nkeys ? ld_cg_once(reinterpret_cast<const uint32_t*>(a.V + (head_base + k0 + kk) * kAttDim) + pair) : 0u;
+      for (int i = 0; i < 4; ++i) split2(vec[8 * lane + 2 * i], vec[8 * lane + 2 * i + 1], h[i], l[i]);
+    }
+    // lane's dims 8 lane .. +7 = 8-byte units 2 lane, 2 lane + 1
+    *reinterpret_cast<uint2*>(qhi + q_unit_off(job, 2 * lane)) = make_uint2(h[0], h[1]);
+    *reinterpret_cast<uint2*>(qhi + q_unit_off(job, 2 * lane + 1)) = make_uint2(h[2], h[3]);
+    *reinterpret_cast<uint2*>(qlo + q_unit_off(job, 2 * lane)) = make_uint2(l[0], l[1]);
+    *reinterpret_cast<uint2*>(qlo + q_unit_off(job, 2 * lane + 1)) = make_uint2(l[2], l[3]);
   }
   named_sync(kBarMix, 256);
 
-  // chunk softmax statistics, one warp per query
-  for (int job = warp; job < njobs; job += 8) {
-    const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
-    const int nk = min(kAttChunk, pos + t + 1 - k0);
-    if (nk <= 0) continue;
-    const bool v0 = lane < nk, v1 = lane + 32 < nk;
-    const float s0 = v0 ? sc[job * kAttChunk + lane] : -INFINITY;
-    const float s1 = v1 ? sc[job * kAttChunk + lane + 32] : -INFINITY;
-    const float m = warp_max(fmaxf(s0, s1));
-    const float e0 = v0 ? expf(__fsub_rn(s0, m)) : 0.f;
-    const float e1 = v1 ? expf(__fsub_rn(s1, m)) : 0.f;
-    const float l = warp_sum(__fadd_rn(e0, e1));
-    sc[job * kAttChunk + lane] = e0;
-    sc[job * kAttChunk + lane + 32] = e1;
-    if (lane == 0) {
-      const size_t idx = ((size_t)t * a.Hq + g * rep + j) * a.nchunk + c;
-      a.pm[idx] = m;
-      a.pl[idx] = l;
+  // 3. score partials S^T[key][job] over the warp's 128 dimensions: A = K
+  //    (keys 16 (w % 4) ..), B = q (jobs 8 nn ..); each 16-wide MMA step takes
+  //    dimensions 32 s + 8t + 4h + {0, 1 | 2, 3} (s = 4 (w / 4) + i), the
+  //    order in which a lane holds K; high part, then remainder
+  const int kq = warp & 3, dh = warp >> 2;
+  const int nnt = (njobs + 7) / 8;
+  float sacc[4][4];
+#pragma unroll
+  for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[nn][e] = 0.f;
+#pragma unroll
+  for (int nn = 0; nn < 4; ++nn) {
+    if (nn < nnt) {
+      const int qr = 8 * nn + gl;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int s8 = 4 * dh + i;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a0 = h ? R.k[i].z : R.k[i].x, a2 = h ? R.k[i].w : R.k[i].y;
+          const uint32_t a1 = h ? R.k[4 + i].z : R.k[4 + i].x, a3 = h ? R.k[4 + i].w : R.k[4 + i].y;
+          const int u = 8 * s8 + 2 * tl + h;
+          const uint2 bh = *reinterpret_cast<const uint2*>(qhi + q_unit_off(qr, u));
+          const uint2 bl = *reinterpret_cast<const uint2*>(qlo + q_unit_off(qr, u));
+          mma_f16_16816(sacc[nn], a0, a1, a2, a3, bh.x, bh.y);
+          mma_f16_16816(sacc[nn], a0, a1, a2, a3, bl.x, bl.y);
+        }
+      }
+    }
+  }
+  named_sync(kBarMix, 256);   // every query read: the space takes the partials
+  float* sc = reinterpret_cast<float*>(smem);   // [2][rows][64]
+#pragma unroll
+  for (int nn = 0; nn < 4; ++nn) {
+    if (nn < nnt) {
+      const int key = 16 * kq + gl, job = 8 * nn + 2 * tl;
+      float* d = sc + ((size_t)dh * rows + job) * kAttChunk + key;
+      d[0] = sacc[nn][0];
+      d[kAttChunk] = sacc[nn][1];
+      d[8] = sacc[nn][2];
+      d[kAttChunk + 8] = sacc[nn][3];
     }
   }
   named_sync(kBarMix, 256);
 
-  // exp-weighted V: per (query, dim) the keys of each half in order, then
-  // half 0 + half 1; 4 queries at a time (vec_all holds half 1's sums), so
-  // the V rows stay in registers across the batches
-  constexpr int JB = 4;
-  float* part = vec_all;   // [JB][256]
-  for (int j0 = 0; j0 < njobs; j0 += JB) {
-    float o0[JB], o1[JB];
-    int nk[JB];
-#pragma unroll
-    for (int jj = 0; jj < JB; ++jj) {
-      o0[jj] = 0.f;
-      o1[jj] = 0.f;
-      nk[jj] = j0 + jj < njobs ? min(kAttChunk, pos + t0 + (j0 + jj) / rep + 1 - k0) : 0;
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int kk = half * 32 + i;
-      const float vlo = __half2float(__ushort_as_half(static_cast<unsigned short>(vr[i] & 0xFFFFu)));
-      const float vhi = __half2float(__ushort_as_half(static_cast<unsigned short>(vr[i] >> 16)));
-#pragma unroll
-      for (int jj = 0; jj < JB; ++jj) {
-        if (kk < nk[jj]) {
-          const float pr = sc[(j0 + jj) * kAttChunk + kk];
-          o0[jj] = __fmaf_rn(pr, vlo, o0[jj]);
-          o1[jj] = __fmaf_rn(pr, vhi, o1[jj]);
-        }
+  // 4. chunk softmax statistics, one warp per job: score = (half 0 + half 1) / 16;
+  //    probabilities as f16 high and low planes [rows][72]
+  uint16_t* phi = reinterpret_cast<uint16_t*>(smem + (size_t)2 * rows * kAttChunk * 4);
+  uint16_t* plo = phi + rows * 72;
+  for (int job = warp; job < rows; job += 8) {
+    const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
+    const int nk = job < njobs ? min(kAttChunk, pos + t + 1 - k0) : 0;
+    float e0 = 0.f, e1 = 0.f;
+    if (nk > 0) {
+      const bool v0 = lane < nk, v1 = lane + 32 < nk;
+      const float* s0p = sc + (size_t)job * kAttChunk;
+      const float* s1p = sc + ((size_t)rows + job) * kAttChunk;
+      const float s0 = v0 ? __fmul_rn(__fadd_rn(s0p[lane], s1p[lane]), 1.f / 16.f) : -INFINITY;
+      const float s1 = v1 ? __fmul_rn(__fadd_rn(s0p[lane + 32], s1p[lane + 32]), 1.f / 16.f) : -INFINITY;
+      const float m = warp_max(fmaxf(s0, s1));
+      e0 = v0 ? expf(__fsub_rn(s0, m)) : 0.f;
+      e1 = v1 ? expf(__fsub_rn(s1, m)) : 0.f;
+      const float l = warp_sum(__fadd_rn(e0, e1));
+      if (lane == 0) {
+        const size_t idx = ((size_t)t * a.Hq + g * rep + j) * a.nchunk + c;
+        a.pm[idx] = m;
+        a.pl[idx] = l;
       }
     }
-    if (half == 1) {
-#pragma unroll
-      for (int jj = 0; jj < JB; ++jj)
-        reinterpret_cast<float2*>(part + jj * kAttDim)[pair] = make_float2(o0[jj], o1[jj]);
-    }
-    named_sync(kBarMix, 256);
-    if (half == 0) {
-#pragma unroll
-      for (int jj = 0; jj < JB; ++jj) {
-        const int job = j0 + jj;
-        if (job < njobs && nk[jj] > 0) {
-          const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
-          const float2 h1 = reinterpret_cast<const float2*>(part + jj * kAttDim)[pair];
-          float2* dst = reinterpret_cast<float2*>(a.po + (((size_t)t * a.Hq + g * rep + j) * a.nchunk + c) * kAttDim);
-          dst[pair] = make_float2(__fadd_rn(o0[jj], h1.x), __fadd_rn(o1[jj], h1.y));
-        }
-      }
-    }
-    named_sync(kBarMix, 256);
+    const __half h0 = __float2half_rn(e0), h1 = __float2half_rn(e1);
+    phi[job * 72 + lane] = __half_as_ushort(h0);
+    phi[job * 72 + lane + 32] = __half_as_ushort(h1);
+    plo[job * 72 + lane] = __half_as_ushort(__float2half_rn(__fsub_rn(e0, __half2float(h0))));
+    plo[job * 72 + lane + 32] = __half_as_ushort(__float2half_rn(__fsub_rn(e1, __half2float(h1))));
   }
+  named_sync(kBarMix, 256);
+
+  // 5. exp-weighted V: O[job][dim] over the chunk's 64 keys, A = p (jobs
+  //    16 m ..), B = V (warp w: dims 32w .. +31 as an even-dimension and an
+  //    odd-dimension tile per 16 dims); high part, then remainder
+  float oacc[2][2][2][4];   // [m][qq][even / odd][4]
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq)
+#pragma unroll
+      for (int o = 0; o < 2; ++o)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[m][qq][o][e] = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      if (m < MT) {
+        const uint16_t* rh0 = phi + (16 * m + gl) * 72 + 16 * j + 2 * tl;
+        const uint16_t* rl0 = plo + (16 * m + gl) * 72 + 16 * j + 2 * tl;
+        const uint32_t ah0 = *reinterpret_cast<const uint32_t*>(rh0);
+        const uint32_t ah1 = *reinterpret_cast<const uint32_t*>(rh0 + 8 * 72);
+        const uint32_t ah2 = *reinterpret_cast<const uint32_t*>(rh0 + 8);
+        const uint32_t ah3 = *reinterpret_cast<const uint32_t*>(rh0 + 8 * 72 + 8);
+        const uint32_t al0 = *reinterpret_cast<const uint32_t*>(rl0);
+        const uint32_t al1 = *reinterpret_cast<const uint32_t*>(rl0 + 8 * 72);
+        const uint32_t al2 = *reinterpret_cast<const uint32_t*>(rl0 + 8);
+        const uint32_t al3 = *reinterpret_cast<const uint32_t*>(rl0 + 8 * 72 + 8);
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const uint32_t* x = R.v + (qq * 4 + j) * 4;
+          const uint32_t be0 = __byte_perm(x[0], x[1], 0x5410), be1 = __byte_perm(x[2], x[3], 0x5410);
+          const uint32_t bo0 = __byte_perm(x[0], x[1], 0x7632), bo1 = __byte_perm(x[2], x[3], 0x7632);
+          mma_f16_16816(oacc[m][qq][0], ah0, ah1, ah2, ah3, be0, be1);
+          mma_f16_16816(oacc[m][qq][0], al0, al1, al2, al3, be0, be1);
+          mma_f16_16816(oacc[m][qq][1], ah0, ah1, ah2, ah3, bo0, bo1);
+          mma_f16_16816(oacc[m][qq][1], al0, al1, al2, al3, bo0, bo1);
+        }
+      }
+    }
+  }
+  // lane holds, per tile and 16 dims, dims 16 (2w + qq) + 4t .. +3 of jobs
+  // 16m + g and 16m + g + 8
+#pragma unroll
+  for (int m = 0; m < 2; ++m) {
+    if (m < MT) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int job = 16 * m + gl + 8 * half;
+        const int tj = job / rep, j = job - tj * rep, t = t0 + tj;
+        if (job < njobs && pos + t + 1 - k0 > 0) {
+          float* dst = a.po + (((size_t)t * a.Hq + g * rep + j) * a.nchunk + c) * kAttDim;
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const float* ev = oacc[m][qq][0];
+            const float* od = oacc[m][qq][1];
+            reinterpret_cast<float4*>(dst + 16 * (2 * warp + qq) + 4 * tl)[0] =
+                make_float4(ev[2 * half], od[2 * half], ev[2 * half + 1], od[2 * half + 1]);
+          }
+        }
+      }
+    }
+  }
+  named_sync(kBarMix, 256);   // shared memory reusable by the caller
+  (void)nkeys;
+}
+
+template <int NT>
+QHL_DEV void attn_unit(const AttnArgs& a, int c, int g, int pos, int t0, uint8_t* smem) {
+  AttnRegs R;
+  attn_load_old(a, c, g, pos, pos + t0 + min(kAttGroup, NT - t0), R);
+  attn_compute<NT>(a, c, g, pos, t0, smem, R);
 }
 
 template <int NT>
@@ -299,8 +434,10 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
   const int pos = *a.kv_len;
   const int t0 = blockIdx.z * kAttGroup, ntk = min(kAttGroup, NT - t0);
   if ((int)blockIdx.x * kAttChunk >= pos + t0 + ntk) return;   // no token of the group sees the chunk
+  AttnRegs R;
+  attn_load_old(a, blockIdx.x, blockIdx.y, pos, pos + t0 + ntk, R);   // overlaps the in-projection's end
   pdl_wait();
-  attn_unit<NT>(a, blockIdx.x, blockIdx.y, pos, t0, smem);
+  attn_compute<NT>(a, blockIdx.x, blockIdx.y, pos, t0, smem, R);
 }
 
 // Combine the chunk partials of one (token, query head) and apply the sigmoid
