@@ -33,6 +33,7 @@ namespace qhl {
 constexpr int kAttDim = 256;
 constexpr int kRopeDims = 64;
 constexpr int kAttChunk = 64;
+constexpr int kAttMaxCtx = 1 << 18;   // largest cache a stage accepts (rows per KV head)
 // Tokens one attention unit serves: a 16-token pass splits its tokens into
 // groups of 4, so its (chunk, KV head, group) units spread over 4x the CTAs.
 constexpr int kAttGroup = 4;
@@ -441,21 +442,39 @@ __global__ void __launch_bounds__(256) attn_partial_kernel(const AttnArgs a) {
 }
 
 // Combine the chunk partials of one (token, query head) and apply the sigmoid
-// output gate.  Thread = dim.  The chunk statistics are staged in shared
-// memory (cs: 3 * nchunk floats); the global max is exact in any order; the
-// normaliser is summed with a fixed structure (lane l takes chunks l, l + 32,
-// .. in order, then a butterfly) and the weighted V sums chunk by chunk in
-// order, with the loads issued in batches ahead of the accumulation.  The
-// result depends only on the token's position, never on NT.
+// output gate, for 64 of the head's dimensions (quarter qd: 64 qd .. +63), so
+// a (token, head) takes four CTAs.  Thread (cq = tid / 64, d = tid % 64) sums
+// dimension 64 qd + d over chunks cq, cq + 4, cq + 8, .. in order; the four
+// sums are added as (0 + 1) + (2 + 3).  Its first 32 chunks' partials are
+// requested together with the chunk statistics (staged in shared memory: cs
+// holds [nchunk] max, [nchunk] weight, [nchunk] sum, then [4][64] partial
+// sums), so a context up to 8192 rows costs one memory round trip.  The global
+// max is exact in any order; the normaliser is summed with a fixed structure
+// (lane l takes chunks l, l + 32, .. in order, then a butterfly).  The result
+// depends only on the token's position, never on NT.
+constexpr int kCombineParts = 4;
+__host__ __device__ constexpr int combine_smem_bytes(int nchunk) { return (3 * nchunk + kCombineParts * 64) * 4; }
+
 template <int NT>
-QHL_DEV void combine_unit(const AttnArgs& a, int t, int head, int pos, float* cs) {
-  const int dim = threadIdx.x, lane = dim & 31;
+QHL_DEV void combine_unit(const AttnArgs& a, int t, int head, int qd, int pos, float* cs) {
+  const int tid = threadIdx.x, lane = tid & 31, cq = tid >> 6, d = tid & 63;
+  const int dim = 64 * qd + d;
   const int nc = (pos + t + 1 + kAttChunk - 1) / kAttChunk;
   const size_t base = ((size_t)t * a.Hq + head) * a.nchunk;
   float* cm = cs;
   float* cw = cs + a.nchunk;
   float* cl = cs + 2 * a.nchunk;
-  for (int c = dim; c < nc; c += 256) {
+  float* part = cs + 3 * a.nchunk;
+  constexpr int B = 32;
+  const float* po = a.po + base * kAttDim + dim;
+  float v[B];
+#pragma unroll
+  for (int j = 0; j < B; ++j) {
+    const int c = cq + kCombineParts * j;
+    v[j] = c < nc ? ld_cg_once(po + (size_t)c * kAttDim) : 0.f;
+  }
+  const float gate = cq == 0 ? __ldcg(a.y + (size_t)t * a.y_stride + a.Hq * kAttDim + head * kAttDim + dim) : 0.f;
+  for (int c = tid; c < nc; c += 256) {
     cm[c] = __ldcg(a.pm + base + c);
     cl[c] = __ldcg(a.pl + base + c);
   }
@@ -463,37 +482,49 @@ QHL_DEV void combine_unit(const AttnArgs& a, int t, int head, int pos, float* cs
   float M = -INFINITY;
   for (int c = lane; c < nc; c += 32) M = fmaxf(M, cm[c]);
   M = warp_max(M);
-  for (int c = dim; c < nc; c += 256) cw[c] = expf(__fsub_rn(cm[c], M));
+  for (int c = tid; c < nc; c += 256) cw[c] = expf(__fsub_rn(cm[c], M));
   named_sync(kBarMix, 256);
   float L = 0.f;
   for (int c = lane; c < nc; c += 32) L = __fmaf_rn(cl[c], cw[c], L);
   L = warp_sum(L);
   float O = 0.f;
-  constexpr int B = 32;
-  const float* po = a.po + base * kAttDim + dim;
-  for (int c0 = 0; c0 < nc; c0 += B) {
-    float v[B];
 #pragma unroll
-    for (int j = 0; j < B; ++j) v[j] = c0 + j < nc ? ld_cg_once(po + (size_t)(c0 + j) * kAttDim) : 0.f;
-#pragma unroll
-    for (int j = 0; j < B; ++j)
-      if (c0 + j < nc) O = __fmaf_rn(v[j], cw[c0 + j], O);
+  for (int j = 0; j < B; ++j) {
+    const int c = cq + kCombineParts * j;
+    if (c < nc) O = __fmaf_rn(v[j], cw[c], O);
   }
-  const float gate = __ldcg(a.y + (size_t)t * a.y_stride + a.Hq * kAttDim + head * kAttDim + dim);
-  const float r = __fmul_rn(__fdiv_rn(O, L), sigmoidf_(gate));
-  if (a.out) a.out[(size_t)t * a.out_stride + head * kAttDim + dim] = r;
-  if (a.qout)   // warp w holds dims 32w..32w+31: one block
-    qact_store_block(r, a.qout + (size_t)t * a.qout_stride, head * (kAttDim / 32) + (dim >> 5), dim & 31);
+  for (int c0 = kCombineParts * B; c0 < nc; c0 += kCombineParts * B) {
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      const int c = c0 + cq + kCombineParts * j;
+      v[j] = c < nc ? ld_cg_once(po + (size_t)c * kAttDim) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+      const int c = c0 + cq + kCombineParts * j;
+      if (c < nc) O = __fmaf_rn(v[j], cw[c], O);
+    }
+  }
+  part[cq * 64 + d] = O;
+  named_sync(kBarMix, 256);
+  if (cq == 0) {   // warps 0 and 1: dims 64 qd .. +31 and +32 .. +63, one block each
+    const float o = __fadd_rn(__fadd_rn(part[d], part[64 + d]), __fadd_rn(part[128 + d], part[192 + d]));
+    const float r = __fmul_rn(__fdiv_rn(o, L), sigmoidf_(gate));
+    if (a.out) a.out[(size_t)t * a.out_stride + head * kAttDim + dim] = r;
+    if (a.qout)
+      qact_store_block(r, a.qout + (size_t)t * a.qout_stride, head * (kAttDim / 32) + (dim >> 5), dim & 31);
+  }
   named_sync(kBarMix, 256);   // cs reusable by the caller
 }
 
 template <int NT>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnArgs a) {
-  extern __shared__ float cs[];                  // [nchunk] max, [nchunk] weight, [nchunk] sum
+  extern __shared__ float cs[];
   if (threadIdx.x == 0) pdl_launch();
   const int pos = *a.kv_len;
   pdl_wait();
-  combine_unit<NT>(a, blockIdx.x / a.Hq, blockIdx.x % a.Hq, pos, cs);
+  const int u = blockIdx.x;   // (token, head, quarter)
+  combine_unit<NT>(a, u / (kCombineParts * a.Hq), (u / kCombineParts) % a.Hq, u % kCombineParts, pos, cs);
 }
 
 }  // namespace qhl

@@ -79,6 +79,9 @@ cudaError_t mixers_prepare(int rep) {
     e = cudaFuncSetAttribute(attn_partial_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
                              attn_smem_bytes<N>(rep));                                                  \
   if (e == cudaSuccess) e = max_carveout(attn_partial_kernel<N>);                                       \
+  if (e == cudaSuccess)                                                                                 \
+    e = cudaFuncSetAttribute(attn_combine_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
+                             combine_smem_bytes(kAttMaxCtx / kAttChunk));                                \
   if (e == cudaSuccess) e = max_carveout(attn_combine_kernel<N>);                                       \
   if (e == cudaSuccess) e = max_carveout(dn_step_kernel<N>);                                            \
   if (e == cudaSuccess) e = max_carveout(stage_input_kernel<N>);
@@ -112,7 +115,10 @@ cudaError_t launch_attn_partial(int nt, const AttnArgs& a, int nchunk, int hkv, 
 
 cudaError_t launch_attn_combine(int nt, const AttnArgs& a, cudaStream_t s, bool pdl) {
   switch (nt) {
-#define C(N) case N: return launch_ex(attn_combine_kernel<N>, dim3(N * a.Hq), dim3(256), (size_t)3 * a.nchunk * 4, s, pdl, a);
+#define C(N)                                                                                                \
+  case N:                                                                                                   \
+    return launch_ex(attn_combine_kernel<N>, dim3(N * a.Hq * kCombineParts), dim3(256),                     \
+                     (size_t)combine_smem_bytes(a.nchunk), s, pdl, a);
     QHL_NT_CASES(C)
 #undef C
     default: return cudaErrorInvalidValue;

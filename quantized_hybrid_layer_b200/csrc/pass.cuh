@@ -65,7 +65,7 @@ struct PassArgs {
 };
 
 // Mixer scratch of the persistent kernel: attention at up to 4 tokens with up
-// to 6 query heads per KV head, the combine's chunk statistics, the DeltaNet
+// to 7 query heads per KV head, the combine's chunk statistics, the DeltaNet
 // unit, the stage input.
 constexpr int kPassMixBytes = 40 * 1024;
 constexpr int kPassMaxTok = 4;
@@ -341,8 +341,9 @@ __global__ void __maxnreg__(128) stage_pass_kernel(const PassArgs p) {
         }
         group_arrive(p, kBarMix + 1, 256, lead);
         if (!(ok = group_phase_wait(p, ph + 1, kBarMix + 1, 256, lead))) break;
-        for (int u = cta; u < NT * p.Hq; u += p.grid)
-          combine_unit<NT>(L.at, u / p.Hq, u % p.Hq, pos, reinterpret_cast<float*>(mix));
+        for (int u = cta; u < NT * p.Hq * kCombineParts; u += p.grid)
+          combine_unit<NT>(L.at, u / (kCombineParts * p.Hq), (u / kCombineParts) % p.Hq, u % kCombineParts, pos,
+                           reinterpret_cast<float*>(mix));
         group_arrive(p, kBarMix + 1, 256, lead);
       }
       // out-projection, gate/up, down (warps 0..3; 4..7 go on to the next

@@ -332,7 +332,7 @@ bool pass_eligible(stage* st, int n) {
     return false;
   }
   const int rep = st->cfg.att_q_heads / st->cfg.att_kv_heads;
-  const int need = std::max({dn_smem_floats(n) * 4, st->nchunk * 3 * 4,
+  const int need = std::max({dn_smem_floats(n) * 4, combine_smem_bytes(st->nchunk),
                              st->nchunk ? attn_smem_bytes(std::min(n, kAttGroup), rep) : 0});
   if (need > kPassMixBytes) {
     st->last_error = "persistent pass: mixer scratch " + std::to_string(need) + " bytes";
@@ -448,7 +448,7 @@ stage_status stage_load(const stage_config* cfg, const stage_tensor* tensors, in
   if (c.att_dim != kAttDim || c.rope_dims != kRopeDims || c.att_kv_heads <= 0 || c.att_q_heads <= 0 ||
       c.att_q_heads % c.att_kv_heads || c.att_q_heads / c.att_kv_heads > 7)
     return STAGE_E_UNSUPPORTED;
-  if (c.attn_every <= 0 || c.max_ctx < kMaxTok || c.max_ctx > (1 << 18) || !(c.eps > 0.f) || !(c.rope_theta > 0.0))
+  if (c.attn_every <= 0 || c.max_ctx < kMaxTok || c.max_ctx > kAttMaxCtx || !(c.eps > 0.f) || !(c.rope_theta > 0.0))
     return STAGE_E_ARG;
 
   stage* st = new (std::nothrow) stage();
