@@ -56,6 +56,23 @@ struct DnArgs {
 //                 token-by-token steps, within rounding of them).
 enum DnMode : int { DN_SNAPSHOTS = 0, DN_FINAL = 1, DN_CHUNKED = 2 };
 
+// Sum of each of 32 per-lane values over the warp; lane l returns the total of
+// value l.  Five halving steps: at each, a lane keeps the half of its values
+// that its lane bit selects and adds the partner's copy of that half.
+QHL_DEV float warp_transpose_sum(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool up = lane & w;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float keep = up ? v[w + i] : v[i];
+      const float send = up ? v[i] : v[w + i];
+      v[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, w));
+    }
+  }
+  return v[0];
+}
+
 QHL_DEV float dot4(float4 a, float4 b) {
   float s = __fmul_rn(a.x, b.x);
   s = __fmaf_rn(a.y, b.y, s);
@@ -233,16 +250,28 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
     for (int t = 0; t < NT; ++t) ef[t] = expf(__fsub_rn(cl[NT - 1], cl[t]));
   }
   named_sync(kBarMix, 256);
-  for (int p = warp; p < NT * NT; p += 8) {
-    const int t = p / NT, j = p % NT;
-    const float4 kj = reinterpret_cast<const float4*>(sk + j * kDnDim)[lane];
-    const float kk = warp_sum(dot4(kj, reinterpret_cast<const float4*>(sk + t * kDnDim)[lane]));
-    const float qk = warp_sum(dot4(kj, reinterpret_cast<const float4*>(sq + t * kDnDim)[lane]));
-    if (lane == 0) {
-      const float e = j <= t ? expf(__fsub_rn(cl[t], cl[j])) : 0.f;
-      Lm[p] = j < t ? __fmul_rn(e, kk) : 0.f;
-      Pm[p] = __fmul_rn(e, qk);
+  // token pairs, one thread each: k_j . k_t and q_t . k_j over the 128 dims,
+  // float4s taken in order from float4 j (mod 32) so that the 8 lanes of a
+  // shared-memory phase read distinct banks, two partial sums per product over
+  // alternate float4s
+  if (tid < NT * NT) {
+    const int t = tid / NT, j = tid % NT;
+    const float4* kj = reinterpret_cast<const float4*>(sk + j * kDnDim);
+    const float4* kt = reinterpret_cast<const float4*>(sk + t * kDnDim);
+    const float4* qt = reinterpret_cast<const float4*>(sq + t * kDnDim);
+    float kk0 = 0.f, kk1 = 0.f, qk0 = 0.f, qk1 = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < kDnDim / 4; i += 2) {
+      const int d0 = (i + j) & 31, d1 = (i + 1 + j) & 31;
+      const float4 a0 = kj[d0], a1 = kj[d1];
+      kk0 = __fmaf_rn(a0.w, kt[d0].w, __fmaf_rn(a0.z, kt[d0].z, __fmaf_rn(a0.y, kt[d0].y, __fmaf_rn(a0.x, kt[d0].x, kk0))));
+      kk1 = __fmaf_rn(a1.w, kt[d1].w, __fmaf_rn(a1.z, kt[d1].z, __fmaf_rn(a1.y, kt[d1].y, __fmaf_rn(a1.x, kt[d1].x, kk1))));
+      qk0 = __fmaf_rn(a0.w, qt[d0].w, __fmaf_rn(a0.z, qt[d0].z, __fmaf_rn(a0.y, qt[d0].y, __fmaf_rn(a0.x, qt[d0].x, qk0))));
+      qk1 = __fmaf_rn(a1.w, qt[d1].w, __fmaf_rn(a1.z, qt[d1].z, __fmaf_rn(a1.y, qt[d1].y, __fmaf_rn(a1.x, qt[d1].x, qk1))));
     }
+    const float e = j <= t ? expf(__fsub_rn(cl[t], cl[j])) : 0.f;
+    Lm[tid] = j < t ? __fmul_rn(e, __fadd_rn(kk0, kk1)) : 0.f;
+    Pm[tid] = __fmul_rn(e, __fadd_rn(qk0, qk1));
   }
   named_sync(kBarMix, 256);
 
@@ -250,12 +279,19 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
                      : a.ring + (size_t)(NT - 1) * a.state_elems;
 #pragma unroll 1
   for (int r = 0; r < 4; ++r) {
-    float A[NT], B[NT], u[NT];
+    // the row's 2 NT products with the starting state, S_0 k_t (value t) and
+    // S_0 q_t (value 16 + t), reduced over the warp in one transposed
+    // butterfly: lane l ends with value l
+    float x32[32];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      A[t] = warp_sum(dot4(S[r], reinterpret_cast<const float4*>(sk + t * kDnDim)[lane]));
-      B[t] = warp_sum(dot4(S[r], reinterpret_cast<const float4*>(sq + t * kDnDim)[lane]));
+    for (int t = 0; t < 16; ++t) {
+      x32[t] = t < NT ? dot4(S[r], reinterpret_cast<const float4*>(sk + t * kDnDim)[lane]) : 0.f;
+      x32[16 + t] = t < NT ? dot4(S[r], reinterpret_cast<const float4*>(sq + t * kDnDim)[lane]) : 0.f;
     }
+    const float mine = warp_transpose_sum(x32, lane);
+    float A[NT], u[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) A[t] = __shfl_sync(0xffffffffu, mine, t);
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       float x = __fsub_rn(sv[t * 32 + warp * 4 + r], __fmul_rn(eg[t], A[t]));
@@ -263,15 +299,15 @@ QHL_DEV void dn_run_chunked(const DnArgs& a, int unit, float4 (&S)[4], float* sm
       for (int j = 0; j < t; ++j) x = __fsub_rn(x, __fmul_rn(Lm[t * NT + j], u[j]));
       u[t] = __fmul_rn(sb[t], x);
     }
+    // output of token t in lane 16 + t
+    if (lane >= 16 && lane - 16 < NT) {
+      const int t = lane - 16;
+      float o = __fmul_rn(eg[t], mine);
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      float o = __fmul_rn(eg[t], B[t]);
-#pragma unroll
-      for (int j = 0; j <= t; ++j) o = __fmaf_rn(Pm[t * NT + j], u[j], o);
-      if (lane == 0) {
-        ob[t][warp * 4 + r] = o;
-        if (a.o) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
-      }
+      for (int j = 0; j < NT; ++j)
+        if (j <= t) o = __fmaf_rn(Pm[t * NT + j], u[j], o);
+      ob[t][warp * 4 + r] = o;
+      if (a.o) a.o[(size_t)t * a.o_stride + h * kDnDim + row0 + r] = o;
     }
     const float e = eg[NT - 1];
     float4 sn = make_float4(__fmul_rn(e, S[r].x), __fmul_rn(e, S[r].y), __fmul_rn(e, S[r].z), __fmul_rn(e, S[r].w));
