@@ -454,7 +454,7 @@ def run_ours(args, rank, world, local, pg):
         prefill = None
         if not args.no_prefill:
             st.reset()
-            n_chunks = PROMPT // CHUNK
+            n_chunks = min(PROMPT // CHUNK, args.prefill_chunks) if args.prefill_chunks > 0 else PROMPT // CHUNK
             ph = torch.from_numpy(synth.normal_f32(synth.rng_for(SEED, rank, 79), (n_chunks, CHUNK, H))).to(dev)
             st.prefill(ph[0].clone(), 0, chunked=True)      # builds the 16-token prefill graph
             st.reset()
@@ -470,7 +470,7 @@ def run_ours(args, rank, world, local, pg):
             st.sync()
             dtp = max_over_ranks(p0.elapsed_time(p1) / 1e3, pg)
             pbp = pass_bytes(shape, qtype, layers, PROMPT // 2, CHUNK)
-            prefill = {"tok_s": PROMPT / dtp * world, "ms_per_chunk": dtp / n_chunks * 1e3,
+            prefill = {"tok_s": n_chunks * CHUNK / dtp * world, "ms_per_chunk": dtp / n_chunks * 1e3,
                        "weight_gbs": pbp["weights"] * n_chunks / dtp / 1e9, "chunks": n_chunks,
                        "call": "stage_prefill, chunked DeltaNet form"}
 
@@ -565,6 +565,8 @@ def main(argv=None):
     ap.add_argument("--qtype", choices=("q4_0", "q8_0"), default="q4_0")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-chunks", type=int, default=0,
+                    help="time only the first N 16-token chunks of the prompt (0: all; for short profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-roofline", action="store_true")
     ap.add_argument("--pass-mode", choices=("kernels", "persistent"), default="kernels",
