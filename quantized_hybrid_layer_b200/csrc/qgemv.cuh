@@ -638,15 +638,18 @@ QHL_DEV bool produce_weights(const GemvArgs& a, const GemvSmem<C>& S, int cta, i
 // The x producer is a whole warp.  Its lane 0 bulk-copies each item's block
 // scales and x columns into the x ring as slots are released.  Bulk copies of
 // one SM are served in order, so at the start of a projection the first x
-// columns (a few KB from L2) would queue behind the ring of weight copies just
-// requested; up to two tokens the whole warp moves the first kHead items' x
-// columns through the load/store path instead (each lane loads its 16-byte
-// pieces, stores them and fences them for the tensor core's async proxy).
+// columns (a few KB from L2) queue behind the weight copies already requested.
+// At two tokens, behind a twelve-item weight ring, the whole warp moves the
+// first two items' x columns through the load/store path instead (each lane
+// loads its 16-byte pieces, stores them and fences them for the tensor core's
+// async proxy).  At one token the four-item ring holds few copies ahead of
+// them, and the bulk copies alone are faster (0 to 4 head items on the
+// 64-layer decode pass: 234.6, 232.9, 232.1, 231.7, 231.0 tok/s).
 template <class C>
 QHL_DEV bool produce_x(const GemvArgs& a, const GemvSmem<C>& S, int i0, int n, int lane) {
   constexpr int QT = C::kQT, NT = C::kNT, SX = C::kSX;
   constexpr int kPer = kQChunkBytes / 16 / 32;      // 16-byte pieces per lane and token
-  constexpr int kHead = NT <= 2 ? 4 / NT : 0;       // items through the load/store path (16 pieces a lane)
+  constexpr int kHead = NT == 2 ? 2 : 0;            // items through the load/store path (16 pieces a lane)
   static_assert(kHead <= SX, "head items take distinct x slots");
   const uint64_t pol = policy_evict_first();
   if (lane == 0)
