@@ -149,6 +149,11 @@ constexpr int kBarMix = 5;
 QHL_DEV void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Arrive on a named barrier without waiting for it (the other participants
+// use named_sync with the same count).
+QHL_DEV void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 // Named barrier that also ANDs a predicate over the participating threads:
 // every thread gets the same answer.
 QHL_DEV bool bar_and(int id, int nthreads, bool pred) {

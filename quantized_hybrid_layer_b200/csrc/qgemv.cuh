@@ -109,6 +109,7 @@ constexpr int kBarUpdate = 1;
 constexpr int kBarTmem = 2;
 constexpr int kBarUpdate2 = 3;
 constexpr int kBarUpdateAll = 4;
+constexpr int kBarSetup = 7;
 
 // Geometry and shared-memory layout of one GEMV configuration: weight type,
 // token count, shared-memory budget, x-ring depth SX, tensor-memory A and D
@@ -972,17 +973,21 @@ __global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kM
   const int i0 = sk.begin(cta), n = sk.begin(cta + 1) - i0;
   if (n == 0) return;
 
-  if (warp == kProducerWarp) S.init(lane);
-  if (warp == kMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *S.tslot;
-
+  // The weight producer sets up the barriers and starts its ring at once; the
+  // other warps wait for the barriers and the tensor-memory address.
   if (warp == kProducerWarp) {
+    S.init(lane);
+    __syncwarp();
+    named_arrive(kBarSetup, C::kThreads);
     if (lane == 0 && !produce_weights<C>(a, S, cta, i0, n)) drain_inflight_copies();   // error path
     return;   // the producers take no part in the tensor-memory teardown
   }
+  if (warp == kMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
+  tc_fence_before();
+  named_sync(kBarSetup, C::kThreads);
+  tc_fence_after();
+  const uint32_t tmem = *S.tslot;
+
   if (warp == C::kXWarp) {
     if (!produce_x<C>(a, S, i0, n, lane) && lane == 0) drain_inflight_copies();   // error path
     return;
