@@ -110,6 +110,7 @@ constexpr int kBarTmem = 2;
 constexpr int kBarUpdate2 = 3;
 constexpr int kBarUpdateAll = 4;
 constexpr int kBarSetup = 7;
+constexpr int kBarInit = 8;
 
 // Geometry and shared-memory layout of one GEMV configuration: weight type,
 // token count, shared-memory budget, x-ring depth SX, tensor-memory A and D
@@ -974,13 +975,22 @@ __global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kM
   if (n == 0) return;
 
   // The weight producer sets up the barriers and starts its ring at once; the
-  // other warps wait for the barriers and the tensor-memory address.
+  // x producer waits for the barriers only; the other warps also wait for the
+  // tensor-memory address.  (Counts: kBarInit 32 + 32, kBarSetup 32 + 32
+  // arriving + the rest waiting.)
   if (warp == kProducerWarp) {
     S.init(lane);
     __syncwarp();
+    named_arrive(kBarInit, 64);
     named_arrive(kBarSetup, C::kThreads);
     if (lane == 0 && !produce_weights<C>(a, S, cta, i0, n)) drain_inflight_copies();   // error path
     return;   // the producers take no part in the tensor-memory teardown
+  }
+  if (warp == C::kXWarp) {
+    named_sync(kBarInit, 64);
+    named_arrive(kBarSetup, C::kThreads);
+    if (!produce_x<C>(a, S, i0, n, lane) && lane == 0) drain_inflight_copies();   // error path
+    return;
   }
   if (warp == kMmaWarp) tmem_alloc(S.tslot, C::kTmemCols);
   tc_fence_before();
@@ -988,10 +998,6 @@ __global__ void __launch_bounds__(GemvCfg<QT, NT>::kThreads, GemvCfg<QT, NT>::kM
   tc_fence_after();
   const uint32_t tmem = *S.tslot;
 
-  if (warp == C::kXWarp) {
-    if (!produce_x<C>(a, S, i0, n, lane) && lane == 0) drain_inflight_copies();   // error path
-    return;
-  }
   bool ok = true;
   if (warp == kMmaWarp || warp == C::kMma2Warp) {
     if (lane == 0 && (warp == kMmaWarp || C::kMmaThreads == 2)) {
