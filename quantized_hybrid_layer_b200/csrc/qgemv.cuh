@@ -605,10 +605,10 @@ QHL_DEV void issue_x(const GemvArgs& a, const GemvSmem<C>& S, int chunk, uint32_
 
 // Producers of one stand-alone projection (K0 = 0), two threads in two warps
 // so that neither ring waits for the other's slots.  The weight thread keeps
-// the weight ring full: it requests the first two items, the rest of the
-// first ring once item 0 has landed (the weights never depend on earlier
-// kernels), and then each item as soon as its slot is released, sleeping in
-// the barrier wait in between.  The x thread does the
+// the weight ring full: it requests the first ring (beyond one token, the
+// first two items and the rest once item 0 has landed; the weights never
+// depend on earlier kernels), and then each item as soon as its slot is
+// released, sleeping in the barrier wait in between.  The x thread does the
 // same for the x ring (an item's block scales and x columns); the x columns
 // are written by the previous kernel, so they are requested only once
 // griddepcontrol.wait has returned.  Each returns false on a timeout.
@@ -619,9 +619,11 @@ QHL_DEV bool produce_weights(const GemvArgs& a, const GemvSmem<C>& S, int cta, i
   const uint64_t pol = policy_evict_first();
   for (int k = 0; k < n; ++k) {
     if (k >= SW && !mbar_wait(smem_u32(&S.wempty[k % SW]), ((k / SW) - 1) & 1u, a.err, a.wait_limit)) return false;
-    // the rest of the first ring only once the first item is in: the copies
-    // in flight share the SM's bandwidth, and the pipeline starts on item 0
-    if (k == 2 && n > 2 && !(cta == 0 && a.fault_item == 0) &&
+    // beyond one token (a twelve-item ring) the rest of the first ring only
+    // once the first item is in: the copies in flight share the SM's
+    // bandwidth, and the pipeline starts on item 0; the four-item ring of one
+    // token goes out at once
+    if (C::kNT > 1 && k == 2 && n > 2 && !(cta == 0 && a.fault_item == 0) &&
         !mbar_wait(smem_u32(&S.wfull[0]), 0u, a.err, a.wait_limit))
       return false;
     if (cta == 0 && k == a.fault_item) continue;   // injected failure: this slot never fills
