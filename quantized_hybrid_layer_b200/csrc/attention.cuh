@@ -130,20 +130,20 @@ QHL_DEV void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   lo = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
 }
 
-// The K and V fragments of one attention unit, held in registers.  Warp w
-// takes keys 16 (w % 4) .. +15 and dimensions 128 (w / 4) .. +127 for the
-// scores: k[i] (k[4 + i]) = the 8 dimensions 32 (4 (w / 4) + i) + 8t .. +7 of
-// key 16 (w % 4) + g (+ 8).  For the weighted sum it takes dimensions
-// 32w .. 32w + 31: v[(2 qq + ...)] = the dimension pair 16 (2w + qq) + 2g of keys
-// 16j + 2t + {0, 1, 8, 9}, at index (qq * 4 + j) * 4 + e.
+// The K and V fragments of one attention unit, held in registers (lane =
+// 4g + t).  For the scores warp w takes keys 16 (w % 4) .. +15 and dimensions
+// 128 (w / 4) .. +127: k[i] (k[4 + i]) holds the 8 dimensions
+// 32 (4 (w / 4) + i) + 8t .. +7 of key 16 (w % 4) + g (+ 8).  For the weighted
+// sum it takes dimensions 32w .. 32w + 31: v[(qq * 4 + j) * 4 + e] holds the
+// dimension pair 16 (2w + qq) + 2g, +1 of key 16j + 2t + (e % 2) + 8 (e / 2).
 struct AttnRegs {
   uint4 k[8];
   uint32_t v[32];
 };
 
 // Fill the fragments from cache rows of earlier passes (rows < pos) and zero
-// the rows past the last key the unit's tokens see; rows pos .. come from
-// attn_compute.  Needs nothing written by this pass, so a kernel issues it
+// the others; attn_compute then fills in this pass's rows that the unit's
+// tokens see.  Needs nothing written by this pass, so a kernel issues it
 // before waiting for the in-projection.
 QHL_DEV void attn_load_old(const AttnArgs& a, int c, int g, int pos, int ctx_end, AttnRegs& R) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gl = lane >> 2, tl = lane & 3;
@@ -171,7 +171,7 @@ QHL_DEV void attn_load_old(const AttnArgs& a, int c, int g, int pos, int ctx_end
                                      8 * (2 * warp + qq) + gl)
                         : 0u;
       }
-  (void)ctx_end;
+  (void)ctx_end;   // the unit's last visible row + 1 (rows from pos on come later)
 }
 
 // Byte offset of the 8-byte unit u of query row r in a [rows][256] f16 plane:
